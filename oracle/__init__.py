@@ -1,0 +1,6 @@
+"""CPU oracle for the SageSLA attention forward (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of ``bench.py`` may
+import this package. The product path never does.
+"""
+from .sagesla_oracle import *  # noqa: F401,F403

@@ -1,0 +1,259 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle function to a library routine, a brute-force evaluation on tiny
+inputs, an exact-arithmetic computation, a closed form, an invariant of the definition, or a
+fixture under tests/golden/ with its citation. Together they are chosen so that a dropped
+term, a wrong sign or index, or a transposed operand anywhere in the oracle fails one of them.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from sparse_bit_attention_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_head(n, seed, scale=1.0, k_offset=0.0):
+    q, k, v = inputs.make_random(1, 1, n, seed, k_offset_std=k_offset, scale=scale)
+    return inputs.as_float64(q[0, 0]), inputs.as_float64(k[0, 0]), inputs.as_float64(v[0, 0])
+
+
+def _sdpa64(q, k, v, mask=None):
+    """Dense softmax attention in float64 through torch's library routine."""
+    qt = torch.from_numpy(q)[None, None]
+    kt = torch.from_numpy(k)[None, None]
+    vt = torch.from_numpy(v)[None, None]
+    m = None if mask is None else torch.from_numpy(mask)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=m)[0, 0].numpy()
+
+
+# ---------------------------------------------------------------- number formats
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.integers(-6, 6, 20000),
+        rng.standard_normal(2000) * 1e-39,               # bf16 subnormal range
+        np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -1.0 - 2.0 ** -8, 0.0]),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(orc.round_bf16(x.astype(np.float64)), ref)
+
+
+def test_e4m3_rounding_matches_torch_in_range():
+    rng = np.random.default_rng(2)
+    x = np.concatenate([
+        rng.uniform(-463.0, 463.0, 20000),
+        rng.uniform(-0.02, 0.02, 20000),                 # subnormal and low normal range
+        orc.e4m3_decode(np.arange(0, 126)) * 1.0,       # grid points
+        (orc.e4m3_decode(np.arange(0, 125)) + orc.e4m3_decode(np.arange(1, 126))) / 2,  # ties
+    ]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn)
+    got = orc.round_e4m3(x.astype(np.float64))
+    np.testing.assert_array_equal(got, ref.to(torch.float64).numpy())
+    np.testing.assert_array_equal(orc.e4m3_code(got), ref.view(torch.uint8).numpy())
+
+
+def test_e4m3_golden_points():
+    path = os.path.join(GOLDEN, "e4m3_points.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    for xin, xout, code in rows:
+        got = orc.round_e4m3(np.array([float(xin)]))
+        assert got[0] == float(xout), (xin, got)
+        assert int(orc.e4m3_code(got)[0]) == int(code, 16), (xin, code)
+
+
+def test_e4m3_decode_table_matches_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = orc.e4m3_decode(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[fin], ref[fin])
+    # every finite pattern survives decode -> encode (the zero pattern 0x80 is -0.0)
+    np.testing.assert_array_equal(orc.e4m3_code(got[fin]), codes[fin])
+
+
+def test_int8_quantizer_round_trip_bound():
+    rng = np.random.default_rng(3)
+    for trial in range(50):
+        x = (rng.standard_normal((64, 128)) * 10.0 ** rng.uniform(-3, 3)).astype(np.float32)
+        codes, s = orc.quant_int8_block(x)
+        assert codes.dtype == np.int8 and np.abs(codes.astype(int)).max() == 127
+        err = np.abs(x.astype(np.float64) - float(s) * codes.astype(np.float64))
+        # half a step, plus the binary32 rounding of inv, of x*inv and of s
+        assert err.max() <= float(s) * (0.5 + 1e-5)
+    codes, s = orc.quant_int8_block(np.zeros((64, 128), np.float32))
+    assert s == 1.0 and not codes.any()
+
+
+def test_int8_quantizer_closed_form():
+    # integers with max 127: inv = 1 exactly, so the codes are the integers themselves
+    x = np.tile(np.arange(-127, 128, dtype=np.float32)[:128], (64, 1))
+    codes, s = orc.quant_int8_block(x)
+    assert s == 1.0
+    np.testing.assert_array_equal(codes.astype(np.float32), x)
+
+
+def test_v_fp8_quantizer_bound():
+    q, k, v = _rand_head(300, 4)
+    vals, s_v = orc.quant_v_fp8(v)
+    assert np.abs(vals).max() == 448.0
+    rec = vals * s_v.astype(np.float64)[None, :]
+    # e4m3 relative step 2^-3 for normals -> error <= 2^-4 relative (+ subnormal floor)
+    bound = np.abs(v) * 2.0 ** -4 + (2.0 ** -10) * s_v[None, :] + 1e-7 * np.abs(v)
+    assert np.all(np.abs(rec - v) <= bound)
+
+
+def test_smoothing_mean_exact_arithmetic():
+    q, k, v = _rand_head(777, 5, k_offset=1.5)
+    mu = orc.smoothing_mean(k)
+    for c in range(0, 128, 9):
+        exact = sum(Fraction(float(x)) for x in k[:, c]) / k.shape[0]
+        assert mu[c] == orc.round_bf16(np.array([float(exact)]))[0]
+        # the bf16 value is the nearest one to the exact mean
+        assert abs(Fraction(float(mu[c])) - exact) <= abs(Fraction(float(mu[c])) * 2 ** -8) + Fraction(1, 2 ** 140)
+
+
+# ---------------------------------------------------------------- blocks, Top-K
+
+def test_topk_counts_golden():
+    path = os.path.join(GOLDEN, "topk_counts.txt")
+    for line in open(path):
+        if not line.strip() or line.startswith("#"):
+            continue
+        n, nb, r, k = line.split()
+        assert orc.n_blocks(int(n)) == int(nb)
+        assert orc.topk_count(float(r), int(nb)) == int(k), line
+
+
+def test_topk_matches_bruteforce_sort_with_ties():
+    rng = np.random.default_rng(6)
+    for trial in range(200):
+        nb = int(rng.integers(1, 40))
+        k = int(rng.integers(1, nb + 1))
+        s = rng.integers(-5, 5, nb).astype(np.float64)          # many ties
+        brute = sorted(sorted(range(nb), key=lambda j: (-s[j], j))[:k])
+        assert list(orc.select_topk(s, k)) == brute
+
+
+def test_pooled_means_and_scores_bruteforce():
+    q, k, v = _rand_head(150, 7)                   # 3 blocks, last one 22 tokens
+    qb = orc.pooled_means(q)
+    assert qb.shape == (3, 128)
+    np.testing.assert_allclose(qb[2], np.array([sum(q[t, c] for t in range(128, 150)) / 22
+                                                for c in range(128)]), rtol=0, atol=1e-15)
+    s = orc.block_scores(qb, orc.pooled_means(k))
+    i, j = 2, 1
+    brute = sum(qb[i, c] * orc.pooled_means(k)[j, c] for c in range(128)) / math.sqrt(128)
+    assert abs(s[i, j] - brute) < 1e-15
+
+
+def test_margin_definition():
+    s = np.array([3.0, 1.0, 2.0, 2.0 - 1e-6])
+    assert orc.row_margin(s, 2) == pytest.approx((2.0 - (2.0 - 1e-6)) / 3.0)
+    assert orc.row_margin(s, 4) == math.inf
+
+
+# ---------------------------------------------------------------- the two branches
+
+@pytest.mark.parametrize("n", [256, 200, 64, 37])
+def test_dense_limit_equals_softmax_attention(n):
+    """r = 1 with quantization off: the complement is empty and the sparse branch is exact
+    softmax attention over all keys."""
+    q, k, v = _rand_head(n, 8)
+    prep, out = orc.forward_head(q, k, v, 1.0, quant=False)
+    o = np.concatenate([out[i]["o"] for i in range(prep.nb)])
+    assert all(not out[i]["o_l"].any() for i in range(prep.nb))
+    np.testing.assert_allclose(o, _sdpa64(q, k, v), rtol=0, atol=1e-10)
+
+
+def test_sparse_branch_equals_block_masked_attention():
+    """Quantization off, r < 1: the online block loop equals softmax attention restricted
+    to the kept blocks (a boolean block mask given to the library routine)."""
+    n = 300
+    q, k, v = _rand_head(n, 9)
+    prep, out = orc.forward_head(q, k, v, 0.4, quant=False)
+    mask = np.zeros((n, n), dtype=bool)
+    for i in range(prep.nb):
+        for j in prep.kept[i]:
+            mask[orc.block_rows(i, n), orc.block_rows(int(j), n)] = True
+    ref = _sdpa64(q, k, v, mask)
+    o_s = np.concatenate([out[i]["o_s"] for i in range(prep.nb)])
+    np.testing.assert_allclose(o_s, ref, rtol=0, atol=1e-10)
+    # the kept sets really are the top scores
+    for i in range(prep.nb):
+        brute = sorted(sorted(range(prep.nb), key=lambda j: (-prep.scores[i, j], j))[:prep.k])
+        assert list(prep.kept[i]) == brute
+
+
+def test_linear_branch_block_form_equals_per_token_definition():
+    n = 200
+    q, k, v = _rand_head(n, 10)
+    prep, out = orc.forward_head(q, k, v, 0.3, quant=True)
+    for i in range(prep.nb):
+        brute = orc.linear_block_row_bruteforce(prep, i, q, k, v)
+        np.testing.assert_allclose(out[i]["o_l"], brute, rtol=0, atol=1e-12)
+
+
+def test_smoothing_is_a_row_constant_shift():
+    n = 256
+    q, k, v = _rand_head(n, 11, k_offset=2.0)
+    _, a = orc.forward_head(q, k, v, 0.5, quant=False)
+    _, b = orc.forward_head(q, k, v, 0.5, quant=False, smooth_in_quant_off=True)
+    for i in a:
+        np.testing.assert_allclose(a[i]["o"], b[i]["o"], rtol=0, atol=1e-12)
+
+
+def test_constant_v():
+    n = 256
+    q, k, _ = _rand_head(n, 12)
+    c = np.linspace(-2.0, 2.0, 128)
+    v = np.tile(orc.round_bf16(c), (n, 1))
+    prep, out = orc.forward_head(q, k, v, 0.25, quant=False)
+    for i in out:
+        np.testing.assert_allclose(out[i]["o"], 2 * v[: out[i]["o"].shape[0]], atol=1e-12)
+    prep, out = orc.forward_head(q, k, v, 0.25, quant=True)
+    for i in out:
+        vv = v[: out[i]["o"].shape[0]]
+        np.testing.assert_allclose(out[i]["o_l"], vv, atol=1e-12)
+        # sparse branch: each P entry is off by at most 2^-4 relative after e4m3 rounding
+        assert np.all(np.abs(out[i]["o_s"] - vv) <= np.abs(vv) * 2.0 ** -4 + 1e-6)
+
+
+def test_single_block_is_dense_attention():
+    q, k, v = _rand_head(50, 13)
+    prep, out = orc.forward_head(q, k, v, 0.1, quant=False)
+    assert prep.nb == 1 and prep.k == 1
+    assert not out[0]["o_l"].any()
+    np.testing.assert_allclose(out[0]["o"], _sdpa64(q, k, v), atol=1e-10)
+
+
+def test_quantized_scores_are_integer_exact():
+    n = 128
+    q, k, v = _rand_head(n, 14, k_offset=1.0)
+    prep = orc.prepare_head(q, k, v, 1.0)
+    for t, u in [(0, 0), (5, 77), (63, 127), (100, 3)]:
+        brute = sum(int(prep.q8[t, c]) * int(prep.k8[u, c]) for c in range(128))
+        assert float(prep.q8[t].astype(np.float64) @ prep.k8[u].astype(np.float64)) == brute
+    # K smoothing: codes dequantize to k - mu within half a step
+    ks = k - prep.mu[None, :]
+    for j in range(prep.nb):
+        r = orc.block_rows(j, n)
+        assert np.abs(ks[r] - float(prep.sk[j]) * prep.k8[r]).max() <= float(prep.sk[j]) * 0.5001
+
+
+def test_quantized_forward_is_close_to_exact():
+    """Quantization is a small perturbation: INT8/FP8 output within a few 1e-2 of the
+    quantization-off output on the tiny workload's distribution."""
+    q, k, v = _rand_head(512, 15, k_offset=math.sqrt(2.0))
+    _, a = orc.forward_head(q, k, v, 0.25, quant=True)
+    _, b = orc.forward_head(q, k, v, 0.25, quant=False)
+    err = max(np.abs(a[i]["o"] - b[i]["o"]).max() for i in a)
+    assert 1e-4 < err < 0.08

@@ -1,0 +1,161 @@
+/*
+ * sagesla.h — C ABI of the B200 (sm_100a) SageSLA attention forward.
+ *
+ * SageSLA is the attention of the TurboDiffusion video diffusion transformer: sparse-linear
+ * attention (SLA) combined with SageAttention-style low-bit quantization
+ * (news.qq.com TurboDiffusion article, section 第一把钥匙; dgmzs.com.cn README translation,
+ * section 方法论). Per (batch, head), with 64-token blocks:
+ *   1. block scores s_ij = mean(Q_i) . mean(K_j) / sqrt(128); each query block keeps the
+ *      k = clamp(ceil(r*nb - 1e-9), 1, nb) highest-scoring key blocks, ties to the lower j
+ *      (same article, 第一把钥匙: Top-K ratio 0.1; 从训练到部署: 0.1-0.15);
+ *   2. K is smoothed by its bf16-rounded channel mean; Q and smoothed K are quantized to
+ *      INT8 with one scale per 64-token block, V to FP8 e4m3 with one scale per channel
+ *      (same article, 第一把钥匙 and 第三把钥匙);
+ *   3. sparse branch: online softmax over the kept blocks in ascending order, INT8 Q.K^T,
+ *      P in e4m3 with scale 1/448, FP8 P.V;
+ *   4. linear branch over the key blocks not kept: phi(q)(sum phi(k)^T [v|1]) normalized,
+ *      phi = softmax over the 128 channels;
+ *   5. out = sparse branch + linear branch.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are CUDA device addresses of the current device. The caller owns all
+ *     buffers (inputs, output, workspace) and the stream; the library never allocates,
+ *     frees or synchronizes except where stated.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream) unless stated; a return of SAGESLA_OK means the work was enqueued.
+ *   - No exception crosses the ABI. Arguments are validated before anything is launched.
+ *   - Errors detected on the device (a wait that timed out) are recorded in a status word in
+ *     the workspace and read back by sagesla_stream_status().
+ *   - Re-entrant across streams provided each concurrent call has its own workspace.
+ */
+#ifndef SAGESLA_H_
+#define SAGESLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGESLA_OK = 0,
+  SAGESLA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape/stride/ratio, aliasing output */
+  SAGESLA_ERR_UNSUPPORTED = 2,  /* D != 128, block != 64, dtype not supported */
+  SAGESLA_ERR_WORKSPACE = 3,    /* workspace missing, too small or misaligned */
+  SAGESLA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  SAGESLA_ERR_TIMEOUT = 5,      /* a device-side wait exceeded its limit (see stream_status) */
+  SAGESLA_ERR_DEVICE_CHECK = 6, /* a device-side consistency check failed */
+  SAGESLA_ERR_NO_DEVICE = 7     /* no sm_100 device is current */
+} sagesla_status;
+
+typedef enum { SAGESLA_BF16 = 0, SAGESLA_F32 = 1 } sagesla_dtype;
+
+/* A [B, H, N, D] tensor view. Strides are in elements; the D axis is contiguous (stride 1).
+ * Every row (b, h, n) must start on a 16-byte boundary. */
+typedef struct {
+  void* data;
+  int32_t dtype; /* sagesla_dtype */
+  int64_t B, H, N, D;
+  int64_t stride_b, stride_h, stride_n;
+} sagesla_tensor;
+
+/* Optional extra outputs of sagesla_forward_ex (device pointers, may be NULL):
+ *   kept_idx_out [B*H][nb][k] int32: kept key blocks of each query block, ascending;
+ *   mask_out     [B*H][nb][ceil(nb/32)] uint32: bit j%32 of word j/32 set if j is kept;
+ *   scores_out   [B*H][nb][nb] float: the block scores s_ij;
+ *   sparse_out   [B*H][N][128] float: the sparse branch o*s_v/(448 l) before the linear
+ *                branch is added. */
+typedef struct {
+  int32_t* kept_idx_out;
+  uint32_t* mask_out;
+  float* scores_out;
+  float* sparse_out;   /* [B*H][N][128] float: the sparse-branch output alone */
+} sagesla_options;
+
+/* Offsets (bytes, from the workspace start) of the intermediates a forward call leaves in
+ * its workspace, for inspection after the stream has completed. Per-head arrays are
+ * contiguous over B*H; n_pad = 128*ceil(nb/2) token rows per head. */
+typedef struct {
+  size_t total_bytes;
+  int64_t nb, k, n_pad, mask_words, nb_k_pad, nb_m_pad;
+  size_t status;      /* int32 status word */
+  size_t q8, k8;      /* int8  [B*H][n_pad][128] codes (zero rows past N) */
+  size_t v8;          /* uint8 [B*H][n_pad][128] e4m3 codes */
+  size_t sq, sk;      /* float [B*H][2*ceil(nb/2)] per-block scales */
+  size_t s_v;         /* float [B*H][128] per-channel V scale */
+  size_t inv_v;       /* float [B*H][128] 448 / channel amax */
+  size_t mu;          /* float [B*H][128] bf16 channel mean of K, stored as float */
+  size_t qbar, kbar;  /* float [B*H][nb][128] block means */
+  size_t ksum_part;   /* double [B*H][nb][128] per-block K channel sums */
+  size_t vmax_part;   /* float [B*H][nb][128] per-block V channel amax */
+  size_t scores;      /* float [B*H][nb][nb] raw block dot products */
+  size_t kept;        /* int32 [B*H][nb][k] */
+  size_t mask;        /* uint32 [B*H][nb][mask_words] */
+  size_t amask;       /* bf16 [B*H][nb_m_pad][nb_k_pad] complement mask (1 = not kept) */
+  size_t hflat;       /* bf16 [B*H][nb_k_pad][129*128] key-block states H_j as [n][c] */
+  size_t gsum;        /* bf16 [B*H][nb_m_pad][129*128] complement sums G_i as [n][c] */
+} sagesla_workspace_layout;
+
+/* Human-readable name of a status code (static string). */
+const char* sagesla_status_string(sagesla_status status);
+
+/* k, the number of key blocks each query block keeps, for N tokens and ratio r (block 64):
+ * clamp(ceil(r*ceil(N/64) - 1e-9), 1, ceil(N/64)); -1 for invalid arguments. */
+int64_t sagesla_topk_count(int64_t N, double topk_ratio, int block);
+
+/* Bytes of device workspace sagesla_forward needs; 0 for invalid arguments. */
+size_t sagesla_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, double topk_ratio,
+                              int block);
+
+/* Fills *layout for the given problem. Returns SAGESLA_ERR_INVALID_ARG / SAGESLA_ERR_UNSUPPORTED on bad
+ * arguments. Host only, no CUDA call. */
+sagesla_status sagesla_get_workspace_layout(int64_t B, int64_t H, int64_t N, int64_t D,
+                                            double topk_ratio, int block,
+                                            sagesla_workspace_layout* layout);
+
+/* The SageSLA forward: out = sparse(Q,K,V) + linear(Q,K,V) as defined above.
+ *   q, k, v   : bf16 [B,H,N,128] device tensors (read only)
+ *   topk_ratio: r in (0, 1]
+ *   block     : must be 64
+ *   out       : bf16 or f32 [B,H,N,128] device tensor, must not overlap q, k, v or workspace
+ *   workspace : device buffer of at least sagesla_workspace_size() bytes, 256-byte aligned;
+ *               its contents on entry are ignored; it holds the intermediates on exit
+ *   stream    : cudaStream_t as void*
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, NO_DEVICE (nothing launched). */
+sagesla_status sagesla_forward(const sagesla_tensor* q, const sagesla_tensor* k,
+                               const sagesla_tensor* v, double topk_ratio, int block,
+                               sagesla_tensor* out, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* As sagesla_forward, plus the optional outputs of *opt (opt may be NULL). */
+sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor* k,
+                                  const sagesla_tensor* v, double topk_ratio, int block,
+                                  sagesla_tensor* out, void* workspace, size_t workspace_bytes,
+                                  void* stream, const sagesla_options* opt);
+
+/* Bytes of device workspace sagesla_forward_host needs (the forward workspace plus device
+ * copies of Q, K, V and the output); 0 for invalid arguments. */
+size_t sagesla_host_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
+                                   double topk_ratio, int block, int32_t out_dtype);
+
+/* Forward on HOST buffers: contiguous [B,H,N,128] bf16 inputs (uint16 bit patterns) and a
+ * contiguous bf16/f32 output in host memory (page-locked memory gives asynchronous copies).
+ * Copies the inputs into `workspace`, runs the forward there, copies the output back and
+ * synchronizes `stream` before returning. Also returns device-side errors (TIMEOUT). */
+sagesla_status sagesla_forward_host(const uint16_t* q_host, const uint16_t* k_host,
+                                    const uint16_t* v_host, int64_t B, int64_t H, int64_t N,
+                                    int64_t D, double topk_ratio, int block, void* out_host,
+                                    int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* Synchronizes `stream`, then reads and clears the device status word of `workspace`
+ * (the one used by the last forward on that workspace). Returns SAGESLA_OK, TIMEOUT,
+ * DEVICE_CHECK, or CUDA if the stream reported an error. */
+sagesla_status sagesla_stream_status(void* stream, void* workspace);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGESLA_H_ */

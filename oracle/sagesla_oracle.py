@@ -232,8 +232,9 @@ class HeadPrep:
     qbar: np.ndarray
     kbar: np.ndarray
     scores: np.ndarray
-    kept: list
+    kept: list                          # blocks the branches use (selected, or the override)
     margin: np.ndarray
+    selected: list | None = None        # the oracle's own Top-K selection
     mu: np.ndarray | None = None
     q8: np.ndarray | None = None       # int8 codes [N, D]
     sq: np.ndarray | None = None       # float32 [nb]
@@ -256,11 +257,12 @@ def prepare_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, topk_ratio: float,
     qbar, kbar = pooled_means(q), pooled_means(k)
     scores = block_scores(qbar, kbar)
     kept = [select_topk(scores[i], kk) for i in range(nb)]
+    selected = kept
     if kept_override is not None:
         kept = [np.asarray(kept_override[i], dtype=np.int64) for i in range(nb)]
     margin = np.array([row_margin(scores[i], kk) for i in range(nb)])
     prep = HeadPrep(n=n, nb=nb, k=kk, qbar=qbar, kbar=kbar, scores=scores, kept=kept,
-                    margin=margin)
+                    margin=margin, selected=selected)
     if quant:
         prep.mu = smoothing_mean(k)
         ks = (f32(k) - f32(prep.mu)[None, :]).astype(np.float32)

@@ -1,0 +1,8 @@
+"""B200-native SageSLA attention forward: a C-ABI CUDA library (libsagesla.so, sm_100a) and
+its thin Python binding. See include/sagesla.h for the ABI."""
+from .binding import (  # noqa: F401
+    SAGESLA_BF16, SAGESLA_F32, SageslaError, alloc_workspace, load_library,
+    sagesla_forward, sagesla_forward_host, sagesla_get_workspace_layout,
+    sagesla_host_workspace_size, sagesla_status_string, sagesla_stream_status,
+    sagesla_topk_count, sagesla_workspace_size,
+)

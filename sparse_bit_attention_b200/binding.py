@@ -1,0 +1,215 @@
+"""Thin ctypes binding of libsagesla.so: the same entry points as include/sagesla.h.
+
+Argument marshalling only — every step of the forward runs in the library's CUDA kernels.
+PyTorch provides device memory and streams. There is no fallback: if the library is missing
+or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsagesla.so")
+
+SAGESLA_BF16 = 0
+SAGESLA_F32 = 1
+BLOCK = 64
+HEAD_DIM = 128
+
+STATUS_NAMES = {
+    0: "SAGESLA_OK", 1: "SAGESLA_ERR_INVALID_ARG", 2: "SAGESLA_ERR_UNSUPPORTED",
+    3: "SAGESLA_ERR_WORKSPACE", 4: "SAGESLA_ERR_CUDA", 5: "SAGESLA_ERR_TIMEOUT",
+    6: "SAGESLA_ERR_DEVICE_CHECK", 7: "SAGESLA_ERR_NO_DEVICE",
+}
+
+
+class SageslaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} "
+                         f"({sagesla_status_string(status)})")
+
+
+class SageslaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32),
+                ("B", ctypes.c_int64), ("H", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("D", ctypes.c_int64), ("stride_b", ctypes.c_int64),
+                ("stride_h", ctypes.c_int64), ("stride_n", ctypes.c_int64)]
+
+
+class SageslaOptions(ctypes.Structure):
+    _fields_ = [("kept_idx_out", ctypes.c_void_p), ("mask_out", ctypes.c_void_p),
+                ("scores_out", ctypes.c_void_p), ("sparse_out", ctypes.c_void_p)]
+
+
+_LAYOUT_FIELDS = ["status", "q8", "k8", "v8", "sq", "sk", "s_v", "inv_v", "mu", "qbar", "kbar",
+                  "ksum_part", "vmax_part", "scores", "kept", "mask", "amask", "hflat", "gsum"]
+
+
+class SageslaWorkspaceLayout(ctypes.Structure):
+    _fields_ = ([("total_bytes", ctypes.c_size_t)] +
+                [(n, ctypes.c_int64) for n in
+                 ("nb", "k", "n_pad", "mask_words", "nb_k_pad", "nb_m_pad")] +
+                [(n, ctypes.c_size_t) for n in _LAYOUT_FIELDS])
+
+
+# Every symbol the header declares, with its signature.
+_SIGNATURES = {
+    "sagesla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "sagesla_topk_count": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_double, ctypes.c_int]),
+    "sagesla_workspace_size": (ctypes.c_size_t, [ctypes.c_int64] * 4 + [ctypes.c_double, ctypes.c_int]),
+    "sagesla_get_workspace_layout": (ctypes.c_int, [ctypes.c_int64] * 4 + [
+        ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaWorkspaceLayout)]),
+    "sagesla_forward": (ctypes.c_int, [ctypes.POINTER(SageslaTensor)] * 3 + [
+        ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaTensor), ctypes.c_void_p,
+        ctypes.c_size_t, ctypes.c_void_p]),
+    "sagesla_forward_ex": (ctypes.c_int, [ctypes.POINTER(SageslaTensor)] * 3 + [
+        ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaTensor), ctypes.c_void_p,
+        ctypes.c_size_t, ctypes.c_void_p, ctypes.POINTER(SageslaOptions)]),
+    "sagesla_host_workspace_size": (ctypes.c_size_t, [ctypes.c_int64] * 4 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_int32]),
+    "sagesla_forward_host": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 4 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+        ctypes.c_size_t, ctypes.c_void_p]),
+    "sagesla_stream_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+}
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libsagesla.so (built by ``python -m sparse_bit_attention_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m sparse_bit_attention_b200.build` (there is no fallback)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIGNATURES)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SageslaError(status, where)
+
+
+def _view(t: torch.Tensor) -> SageslaTensor:
+    if t.dim() != 4:
+        raise ValueError("expected a [B, H, N, D] tensor")
+    if t.stride(3) != 1:
+        raise ValueError("the head dimension must be contiguous")
+    dt = {torch.bfloat16: SAGESLA_BF16, torch.float32: SAGESLA_F32}.get(t.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    B, H, N, D = t.shape
+    return SageslaTensor(t.data_ptr(), dt, B, H, N, D, t.stride(0), t.stride(1), t.stride(2))
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def sagesla_status_string(status: int) -> str:
+    return load_library().sagesla_status_string(int(status)).decode()
+
+
+def sagesla_topk_count(N: int, topk_ratio: float, block: int = BLOCK) -> int:
+    return int(load_library().sagesla_topk_count(N, float(topk_ratio), block))
+
+
+def sagesla_workspace_size(B: int, H: int, N: int, D: int = HEAD_DIM, topk_ratio: float = 0.1,
+                           block: int = BLOCK) -> int:
+    return int(load_library().sagesla_workspace_size(B, H, N, D, float(topk_ratio), block))
+
+
+def sagesla_get_workspace_layout(B: int, H: int, N: int, D: int = HEAD_DIM,
+                                 topk_ratio: float = 0.1, block: int = BLOCK) -> dict:
+    lay = SageslaWorkspaceLayout()
+    _check(load_library().sagesla_get_workspace_layout(B, H, N, D, float(topk_ratio), block,
+                                                       ctypes.byref(lay)),
+           "sagesla_get_workspace_layout")
+    return {name: getattr(lay, name) for name, _ in SageslaWorkspaceLayout._fields_}
+
+
+def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A device byte buffer for the workspace (the caching allocator returns 512-byte-aligned
+    blocks, above the library's 256-byte requirement)."""
+    ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device or "cuda")
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_ratio: float = 0.1,
+                    block: int = BLOCK, out: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream=None,
+                    out_dtype: torch.dtype = torch.float32, kept_idx_out=None, mask_out=None,
+                    scores_out=None, sparse_out=None) -> torch.Tensor:
+    """SageSLA forward on device tensors q, k, v (bf16 [B, H, N, 128]); returns ``out``."""
+    lib = load_library()
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    B, H, N, D = q.shape
+    need = sagesla_workspace_size(B, H, N, D, topk_ratio, block)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
+    extra = (kept_idx_out, mask_out, scores_out, sparse_out)
+    args = (ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), float(topk_ratio), int(block),
+            ctypes.byref(vo), ctypes.c_void_p(workspace.data_ptr()),
+            workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_ptr(stream)))
+    if any(x is not None for x in extra):
+        opt = SageslaOptions(*[None if x is None else x.data_ptr() for x in extra])
+        _check(lib.sagesla_forward_ex(*args, ctypes.byref(opt)), "sagesla_forward_ex")
+    else:
+        _check(lib.sagesla_forward(*args), "sagesla_forward")
+    return out
+
+
+def sagesla_host_workspace_size(B: int, H: int, N: int, D: int = HEAD_DIM,
+                                topk_ratio: float = 0.1, block: int = BLOCK,
+                                out_dtype: int = SAGESLA_F32) -> int:
+    return int(load_library().sagesla_host_workspace_size(B, H, N, D, float(topk_ratio), block,
+                                                          int(out_dtype)))
+
+
+def sagesla_forward_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+                         out_host: torch.Tensor, topk_ratio: float = 0.1, block: int = BLOCK,
+                         workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Forward on contiguous CPU tensors (pinned memory gives asynchronous copies): copies in,
+    runs, copies out and synchronizes the stream."""
+    lib = load_library()
+    for t in (q_host, k_host, v_host, out_host):
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError("host tensors must be contiguous CPU tensors")
+    B, H, N, D = q_host.shape
+    odt = SAGESLA_F32 if out_host.dtype == torch.float32 else SAGESLA_BF16
+    need = sagesla_host_workspace_size(B, H, N, D, topk_ratio, block, odt)
+    if workspace is None:
+        workspace = alloc_workspace(need)
+    _check(lib.sagesla_forward_host(
+        ctypes.c_void_p(q_host.data_ptr()), ctypes.c_void_p(k_host.data_ptr()),
+        ctypes.c_void_p(v_host.data_ptr()), B, H, N, D, float(topk_ratio), int(block),
+        ctypes.c_void_p(out_host.data_ptr()), odt, ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel(), ctypes.c_void_p(_stream_ptr(stream))), "sagesla_forward_host")
+    return out_host
+
+
+def sagesla_stream_status(stream=None, workspace: torch.Tensor | None = None) -> int:
+    """Synchronizes the stream and returns (and clears) the workspace's device status word."""
+    wp = None if workspace is None else ctypes.c_void_p(workspace.data_ptr())
+    return int(load_library().sagesla_stream_status(ctypes.c_void_p(_stream_ptr(stream)), wp))

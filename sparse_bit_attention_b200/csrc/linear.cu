@@ -1,0 +1,147 @@
+// Linear branch, step 1: the complement sums G_i = sum over key blocks j NOT kept by query
+// block i of H_j (H_j = phi(K_j)^T [V_j | 1], built by k_stats).
+//
+// "Sparse-Linear Attention" (dgmzs.com.cn README translation, section 方法论; bonega.ai
+// article, section "SLA: Sparse-Linear Attention"): the blocks the sparse branch skips are
+// covered by linear attention. Per head this is one dense GEMM
+//     G[nb x 16512] = (1 - M)[nb x nb] . Hflat[nb x 16512]
+// with the binary complement mask as the A operand (exact in bf16). It runs on tcgen05:
+// 128 x 256 output tiles, 64-deep K steps, a 3-stage TMA pipeline (A K-major, B MN-major, both
+// 128-byte swizzled), one MMA-issuing thread, fp32 accumulation in TMEM and a bf16 epilogue.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sagesla {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kTileM = 128, kTileN = 256, kTileK = 64;
+constexpr uint32_t kABytes = kTileM * kTileK * 2;   // 16 KB
+constexpr uint32_t kBBytes = kTileK * kTileN * 2;   // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kGemmSmem = kStages * kStageBytes + 1024 + 256;
+
+__global__ void __launch_bounds__(192, 1)
+k_complement_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                  int nb_m_pad, int nb_k_pad, __nv_bfloat16* __restrict__ gsum, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* done = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f0 = blockIdx.x * kTileN;
+  const int m0 = blockIdx.y * kTileM;
+  const int64_t bh = blockIdx.z;
+  const int nkt = nb_k_pad / kTileK;
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 128 + 32) { prefetch_tmap(&tm_a); prefetch_tmap(&tm_b); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4 && lane == 0) {   // TMA producer
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int s = kt % kStages;
+      if (kt >= kStages && !mbar_wait(&empty[s], ((kt / kStages) - 1) & 1, status)) break;
+      uint8_t* a = smem + s * kStageBytes;
+      uint8_t* b = a + kABytes;
+      mbar_arrive_expect_tx(&full[s], kStageBytes);
+      tma_load_2d(a, &tm_a, &full[s], kt * kTileK, static_cast<int>(bh * nb_m_pad + m0));
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tma_load_2d(b + q * 8192, &tm_b, &full[s], f0 + 64 * q,
+                    static_cast<int>(bh * nb_k_pad + kt * kTileK));
+    }
+  } else if (warp == 5 && lane == 0) {   // MMA issuer
+    constexpr uint32_t idesc = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 1, kTileM, kTileN);
+    bool ok = true;
+    for (int kt = 0; kt < nkt && ok; ++kt) {
+      const int s = kt % kStages;
+      ok = mbar_wait(&full[s], (kt / kStages) & 1, status);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t a = smem_u32(smem + s * kStageBytes);
+      const uint32_t b = a + kABytes;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {   // 4 x K=16
+        const uint64_t ad = make_sdesc(a + kk * 32, 16, 1024, kLayoutSW128);
+        const uint64_t bd = make_sdesc(b + kk * 2048, 8192, 1024, kLayoutSW128);
+        mma_bf16(tmem, ad, bd, idesc, (kt | kk) ? 1u : 0u);
+      }
+      mma_commit(&empty[s]);
+    }
+    mma_commit(done);
+  } else if (warp < 4) {   // epilogue: TMEM -> bf16 -> global
+    const bool ok = mbar_wait(done, 0, status);
+    tc_fence_after();
+    if (ok) {
+      const int64_t row = bh * nb_m_pad + m0 + 32 * warp + lane;
+      __nv_bfloat16* grow = gsum + row * static_cast<int64_t>(kHFlat);
+#pragma unroll 1
+      for (int cc = 0; cc < kTileN / 32; ++cc) {
+        const int f = f0 + 32 * cc;
+        if (f >= kHFlat) break;   // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(tmem_addr(tmem, 32 * warp, 32 * cc), r);
+        tmem_ld_wait();
+        uint32_t packed[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]),
+                                                    __uint_as_float(r[2 * e + 1]));
+          packed[e] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(grow + f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+}  // namespace
+
+cudaError_t launch_complement_gemm(const ForwardPlan& p, char* ws, cudaStream_t stream) {
+  const auto& L = p.lay;
+  CUtensorMap ta, tb;
+  if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.nb_k_pad, p.BH * p.nb_m_pad,
+                      p.nb_k_pad * 2, ws + L.amask, kTileK, kTileM,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHFlat, p.BH * p.nb_k_pad,
+                      static_cast<uint64_t>(kHFlat) * 2, ws + L.hflat, 64, kTileK,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k_complement_gemm,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((kHFlat + kTileN - 1) / kTileN, static_cast<unsigned>(p.nb_m_pad / kTileM),
+            static_cast<unsigned>(p.BH));
+  k_complement_gemm<<<grid, 192, kGemmSmem, stream>>>(
+      ta, tb, static_cast<int>(p.nb_m_pad), static_cast<int>(p.nb_k_pad),
+      reinterpret_cast<__nv_bfloat16*>(ws + L.gsum), reinterpret_cast<int*>(ws + L.status));
+  return cudaGetLastError();
+}
+
+}  // namespace sagesla

@@ -1,0 +1,359 @@
+// Host side of the C ABI: argument validation, the workspace plan, tensor-map encoding and
+// the launch sequence of one SageSLA forward. No allocation, no synchronization (except in
+// sagesla_forward_host and sagesla_stream_status, which say so).
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sagesla {
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool valid_ratio(double r) { return std::isfinite(r) && r > 0.0 && r <= 1.0; }
+
+int64_t topk_count(int64_t nb, double r) {
+  int64_t k = static_cast<int64_t>(std::ceil(r * static_cast<double>(nb) - 1e-9));
+  if (k < 1) k = 1;
+  if (k > nb) k = nb;
+  return k;
+}
+
+// Problem-size limits of this implementation.
+constexpr int64_t kMaxBH = 65535;              // grid.y
+constexpr int64_t kMaxBlocks = 1 << 15;        // score row must fit in shared memory
+constexpr size_t kMaxListSmem = 120 * 1024;    // kept-list union in the attention kernel
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+}  // namespace
+
+bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* p) {
+  if (B < 1 || H < 1 || N < 1 || !valid_ratio(topk_ratio)) return false;
+  std::memset(p, 0, sizeof(*p));
+  p->B = B;
+  p->H = H;
+  p->N = N;
+  p->BH = B * H;
+  p->nb = ceil_div(N, kBlock);
+  p->k = topk_count(p->nb, topk_ratio);
+  p->n_pairs = ceil_div(p->nb, 2);
+  p->n_pad = 128 * p->n_pairs;
+  p->mask_words = ceil_div(p->nb, 32);
+  p->nb_k_pad = ceil_div(p->nb, 64) * 64;
+  p->nb_m_pad = ceil_div(p->nb, 128) * 128;
+  p->n_last = static_cast<int32_t>(N - kBlock * (p->nb - 1));
+  p->linear_empty = p->k == p->nb;
+  if (p->BH > kMaxBH || p->nb > kMaxBlocks) return false;
+  if (static_cast<size_t>(p->nb < 2 * p->k ? p->nb : 2 * p->k) * 8 > kMaxListSmem) return false;
+  if (p->BH * p->nb_m_pad * 129 >= (int64_t(1) << 31) || p->BH * p->n_pad >= (int64_t(1) << 31))
+    return false;
+
+  sagesla_workspace_layout& L = p->lay;
+  const int64_t BH = p->BH, nb = p->nb, nbq = 2 * p->n_pairs;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  L.nb = nb;
+  L.k = p->k;
+  L.n_pad = p->n_pad;
+  L.mask_words = p->mask_words;
+  L.nb_k_pad = p->nb_k_pad;
+  L.nb_m_pad = p->nb_m_pad;
+  L.status = take(sizeof(int32_t));
+  L.q8 = take(static_cast<size_t>(BH * p->n_pad * 128));
+  L.k8 = take(static_cast<size_t>(BH * p->n_pad * 128));
+  L.v8 = take(static_cast<size_t>(BH * p->n_pad * 128));
+  L.sq = take(static_cast<size_t>(BH * nbq) * 4);
+  L.sk = take(static_cast<size_t>(BH * nbq) * 4);
+  L.s_v = take(static_cast<size_t>(BH * 128) * 4);
+  L.inv_v = take(static_cast<size_t>(BH * 128) * 4);
+  L.mu = take(static_cast<size_t>(BH * 128) * 4);
+  L.qbar = take(static_cast<size_t>(BH * nb * 128) * 4);
+  L.kbar = take(static_cast<size_t>(BH * nb * 128) * 4);
+  L.ksum_part = take(static_cast<size_t>(BH * nb * 128) * 8);
+  L.vmax_part = take(static_cast<size_t>(BH * nb * 128) * 4);
+  L.scores = take(static_cast<size_t>(BH * nb * nb) * 4);
+  L.kept = take(static_cast<size_t>(BH * nb * p->k) * 4);
+  L.mask = take(static_cast<size_t>(BH * nb * p->mask_words) * 4);
+  L.amask = take(static_cast<size_t>(BH * p->nb_m_pad * p->nb_k_pad) * 2);
+  L.hflat = take(static_cast<size_t>(BH * p->nb_k_pad) * kHFlat * 2);
+  L.gsum = take(static_cast<size_t>(BH * p->nb_m_pad) * kHFlat * 2);
+  L.total_bytes = off;
+  return true;
+}
+
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, const void* base, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+size_t elem_bytes(int32_t dtype) { return dtype == SAGESLA_F32 ? 4 : 2; }
+
+// Byte range [lo, hi) touched by a tensor view.
+void extent(const sagesla_tensor* t, uintptr_t* lo, uintptr_t* hi) {
+  const size_t eb = elem_bytes(t->dtype);
+  const int64_t last = (t->B - 1) * t->stride_b + (t->H - 1) * t->stride_h +
+                       (t->N - 1) * t->stride_n + t->D;
+  *lo = reinterpret_cast<uintptr_t>(t->data);
+  *hi = *lo + static_cast<uintptr_t>(last) * eb;
+}
+
+bool overlaps(uintptr_t a0, uintptr_t a1, uintptr_t b0, uintptr_t b1) {
+  return a0 < b1 && b0 < a1;
+}
+
+sagesla_status check_view(const sagesla_tensor* t, const sagesla_tensor* ref, bool is_out) {
+  if (!t || !t->data) return SAGESLA_ERR_INVALID_ARG;
+  if (t->D != kHeadDim) return SAGESLA_ERR_UNSUPPORTED;
+  if (is_out ? (t->dtype != SAGESLA_BF16 && t->dtype != SAGESLA_F32) : t->dtype != SAGESLA_BF16)
+    return SAGESLA_ERR_UNSUPPORTED;
+  if (t->B < 1 || t->H < 1 || t->N < 1) return SAGESLA_ERR_INVALID_ARG;
+  if (ref && (t->B != ref->B || t->H != ref->H || t->N != ref->N)) return SAGESLA_ERR_INVALID_ARG;
+  const int64_t eb = static_cast<int64_t>(elem_bytes(t->dtype));
+  if (t->stride_n < t->D || t->stride_h < 0 || t->stride_b < 0) return SAGESLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(t->data) & 15) != 0 || (t->stride_n * eb) % 16 != 0 ||
+      (t->stride_h * eb) % 16 != 0 || (t->stride_b * eb) % 16 != 0)
+    return SAGESLA_ERR_INVALID_ARG;
+  return SAGESLA_OK;
+}
+
+TensorArg to_arg(const sagesla_tensor* t) {
+  TensorArg a;
+  a.data = t->data;
+  a.stride_b = t->stride_b;
+  a.stride_h = t->stride_h;
+  a.stride_n = t->stride_n;
+  a.H = static_cast<int32_t>(t->H);
+  return a;
+}
+
+// The current device must be a compute-capability-10.0 part (B200).
+sagesla_status check_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGESLA_ERR_NO_DEVICE;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return SAGESLA_ERR_NO_DEVICE;
+  if (major != 10 || minor != 0) return SAGESLA_ERR_NO_DEVICE;
+  return SAGESLA_OK;
+}
+
+#define SAGESLA_LAUNCH(call)                            \
+  do {                                                  \
+    if ((call) != cudaSuccess) return SAGESLA_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+}  // namespace sagesla
+
+using namespace sagesla;
+
+extern "C" {
+
+const char* sagesla_status_string(sagesla_status s) {
+  switch (s) {
+    case SAGESLA_OK: return "ok";
+    case SAGESLA_ERR_INVALID_ARG: return "invalid argument";
+    case SAGESLA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case SAGESLA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case SAGESLA_ERR_CUDA: return "CUDA error";
+    case SAGESLA_ERR_TIMEOUT: return "device-side wait timed out";
+    case SAGESLA_ERR_DEVICE_CHECK: return "device-side check failed";
+    case SAGESLA_ERR_NO_DEVICE: return "no sm_100 device current";
+  }
+  return "unknown status";
+}
+
+int64_t sagesla_topk_count(int64_t N, double topk_ratio, int block) {
+  if (N < 1 || block != kBlock || !valid_ratio(topk_ratio)) return -1;
+  return topk_count(ceil_div(N, kBlock), topk_ratio);
+}
+
+sagesla_status sagesla_get_workspace_layout(int64_t B, int64_t H, int64_t N, int64_t D,
+                                            double topk_ratio, int block,
+                                            sagesla_workspace_layout* layout) {
+  if (!layout) return SAGESLA_ERR_INVALID_ARG;
+  if (D != kHeadDim || block != kBlock) return SAGESLA_ERR_UNSUPPORTED;
+  ForwardPlan p;
+  if (!make_plan(B, H, N, topk_ratio, &p)) return SAGESLA_ERR_INVALID_ARG;
+  *layout = p.lay;
+  return SAGESLA_OK;
+}
+
+size_t sagesla_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, double topk_ratio,
+                              int block) {
+  sagesla_workspace_layout L;
+  if (sagesla_get_workspace_layout(B, H, N, D, topk_ratio, block, &L) != SAGESLA_OK) return 0;
+  return L.total_bytes;
+}
+
+sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor* k,
+                                  const sagesla_tensor* v, double topk_ratio, int block,
+                                  sagesla_tensor* out, void* workspace, size_t workspace_bytes,
+                                  void* stream_ptr, const sagesla_options* opt) {
+  sagesla_status st;
+  if ((st = check_view(q, nullptr, false)) != SAGESLA_OK) return st;
+  if ((st = check_view(k, q, false)) != SAGESLA_OK) return st;
+  if ((st = check_view(v, q, false)) != SAGESLA_OK) return st;
+  if ((st = check_view(out, q, true)) != SAGESLA_OK) return st;
+  if (block != kBlock) return SAGESLA_ERR_UNSUPPORTED;
+  if (!valid_ratio(topk_ratio)) return SAGESLA_ERR_INVALID_ARG;
+  ForwardPlan p;
+  if (!make_plan(q->B, q->H, q->N, topk_ratio, &p)) return SAGESLA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
+      workspace_bytes < p.lay.total_bytes)
+    return SAGESLA_ERR_WORKSPACE;
+  uintptr_t o0, o1, a0, a1;
+  extent(out, &o0, &o1);
+  for (const sagesla_tensor* t : {q, k, v}) {
+    extent(t, &a0, &a1);
+    if (overlaps(o0, o1, a0, a1)) return SAGESLA_ERR_INVALID_ARG;
+  }
+  const uintptr_t w0 = reinterpret_cast<uintptr_t>(workspace);
+  if (overlaps(o0, o1, w0, w0 + p.lay.total_bytes)) return SAGESLA_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGESLA_OK) return st;
+
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  char* ws = static_cast<char*>(workspace);
+  const TensorArg qa = to_arg(q), ka = to_arg(k), va = to_arg(v);
+  SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.lay.status, 0, sizeof(int32_t), stream));
+  SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
+  SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
+  SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
+  SAGESLA_LAUNCH(launch_scores(p, ws, stream));
+  SAGESLA_LAUNCH(launch_topk(p, ws, stream));
+  if (!p.linear_empty) SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
+  SAGESLA_LAUNCH(launch_attention(p, qa, out->data, out->dtype, out->stride_b, out->stride_h,
+                                  out->stride_n, opt ? opt->sparse_out : nullptr, ws, stream));
+  if (opt) {
+    if (opt->kept_idx_out)
+      SAGESLA_LAUNCH(cudaMemcpyAsync(opt->kept_idx_out, ws + p.lay.kept,
+                                     static_cast<size_t>(p.BH * p.nb * p.k) * 4,
+                                     cudaMemcpyDeviceToDevice, stream));
+    if (opt->mask_out)
+      SAGESLA_LAUNCH(cudaMemcpyAsync(opt->mask_out, ws + p.lay.mask,
+                                     static_cast<size_t>(p.BH * p.nb * p.mask_words) * 4,
+                                     cudaMemcpyDeviceToDevice, stream));
+    if (opt->scores_out) SAGESLA_LAUNCH(launch_scale_scores(p, ws, opt->scores_out, stream));
+  }
+  return SAGESLA_OK;
+}
+
+sagesla_status sagesla_forward(const sagesla_tensor* q, const sagesla_tensor* k,
+                               const sagesla_tensor* v, double topk_ratio, int block,
+                               sagesla_tensor* out, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return sagesla_forward_ex(q, k, v, topk_ratio, block, out, workspace, workspace_bytes, stream,
+                            nullptr);
+}
+
+size_t sagesla_host_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
+                                   double topk_ratio, int block, int32_t out_dtype) {
+  if (out_dtype != SAGESLA_BF16 && out_dtype != SAGESLA_F32) return 0;
+  const size_t fw = sagesla_workspace_size(B, H, N, D, topk_ratio, block);
+  if (fw == 0) return 0;
+  const size_t elems = static_cast<size_t>(B * H * N * D);
+  return fw + 3 * align_up(elems * 2, kAlign) + align_up(elems * elem_bytes(out_dtype), kAlign);
+}
+
+sagesla_status sagesla_stream_status(void* stream_ptr, void* workspace) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SAGESLA_ERR_CUDA;
+  if (!workspace) return SAGESLA_OK;
+  int32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SAGESLA_ERR_CUDA;
+  if (word != 0) {
+    const int32_t zero = 0;
+    if (cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return SAGESLA_ERR_CUDA;
+  }
+  return static_cast<sagesla_status>(word);
+}
+
+sagesla_status sagesla_forward_host(const uint16_t* q_host, const uint16_t* k_host,
+                                    const uint16_t* v_host, int64_t B, int64_t H, int64_t N,
+                                    int64_t D, double topk_ratio, int block, void* out_host,
+                                    int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream_ptr) {
+  if (!q_host || !k_host || !v_host || !out_host) return SAGESLA_ERR_INVALID_ARG;
+  const size_t need = sagesla_host_workspace_size(B, H, N, D, topk_ratio, block, out_dtype);
+  if (need == 0) {
+    if (D != kHeadDim || block != kBlock) return SAGESLA_ERR_UNSUPPORTED;
+    return SAGESLA_ERR_INVALID_ARG;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
+      workspace_bytes < need)
+    return SAGESLA_ERR_WORKSPACE;
+  const size_t fw = sagesla_workspace_size(B, H, N, D, topk_ratio, block);
+  const size_t elems = static_cast<size_t>(B * H * N * D);
+  const size_t in_bytes = elems * 2, out_bytes = elems * elem_bytes(out_dtype);
+  char* base = static_cast<char*>(workspace);
+  char* dq = base + fw;
+  char* dk = dq + align_up(in_bytes, kAlign);
+  char* dv = dk + align_up(in_bytes, kAlign);
+  char* dout = dv + align_up(in_bytes, kAlign);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  sagesla_status st = check_device();
+  if (st != SAGESLA_OK) return st;
+  if (cudaMemcpyAsync(dq, q_host, in_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k_host, in_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v_host, in_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return SAGESLA_ERR_CUDA;
+  auto view = [&](void* data, int32_t dt) {
+    sagesla_tensor t;
+    t.data = data;
+    t.dtype = dt;
+    t.B = B; t.H = H; t.N = N; t.D = D;
+    t.stride_n = D;
+    t.stride_h = N * D;
+    t.stride_b = H * N * D;
+    return t;
+  };
+  sagesla_tensor tq = view(dq, SAGESLA_BF16), tk = view(dk, SAGESLA_BF16),
+                 tv = view(dv, SAGESLA_BF16), to = view(dout, out_dtype);
+  st = sagesla_forward(&tq, &tk, &tv, topk_ratio, block, &to, base, fw, stream_ptr);
+  if (st != SAGESLA_OK) return st;
+  if (cudaMemcpyAsync(out_host, dout, out_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return SAGESLA_ERR_CUDA;
+  return sagesla_stream_status(stream_ptr, base);
+}
+
+}  // extern "C"

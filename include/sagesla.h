@@ -71,7 +71,15 @@ typedef struct {
   uint32_t* mask_out;
   float* scores_out;
   float* sparse_out;   /* [B*H][N][128] float: the sparse-branch output alone */
+  /* NULL, or SAGESLA_N_STAGES + 1 cudaEvent_t handles (created by the caller): event i is
+   * recorded on the stream before stage i and the last one after the final stage, so that
+   * the caller can time each kernel on the launching stream. Stages, in order: K/V statistics
+   * and key-block states, statistics finalize, quantization, block scores, Top-K selection,
+   * complement sums (skipped when every block is kept), sparse attention + linear branch. */
+  void** stage_events;
 } sagesla_options;
+
+#define SAGESLA_N_STAGES 7
 
 /* Offsets (bytes, from the workspace start) of the intermediates a forward call leaves in
  * its workspace, for inspection after the stream has completed. Per-head arrays are

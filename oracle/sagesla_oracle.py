@@ -217,6 +217,29 @@ def quant_v_fp8(v_head: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 # The two branches
 # --------------------------------------------------------------------------------------
 
+# The P-tile code is a floating-point decision (which e4m3 code 448 p rounds to). Both sides
+# take it in binary32 with one formula: in base-2 units with the factor 448 folded in,
+#   c = fl32(fl32(sq_i * L) * sk_j),  L = fl32(fl32(log2 e) * fl32(1/sqrt(128)))
+#   m = max over the keys seen so far of fl32(S_max * c)        (running, per 64-key block)
+#   x = fl32(S * c + fl32(log2(448) - m))                        (one rounding, as an FMA)
+#   code = e4m3(2^x)
+# 2^x itself is taken exactly here; the kernel's exp2 approximation (relative error <= 3e-7)
+# is the only remaining difference. The row sums and the accumulation stay in float64.
+P_LOG2_SCALE = np.float32(np.float32(1.4426950408889634) * np.float32(0.08838834764831845))
+P_LOG2_448 = np.float32(8.807354922057604)
+
+
+def p_codes_binary32(s_int: np.ndarray, sq_i, sk_j, m_run32: np.ndarray):
+    """e4m3 values of the P tile (448 p) decided in binary32; returns (values, new m32)."""
+    c = np.float32(np.float32(sq_i) * P_LOG2_SCALE) * np.float32(sk_j)
+    mx = (s_int.max(axis=1).astype(np.float32) * c).astype(np.float32)
+    m_new = np.maximum(m_run32, mx).astype(np.float32)
+    neg = (P_LOG2_448 - m_new).astype(np.float32)
+    # S * c is exact in float64 (|S| < 2^22, 24-bit c); one rounding to binary32 like an FMA
+    x = (s_int.astype(np.float64) * np.float64(c) + neg.astype(np.float64)[:, None]).astype(np.float32)
+    return round_e4m3(np.exp2(x.astype(np.float64))), m_new
+
+
 def phi(x: np.ndarray) -> np.ndarray:
     """Softmax over the last (head) dimension."""
     z = np.exp(x - x.max(axis=-1, keepdims=True))
@@ -300,6 +323,7 @@ def sparse_block_row(prep: HeadPrep, i: int, q, k, v, quant: bool = True,
     nq = qrows.stop - qrows.start
     d = q.shape[1]
     m = np.full(nq, -np.inf)
+    m32 = np.full(nq, -np.inf, dtype=np.float32)
     l = np.zeros(nq)
     o = np.zeros((nq, d))
     inv_sqrt_d = 1.0 / math.sqrt(d)
@@ -319,7 +343,7 @@ def sparse_block_row(prep: HeadPrep, i: int, q, k, v, quant: bool = True,
         p = np.exp(s - m_new[:, None])
         l = alpha * l + p.sum(axis=1)
         if quant:
-            p8 = round_e4m3(E4M3_MAX * p)
+            p8, m32 = p_codes_binary32(s_int, prep.sq[i], prep.sk[j], m32)
             o = alpha[:, None] * o + p8 @ prep.v8[krows]
         else:
             o = alpha[:, None] * o + p @ v[krows]

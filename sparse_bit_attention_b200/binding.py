@@ -40,9 +40,14 @@ class SageslaTensor(ctypes.Structure):
                 ("stride_h", ctypes.c_int64), ("stride_n", ctypes.c_int64)]
 
 
+N_STAGES = 7
+STAGE_NAMES = ["stats", "finalize", "quant", "scores", "topk", "complement_gemm", "attention"]
+
+
 class SageslaOptions(ctypes.Structure):
     _fields_ = [("kept_idx_out", ctypes.c_void_p), ("mask_out", ctypes.c_void_p),
-                ("scores_out", ctypes.c_void_p), ("sparse_out", ctypes.c_void_p)]
+                ("scores_out", ctypes.c_void_p), ("sparse_out", ctypes.c_void_p),
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
 
 
 _LAYOUT_FIELDS = ["status", "q8", "k8", "v8", "sq", "sk", "s_v", "inv_v", "mu", "qbar", "kbar",
@@ -158,8 +163,11 @@ def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_rati
                     block: int = BLOCK, out: torch.Tensor | None = None,
                     workspace: torch.Tensor | None = None, stream=None,
                     out_dtype: torch.dtype = torch.float32, kept_idx_out=None, mask_out=None,
-                    scores_out=None, sparse_out=None) -> torch.Tensor:
-    """SageSLA forward on device tensors q, k, v (bf16 [B, H, N, 128]); returns ``out``."""
+                    scores_out=None, sparse_out=None, stage_events=None) -> torch.Tensor:
+    """SageSLA forward on device tensors q, k, v (bf16 [B, H, N, 128]); returns ``out``.
+
+    ``stage_events``: optional list of N_STAGES + 1 torch.cuda.Event(enable_timing=True)
+    recorded around each kernel of the forward on the launching stream."""
     lib = load_library()
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
@@ -172,8 +180,16 @@ def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_rati
     args = (ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), float(topk_ratio), int(block),
             ctypes.byref(vo), ctypes.c_void_p(workspace.data_ptr()),
             workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_ptr(stream)))
-    if any(x is not None for x in extra):
+    if any(x is not None for x in extra) or stage_events is not None:
         opt = SageslaOptions(*[None if x is None else x.data_ptr() for x in extra])
+        if stage_events is not None:
+            if len(stage_events) != N_STAGES + 1:
+                raise ValueError(f"stage_events needs {N_STAGES + 1} events")
+            for e in stage_events:          # torch creates the CUDA event on first record
+                if e.cuda_event == 0:
+                    e.record()
+            handles = (ctypes.c_void_p * (N_STAGES + 1))(*[e.cuda_event for e in stage_events])
+            opt.stage_events = ctypes.cast(handles, ctypes.POINTER(ctypes.c_void_p))
         _check(lib.sagesla_forward_ex(*args, ctypes.byref(opt)), "sagesla_forward_ex")
     else:
         _check(lib.sagesla_forward(*args), "sagesla_forward")

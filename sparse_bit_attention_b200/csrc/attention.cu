@@ -13,13 +13,23 @@
 // B200 mapping. One CTA per PAIR of adjacent query blocks (128 rows = the tcgen05 M=128 tile)
 // walking the union of the two blocks' kept lists; rows of a block that does not keep the
 // current key block get P = 0 and skip their softmax work. Warp roles:
-//   warps 0-3  softmax / correction / epilogue, one query row per thread (TMEM lane = row)
-//   warp 4     TMA producer: Q tile once, then K8/V8 tiles through a 4-stage ring
-//   warp 5     MMA issuer: S(n) = Q K_j^T (kind::i8, M128 N64 K128) into one of two S
+//   warps 0-7  softmax / correction / epilogue: two threads per query row (TMEM lane = row),
+//              warp w exponentiates S columns 32*(w/4) .. +31 (both threads of a row read
+//              all 64 for the block maximum) and owns O columns 64*(w/4) .. +63
+//   warp 8     TMA producer: Q tile once, then K8/V8 tiles through a 4-stage ring
+//   warp 9     MMA issuer: S(n) = Q K_j^T (kind::i8, M128 N64 K128) into one of two S
 //              buffers, then O += P(n-1) V (kind::f8f6f4, M128 N128 K64) — S(n+1) overlaps
 //              the softmax of n.
 // TMEM (256 columns): O fp32 [0,128), S int32 [128,192) and [192,256); after the loop the S
 // columns hold phi(Q) . G for the linear branch. Two CTAs fit on an SM.
+//
+// Softmax arithmetic per score: the int32 score becomes a float exactly through the 1.5*2^23
+// bias (integer add, float subtract: no conversion-pipe instruction); one FFMA forms the
+// base-2 exponent with the factor 448 of the P quantization folded in; 2^x comes from the
+// MUFU ex2 unit for most columns and, for the rest, from Cody-Waite range reduction (round
+// to nearest integer) plus a degree-5 polynomial fitted here by the Remez exchange algorithm
+// for minimax relative error on [-1/2, 1/2] (max relative error 2.3e-7 in fp32), so that the
+// FMA pipe takes part of the exponential load of the MUFU unit.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -30,6 +40,10 @@ namespace sagesla {
 namespace {
 
 constexpr int kNS = 4;                       // K/V ring stages
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
 constexpr uint32_t kQBytes = 128 * 128;      // int8 Q tile
 constexpr uint32_t kKVBytes = 64 * 128;      // one K8 or V8 tile
 constexpr uint32_t kStageBytes = 2 * kKVBytes;
@@ -39,6 +53,11 @@ constexpr uint32_t kOffP = kOffStages + kNS * kStageBytes;
 constexpr uint32_t kOffCtl = kOffP + 2 * kPBytes;      // 96 KB
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemS = 128;              // first S buffer column
+// Columns of each thread's 32 whose exponential uses the polynomial instead of MUFU ex2.
+constexpr int kPolyFrom = 20;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kInvSqrtD = 0.08838834764831845f;
+constexpr float kLog2_448 = 8.807354922057604f;
 
 struct Ctl {
   uint64_t full[kNS], empty[kNS];
@@ -48,6 +67,8 @@ struct Ctl {
   int list_len;
   volatile int abort;
   float s_v[128];
+  float xf[2][128];          // [column half][row]: epilogue exchanges
+  float xd[2][128];
 };
 
 struct AttnParams {
@@ -76,7 +97,40 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ct
   return true;
 }
 
-__global__ void __launch_bounds__(192, 2)
+// Named barrier for the two warps (64 threads) that share a group of 32 rows. Used only in
+// the epilogue, where both threads of a row execute it the same number of times on every
+// path (a named barrier cannot time out).
+__device__ __forceinline__ void pair_sync(int id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+
+// int32 -> float, exact for |s| < 2^22 (the INT8 product of a 128-channel row is < 2^21).
+__device__ __forceinline__ float s32_to_f32(uint32_t s) {
+  return __int_as_float(static_cast<int>(s + 0x4B400000u)) - 12582912.0f;
+}
+
+__device__ __forceinline__ float ex2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe: x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f by a degree-5
+// minimax polynomial (coefficients from a Remez fit of relative error); 2^n added to the
+// exponent field. x is clamped below at -125 so that the result stays a normal float.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;              // rint(x) in the low mantissa bits
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(0.0013276472454890609f, f, 0.009675540961325169f);
+  p = fmaf(p, f, 0.05550713092088699f);
+  p = fmaf(p, f, 0.24022120237350464f);
+  p = fmaf(p, f, 0.6931469440460205f);
+  p = fmaf(p, f, 1.0000001192092896f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
 k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
             AttnParams prm) {
@@ -133,20 +187,20 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     for (int s = 0; s < kNS; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->s_full[s], 1);
-      mbar_init(&ctl->s_free[s], 128);
-      mbar_init(&ctl->p_full[s], 128);
+      mbar_init(&ctl->s_free[s], kSoftmaxThreads);
+      mbar_init(&ctl->p_full[s], kSoftmaxThreads);
       mbar_init(&ctl->pv_done[s], 1);
     }
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->g_full, 1);
-    mbar_init(&ctl->a_full, 128);
+    mbar_init(&ctl->a_full, kSoftmaxThreads);
     mbar_init(&ctl->la_done, 1);
-    mbar_init(&ctl->la_free, 64);
+    mbar_init(&ctl->la_free, kSoftmaxThreads / 2);
     mbar_init(&ctl->lb_done, 1);
     mbar_init(&ctl->mma_done, 1);
     ctl->abort = 0;
     fence_mbar_init();
-  } else if (threadIdx.x == 128) {
+  } else if (threadIdx.x == 96) {
     prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_g);
   }
   tc_fence_before();
@@ -156,7 +210,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   const int U = ctl->list_len;
   const bool has_b = ib < prm.nb;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int row_base = static_cast<int>(bh * prm.n_pad);
@@ -185,7 +239,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc(kFmtS32, kFmtS8, kFmtS8, 0, 0, 128, 64);
@@ -261,75 +315,88 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int row = 32 * warp + lane;            // 0..127, TMEM lane
+    const int quad = warp & 3;                   // TMEM lane quarter
+    const int ch = warp >> 2;                    // column half: S cols 32ch.., O cols 64ch..
+    const int row = 32 * quad + lane;            // 0..127, TMEM lane
     const int half = row >> 6;                   // 0: block ia, 1: block ib
     const uint32_t my_bit = 1u << half;
     const int qblock = ia + half;
-    const float cs = prm.sq[bh * prm.nbq + qblock] * (1.4426950408889634f * 0.08838834764831845f);
-    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
+    const int bar_id = 1 + quad;                 // named barrier of warps quad, quad + 4
+    const float cs = prm.sq[bh * prm.nbq + qblock] * (kLog2e * kInvSqrtD);
+    const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
+    float m_run = -INFINITY, l_part = 0.f;
     bool ok = true;
     for (int n = 0; n < U; ++n) {
       const int b = n & 1;
       const uint32_t e = list[n];
       const int j = static_cast<int>(e & 0xFFFFFFu);
-      const bool mine = ((e >> 24) & my_bit) != 0;     // warp-uniform
+      const bool mine = ((e >> 24) & my_bit) != 0;     // same for both warps of a row group
       if (!wait_or_abort(&ctl->s_full[b], (n >> 1) & 1, ctl, status)) { ok = false; break; }
       tc_fence_after();
-      uint32_t pk[16];
+      uint32_t pk[8];
       float alpha = 1.f;
       if (mine) {
-        uint32_t sr[64];
-        tmem_ld32(tmem + lane_base + kTmemS + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tmem + lane_base + kTmemS + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        // Both threads of a row read all 64 scores for the block maximum (no exchange
+        // between them inside the loop) and exponentiate their own 32.
+        uint32_t sr[32], so[32];
+        tmem_ld32(tmem + lane_base + kTmemS + 64 * b + 32 * ch, sr);
+        tmem_ld32(tmem + lane_base + kTmemS + 64 * b + 32 * (ch ^ 1), so);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&ctl->s_free[b]);
-        const int valid = (j == prm.nb - 1) ? prm.n_last : 64;
-        const float c = cs * list_sk[n];
+        const int nvalid = (j == prm.nb - 1) ? prm.n_last : 64;
+        const int valid = nvalid - 32 * ch;            // may be <= 0
+        const int valid_o = nvalid - 32 * (ch ^ 1);
         int mxi = INT_MIN;
 #pragma unroll
-        for (int q = 0; q < 64; ++q)
+        for (int q = 0; q < 32; ++q) {
           if (q < valid) mxi = max(mxi, static_cast<int>(sr[q]));
-        const float m_new = fmaxf(m_run, static_cast<float>(mxi) * c);
-        alpha = exp2f(m_run - m_new);
+          if (q < valid_o) mxi = max(mxi, static_cast<int>(so[q]));
+        }
+        const float c = cs * list_sk[n];
+        const float m_new = fmaxf(m_run, s32_to_f32(static_cast<uint32_t>(mxi)) * c);
+        alpha = ex2_mufu(m_run - m_new);
+        const float neg = kLog2_448 - m_new;      // exponent offset: 2^(x) = 448 p
         float rs = 0.f;
 #pragma unroll
-        for (int q = 0; q < 64; q += 2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (q < valid) p0 = exp2f(fmaf(static_cast<float>(static_cast<int>(sr[q])), c, -m_new));
-          if (q + 1 < valid) p1 = exp2f(fmaf(static_cast<float>(static_cast<int>(sr[q + 1])), c, -m_new));
-          rs += p0 + p1;
-          const uint32_t two = f32x2_to_e4m3x2(448.f * p0, 448.f * p1);
+        for (int q = 0; q < 32; q += 2) {
+          float y0 = 0.f, y1 = 0.f;
+          const float x0 = fmaf(s32_to_f32(sr[q]), c, neg);
+          const float x1 = fmaf(s32_to_f32(sr[q + 1]), c, neg);
+          if (q < valid) y0 = q < kPolyFrom ? ex2_mufu(x0) : ex2_poly(x0);
+          if (q + 1 < valid) y1 = q + 1 < kPolyFrom ? ex2_mufu(x1) : ex2_poly(x1);
+          rs += y0 + y1;
+          const uint32_t two = f32x2_to_e4m3x2(y0, y1);
           if ((q & 2) == 0) pk[q >> 2] = two; else pk[q >> 2] |= two << 16;
         }
-        l_run = alpha * l_run + rs;
+        l_part = alpha * l_part + rs;
         m_run = m_new;
       } else {
         tc_fence_before();
         mbar_arrive(&ctl->s_free[b]);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) pk[q] = 0u;
+        for (int q = 0; q < 8; ++q) pk[q] = 0u;
       }
       // P(n) into buffer b once P.V(n-2) has read it
       if (n >= 2 && !wait_or_abort(&ctl->pv_done[b], ((n >> 1) - 1) & 1, ctl, status)) { ok = false; break; }
-      uint8_t* pb = smem + kOffP + b * kPBytes + (row >> 3) * 512 + (row & 7) * 16;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(pb + q * 128) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      uint8_t* pb = smem + kOffP + b * kPBytes + (row >> 3) * 512 + (row & 7) * 16 + 2 * ch * 128;
+      *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(pb + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       fence_proxy_async_smem();
-      // rescale O by alpha once P.V(n-1) has landed (skipped when no row's max moved)
+      // rescale this thread's 64 O columns once P.V(n-1) has landed (skipped when no row's
+      // max moved in this warp)
       if (n >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (!wait_or_abort(&ctl->pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_base + 32 * cc, o);
+          const uint32_t ta = tmem + lane_base + 64 * ch + 32 * cc;
+          tmem_ld32(ta, o);
           tmem_ld_wait();
 #pragma unroll
           for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(tmem + lane_base + 32 * cc, o);
+          tmem_st32(ta, o);
         }
         tmem_st_wait();
       }
@@ -340,12 +407,17 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // ------------------------------------------------------------ epilogue
     if (ok) ok = wait_or_abort(&ctl->pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1, ctl, status);
     tc_fence_after();
+    // total row sum (of 448 p) from the two column halves
+    ctl->xf[ch][row] = l_part;
+    pair_sync(bar_id);
+    const float l448 = l_part + ctl->xf[ch ^ 1][row];
     const int tok = 128 * pair + row;            // token index within the head
     const bool store = ok && tok < prm.N;
     const int64_t b_ = bh / prm.q.H, h_ = bh % prm.q.H;
-    float den = 1.f;
+    float den = 0.f;
     if (prm.linear && ok) {
-      // phi(q) for this row into the A operand (bf16, K-major, 128-byte swizzle)
+      // phi(q) for this row; this thread writes channels 64ch .. 64ch+63 of the A operand
+      // (bf16, K-major, 128-byte swizzle) and sums its part of the normalizer.
       const uint16_t* qrow = static_cast<const uint16_t*>(prm.q.data) + b_ * prm.q.stride_b +
                              h_ * prm.q.stride_h + static_cast<int64_t>(min(tok, prm.N - 1)) * prm.q.stride_n;
       const uint4* q4 = reinterpret_cast<const uint4*>(qrow);
@@ -372,7 +444,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           prm.gsum + ((bh * prm.nb_m_pad + qblock) * 129 + 128) * 128);
       float dsum = 0.f;
 #pragma unroll 2
-      for (int u = 0; u < 16; ++u) {
+      for (int uu = 0; uu < 8; ++uu) {
+        const int u = 8 * ch + uu;
         const uint4 r = __ldg(q4 + u);
         const uint4 gg = __ldg(g128 + u);
         const uint32_t w[4] = {r.x, r.y, r.z, r.w};
@@ -387,13 +460,20 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           dsum = fmaf(__low2float(p2), __uint_as_float(gw[z] << 16), dsum);
           dsum = fmaf(__high2float(p2), __uint_as_float(gw[z] & 0xFFFF0000u), dsum);
         }
-        const uint32_t off = (u >> 3) * 16384u + sw128_offset(row, u & 7);
+        const uint32_t off = ch * 16384u + sw128_offset(row, uu);
         *reinterpret_cast<uint4*>(smem + off) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
-      den = dsum;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&ctl->a_full);
+      den = dsum;
+    }
+    // normalizer of the linear branch from the two column halves (executed by every softmax
+    // thread exactly once, whatever path it took)
+    ctl->xd[ch][row] = den;
+    pair_sync(bar_id);
+    den += ctl->xd[ch ^ 1][row];
+    if (prm.linear && ok) {
       // wait for this half's phi(Q) . G (rows of a missing second block store nothing)
       if (half == 0 || has_b) {
         ok = wait_or_abort(half == 0 ? &ctl->la_done : &ctl->lb_done, 0, ctl, status);
@@ -402,7 +482,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         ok = false;
       }
     }
-    const float inv_l = 1.f / (448.f * l_run);
+    const float inv_l = 1.f / l448;
     const float inv_den = 1.f / den;
     float* sp_row = (prm.sparse_out && store) ? prm.sparse_out + (bh * prm.N + tok) * 128 : nullptr;
     char* out_row = static_cast<char*>(prm.out) +
@@ -410,25 +490,26 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         (prm.out_dtype == SAGESLA_F32 ? 4 : 2);
     if (ok) {
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int col0 = 64 * ch + 32 * cc;
         uint32_t o[32], lin[32];
-        tmem_ld32(tmem + lane_base + 32 * cc, o);
-        if (prm.linear) tmem_ld32(tmem + lane_base + kTmemS + 32 * cc, lin);
+        tmem_ld32(tmem + lane_base + col0, o);
+        if (prm.linear) tmem_ld32(tmem + lane_base + kTmemS + col0, lin);
         tmem_ld_wait();
         float res[32];
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-          const float os = __uint_as_float(o[q]) * ctl->s_v[32 * cc + q] * inv_l;
-          if (sp_row) sp_row[32 * cc + q] = os;
+          const float os = __uint_as_float(o[q]) * ctl->s_v[col0 + q] * inv_l;
+          if (sp_row) sp_row[col0 + q] = os;
           res[q] = prm.linear ? os + __uint_as_float(lin[q]) * inv_den : os;
         }
         if (store) {
           if (prm.out_dtype == SAGESLA_F32) {
-            float4* d = reinterpret_cast<float4*>(out_row) + 8 * cc;
+            float4* d = reinterpret_cast<float4*>(out_row) + col0 / 4;
 #pragma unroll
             for (int q = 0; q < 8; ++q) d[q] = make_float4(res[4 * q], res[4 * q + 1], res[4 * q + 2], res[4 * q + 3]);
           } else {
-            uint4* d = reinterpret_cast<uint4*>(out_row) + 4 * cc;
+            uint4* d = reinterpret_cast<uint4*>(out_row) + col0 / 8;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               uint32_t w[4];
@@ -499,7 +580,7 @@ cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(p.n_pairs), static_cast<unsigned>(p.BH));
-  k_attention<<<grid, 192, smem, stream>>>(tq, tk, tv, tg, prm);
+  k_attention<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tg, prm);
   return cudaGetLastError();
 }
 

@@ -253,15 +253,27 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   char* ws = static_cast<char*>(workspace);
   const TensorArg qa = to_arg(q), ka = to_arg(k), va = to_arg(v);
+  void** ev = opt ? opt->stage_events : nullptr;
+  auto mark = [&](int i) -> cudaError_t {
+    return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), stream) : cudaSuccess;
+  };
   SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.lay.status, 0, sizeof(int32_t), stream));
+  SAGESLA_LAUNCH(mark(0));
   SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
+  SAGESLA_LAUNCH(mark(1));
   SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
+  SAGESLA_LAUNCH(mark(2));
   SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
+  SAGESLA_LAUNCH(mark(3));
   SAGESLA_LAUNCH(launch_scores(p, ws, stream));
+  SAGESLA_LAUNCH(mark(4));
   SAGESLA_LAUNCH(launch_topk(p, ws, stream));
+  SAGESLA_LAUNCH(mark(5));
   if (!p.linear_empty) SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
+  SAGESLA_LAUNCH(mark(6));
   SAGESLA_LAUNCH(launch_attention(p, qa, out->data, out->dtype, out->stride_b, out->stride_h,
                                   out->stride_n, opt ? opt->sparse_out : nullptr, ws, stream));
+  SAGESLA_LAUNCH(mark(SAGESLA_N_STAGES));
   if (opt) {
     if (opt->kept_idx_out)
       SAGESLA_LAUNCH(cudaMemcpyAsync(opt->kept_idx_out, ws + p.lay.kept,

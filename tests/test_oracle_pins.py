@@ -257,3 +257,28 @@ def test_quantized_forward_is_close_to_exact():
     _, b = orc.forward_head(q, k, v, 0.25, quant=False)
     err = max(np.abs(a[i]["o"] - b[i]["o"]).max() for i in a)
     assert 1e-4 < err < 0.08
+
+
+def test_p_code_decision_in_binary32_matches_float64_away_from_midpoints():
+    """The P-tile codes decided in binary32 differ from the float64 decision e4m3(448 p) only
+    where 448 p lies within 1e-5 (relative) of a rounding midpoint of the e4m3 grid."""
+    rng = np.random.default_rng(16)
+    grid = orc.e4m3_decode(np.arange(0, 127))
+    mids = (grid[:-1] + grid[1:]) / 2
+    checked = flips = 0
+    for trial in range(40):
+        s_int = rng.integers(-30000, 30000, size=(64, 64))
+        sq, sk = np.float32(rng.uniform(0.01, 0.05)), np.float32(rng.uniform(0.01, 0.05))
+        m0 = np.full(64, -np.inf, dtype=np.float32)
+        p8, m32 = orc.p_codes_binary32(s_int, sq, sk, m0)
+        s = s_int * (float(sq) * float(sk)) / math.sqrt(128)
+        y = 448.0 * np.exp(s - s.max(axis=1, keepdims=True))
+        ref = orc.round_e4m3(y)
+        near = np.min(np.abs(y[..., None] - mids[None, None, :]), axis=-1) <= 1e-5 * y
+        diff = p8 != ref
+        assert not np.any(diff & ~near)
+        checked += diff.size
+        flips += int(diff.sum())
+        # the running maximum is the binary32 image of the row maximum
+        np.testing.assert_allclose(m32, s.max(axis=1) * math.log2(math.e), rtol=1e-6)
+    assert flips < checked * 1e-3

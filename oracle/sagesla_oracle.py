@@ -223,21 +223,37 @@ def quant_v_fp8(v_head: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 #   m = max over the keys seen so far of fl32(S_max * c)        (running, per 64-key block)
 #   x = fl32(S * c + fl32(log2(448) - m))                        (one rounding, as an FMA)
 #   code = e4m3(2^x)
-# 2^x itself is taken exactly here; the kernel's exp2 approximation (relative error <= 3e-7)
-# is the only remaining difference. The row sums and the accumulation stay in float64.
+# 2^x itself is taken exactly here. A binary32 exp2 evaluation (relative error up to
+# EXP2_REL_ERR) can round a value that lies that close to an e4m3 midpoint to the neighbouring
+# code: those codes are ambiguous, and the oracle reports how much choosing the other code
+# could change each output element (``o_s_ambig``). The row sums and the accumulation stay in
+# float64.
 P_LOG2_SCALE = np.float32(np.float32(1.4426950408889634) * np.float32(0.08838834764831845))
 P_LOG2_448 = np.float32(8.807354922057604)
 
 
 def p_codes_binary32(s_int: np.ndarray, sq_i, sk_j, m_run32: np.ndarray):
-    """e4m3 values of the P tile (448 p) decided in binary32; returns (values, new m32)."""
+    """e4m3 values of the P tile (448 p) decided in binary32; returns (values, new m32, and
+    the exact 2^x that was rounded)."""
     c = np.float32(np.float32(sq_i) * P_LOG2_SCALE) * np.float32(sk_j)
     mx = (s_int.max(axis=1).astype(np.float32) * c).astype(np.float32)
     m_new = np.maximum(m_run32, mx).astype(np.float32)
     neg = (P_LOG2_448 - m_new).astype(np.float32)
     # S * c is exact in float64 (|S| < 2^22, 24-bit c); one rounding to binary32 like an FMA
     x = (s_int.astype(np.float64) * np.float64(c) + neg.astype(np.float64)[:, None]).astype(np.float32)
-    return round_e4m3(np.exp2(x.astype(np.float64))), m_new
+    y = np.exp2(x.astype(np.float64))
+    return round_e4m3(y), m_new, y
+
+
+EXP2_REL_ERR = 1e-6
+
+
+def e4m3_ambiguity(y: np.ndarray, rel: float = EXP2_REL_ERR) -> np.ndarray:
+    """|code change| (as a value) when y, perturbed by up to rel relative, can round to the
+    neighbouring e4m3 value instead; 0 where the rounding is unambiguous."""
+    lo = round_e4m3(y * (1.0 - rel))
+    hi = round_e4m3(y * (1.0 + rel))
+    return np.maximum(np.abs(hi - round_e4m3(y)), np.abs(round_e4m3(y) - lo))
 
 
 def phi(x: np.ndarray) -> np.ndarray:
@@ -315,7 +331,7 @@ def key_block_states(k: np.ndarray, v: np.ndarray) -> np.ndarray:
 
 
 def sparse_block_row(prep: HeadPrep, i: int, q, k, v, quant: bool = True,
-                     smooth_in_quant_off: bool = False) -> np.ndarray:
+                     smooth_in_quant_off: bool = False, return_ambiguity: bool = False):
     """Sparse branch for the real query tokens of block i: online softmax over kept(i) in
     ascending order, running max updated per key block (no lazy rescale)."""
     n = prep.n
@@ -326,6 +342,7 @@ def sparse_block_row(prep: HeadPrep, i: int, q, k, v, quant: bool = True,
     m32 = np.full(nq, -np.inf, dtype=np.float32)
     l = np.zeros(nq)
     o = np.zeros((nq, d))
+    amb = np.zeros((nq, d))          # bound on |o| change from ambiguous P codes
     inv_sqrt_d = 1.0 / math.sqrt(d)
     if not quant and smooth_in_quant_off:
         k_used = k - smoothing_mean(k)[None, :]
@@ -343,13 +360,19 @@ def sparse_block_row(prep: HeadPrep, i: int, q, k, v, quant: bool = True,
         p = np.exp(s - m_new[:, None])
         l = alpha * l + p.sum(axis=1)
         if quant:
-            p8, m32 = p_codes_binary32(s_int, prep.sq[i], prep.sk[j], m32)
+            p8, m32, y32 = p_codes_binary32(s_int, prep.sq[i], prep.sk[j], m32)
             o = alpha[:, None] * o + p8 @ prep.v8[krows]
+            amb = alpha[:, None] * amb + e4m3_ambiguity(y32) @ np.abs(prep.v8[krows])
         else:
             o = alpha[:, None] * o + p @ v[krows]
         m = m_new
     if quant:
-        return o * prep.s_v.astype(np.float64)[None, :] / (E4M3_MAX * l[:, None])
+        scale = prep.s_v.astype(np.float64)[None, :] / (E4M3_MAX * l[:, None])
+        if return_ambiguity:
+            return o * scale, amb * scale
+        return o * scale
+    if return_ambiguity:
+        return o / l[:, None], np.zeros_like(o)
     return o / l[:, None]
 
 
@@ -410,10 +433,11 @@ def forward_head(q, k, v, topk_ratio: float, quant: bool = True, rows=None,
         rows = range(prep.nb)
     out = {}
     for i in rows:
-        o_s = sparse_block_row(prep, i, q, k, v, quant=quant,
-                               smooth_in_quant_off=smooth_in_quant_off)
+        o_s, amb = sparse_block_row(prep, i, q, k, v, quant=quant,
+                                    smooth_in_quant_off=smooth_in_quant_off,
+                                    return_ambiguity=True)
         o_l = linear_block_row(prep, i, q, h_blocks)
-        out[i] = {"o_s": o_s, "o_l": o_l, "o": o_s + o_l}
+        out[i] = {"o_s": o_s, "o_l": o_l, "o": o_s + o_l, "o_s_ambig": amb}
     return prep, out
 
 

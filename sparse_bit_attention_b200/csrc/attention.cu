@@ -47,14 +47,20 @@ constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
 constexpr uint32_t kQBytes = 128 * 128;      // int8 Q tile
 constexpr uint32_t kKVBytes = 64 * 128;      // one K8 or V8 tile
 constexpr uint32_t kStageBytes = 2 * kKVBytes;
-constexpr uint32_t kPBytes = 128 * 64;       // e4m3 P tile
+// e4m3 P tile, K-major without swizzle: core matrices of 8 rows x 16 keys (128 B); K-chunks
+// 160 B apart and 8-row groups 672 B apart. The padding makes the 16-byte stores of the
+// softmax threads (lanes of one store phase hold rows r, r+8, r+1, r+9 and key halves 0, 1)
+// fall on eight distinct bank groups.
+constexpr uint32_t kPChunk = 160, kPGroup = 672;
+constexpr uint32_t kPBytes = 16 * kPGroup;
 constexpr uint32_t kOffStages = kQBytes;
 constexpr uint32_t kOffP = kOffStages + kNS * kStageBytes;
-constexpr uint32_t kOffCtl = kOffP + 2 * kPBytes;      // 96 KB
+constexpr uint32_t kOffCtl = kOffP + 2 * kPBytes;
+static_assert(kOffCtl >= 96 * 1024, "the linear epilogue reuses [0, 96 KB) for its operands");
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemS = 128;              // first S buffer column
 // Columns of each thread's 32 whose exponential uses the polynomial instead of MUFU ex2.
-constexpr int kPolyFrom = 20;
+constexpr int kPolyFrom = 28;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kInvSqrtD = 0.08838834764831845f;
 constexpr float kLog2_448 = 8.807354922057604f;
@@ -130,6 +136,44 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// Maximum of this thread's valid scores (eight independent chains).
+template <bool kFull>
+__device__ __forceinline__ int row_block_max(const uint32_t (&a)[32], int valid) {
+  int m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = INT_MIN;
+#pragma unroll
+  for (int q = 0; q < 32; ++q)
+    if (kFull || q < valid) m[q & 7] = max(m[q & 7], static_cast<int>(a[q]));
+  return max(max(max(m[0], m[1]), max(m[2], m[3])), max(max(m[4], m[5]), max(m[6], m[7])));
+}
+
+// 448 p = 2^(S c + neg), neg = log2(448) - m, for this thread's 32 scores -> packed e4m3
+// codes and their sum.
+template <bool kFull>
+__device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int valid, float c,
+                                              float neg, uint32_t (&pk)[8]) {
+  float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+#pragma unroll
+  for (int q = 0; q < 32; q += 4) {
+    float y[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float x = fmaf(s32_to_f32(sr[q + t]), c, neg);
+      float v = (q + t < kPolyFrom) ? ex2_mufu(x) : ex2_poly(x);
+      if (!kFull && q + t >= valid) v = 0.f;
+      y[t] = v;
+    }
+    r0 += y[0];
+    r1 += y[1];
+    r2 += y[2];
+    r3 += y[3];
+    pk[q >> 2] = static_cast<uint32_t>(f32x2_to_e4m3x2(y[0], y[1])) |
+                 (static_cast<uint32_t>(f32x2_to_e4m3x2(y[2], y[3])) << 16);
+  }
+  return (r0 + r1) + (r2 + r3);
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
 k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -187,8 +231,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     for (int s = 0; s < kNS; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->s_full[s], 1);
-      mbar_init(&ctl->s_free[s], kSoftmaxThreads);
-      mbar_init(&ctl->p_full[s], kSoftmaxThreads);
+      mbar_init(&ctl->s_free[s], kSoftmaxWarps);
+      mbar_init(&ctl->p_full[s], kSoftmaxWarps);
       mbar_init(&ctl->pv_done[s], 1);
     }
     mbar_init(&ctl->q_full, 1);
@@ -253,10 +297,9 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const uint32_t v_addr = smem_u32(smem + kOffStages + (m % kNS) * kStageBytes + kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {   // 2 x K=32 keys
-          // P: K-major, no swizzle: 8x16-byte core matrices, K chunks 128 B apart, 8-row
-          // groups 512 B apart. V: MN-major (d contiguous), 128-byte swizzle, 8-key groups
-          // 1024 B apart.
-          const uint64_t ad = make_sdesc(p_addr + kk * 256, 128, 512, kLayoutNone);
+          // P: K-major, no swizzle (layout above). V: MN-major (d contiguous), 128-byte
+          // swizzle, 8-key groups 1024 B apart.
+          const uint64_t ad = make_sdesc(p_addr + kk * 2 * kPChunk, kPChunk, kPGroup, kLayoutNone);
           const uint64_t bd = make_sdesc(v_addr + kk * 4096, 8192, 1024, kLayoutSW128);
           mma_f8(tmem, ad, bd, idesc_pv, (m > 0 || kk > 0) ? 1u : 0u);
         }
@@ -315,103 +358,96 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int quad = warp & 3;                   // TMEM lane quarter
-    const int ch = warp >> 2;                    // column half: S cols 32ch.., O cols 64ch..
-    const int row = 32 * quad + lane;            // 0..127, TMEM lane
-    const int half = row >> 6;                   // 0: block ia, 1: block ib
+    // Loop mapping (16x64b TMEM fragment): warp w reads lanes 32*(w&3) + 16*(w>>2) + 0..15;
+    // lane t holds row lrow = t/4 + 8*(t&1) and key half p = (t>>1)&1, i.e. keys 32p..32p+31
+    // of the block (the K8 rows are stored key-interleaved). Lanes t and t^2 share a row.
+    const int quad = warp & 3;
+    const int sub = warp >> 2;
+    const int row = 32 * quad + 16 * sub + (lane >> 2) + 8 * (lane & 1);   // 0..127
+    const int kh = (lane >> 1) & 1;              // key half
+    const int half = row >> 6;                   // 0: block ia, 1: block ib (warp-uniform)
     const uint32_t my_bit = 1u << half;
     const int qblock = ia + half;
     const int bar_id = 1 + quad;                 // named barrier of warps quad, quad + 4
     const float cs = prm.sq[bh * prm.nbq + qblock] * (kLog2e * kInvSqrtD);
-    const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
+    const uint32_t lane16 = static_cast<uint32_t>(32 * quad + 16 * sub) << 16;
+    const int valid = prm.n_last - 32 * kh;      // valid keys of this thread in the last block
     float m_run = -INFINITY, l_part = 0.f;
     bool ok = true;
     for (int n = 0; n < U; ++n) {
       const int b = n & 1;
       const uint32_t e = list[n];
       const int j = static_cast<int>(e & 0xFFFFFFu);
-      const bool mine = ((e >> 24) & my_bit) != 0;     // same for both warps of a row group
+      const bool mine = ((e >> 24) & my_bit) != 0;     // warp-uniform
       if (!wait_or_abort(&ctl->s_full[b], (n >> 1) & 1, ctl, status)) { ok = false; break; }
       tc_fence_after();
       uint32_t pk[8];
       float alpha = 1.f;
       if (mine) {
-        // Both threads of a row read all 64 scores for the block maximum (no exchange
-        // between them inside the loop) and exponentiate their own 32.
-        uint32_t sr[32], so[32];
-        tmem_ld32(tmem + lane_base + kTmemS + 64 * b + 32 * ch, sr);
-        tmem_ld32(tmem + lane_base + kTmemS + 64 * b + 32 * (ch ^ 1), so);
+        uint32_t sr[32];
+        tmem_ld16x64(tmem + lane16 + kTmemS + 64 * b, sr);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&ctl->s_free[b]);
-        const int nvalid = (j == prm.nb - 1) ? prm.n_last : 64;
-        const int valid = nvalid - 32 * ch;            // may be <= 0
-        const int valid_o = nvalid - 32 * (ch ^ 1);
-        int mxi = INT_MIN;
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          if (q < valid) mxi = max(mxi, static_cast<int>(sr[q]));
-          if (q < valid_o) mxi = max(mxi, static_cast<int>(so[q]));
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->s_free[b]);
+        const bool full = j != prm.nb - 1 || prm.n_last == 64;   // no padded keys
+        int mxi = full ? row_block_max<true>(sr, 32) : row_block_max<false>(sr, valid);
+        mxi = max(mxi, __shfl_xor_sync(0xffffffffu, mxi, 2));
         const float c = cs * list_sk[n];
         const float m_new = fmaxf(m_run, s32_to_f32(static_cast<uint32_t>(mxi)) * c);
         alpha = ex2_mufu(m_run - m_new);
-        const float neg = kLog2_448 - m_new;      // exponent offset: 2^(x) = 448 p
-        float rs = 0.f;
-#pragma unroll
-        for (int q = 0; q < 32; q += 2) {
-          float y0 = 0.f, y1 = 0.f;
-          const float x0 = fmaf(s32_to_f32(sr[q]), c, neg);
-          const float x1 = fmaf(s32_to_f32(sr[q + 1]), c, neg);
-          if (q < valid) y0 = q < kPolyFrom ? ex2_mufu(x0) : ex2_poly(x0);
-          if (q + 1 < valid) y1 = q + 1 < kPolyFrom ? ex2_mufu(x1) : ex2_poly(x1);
-          rs += y0 + y1;
-          const uint32_t two = f32x2_to_e4m3x2(y0, y1);
-          if ((q & 2) == 0) pk[q >> 2] = two; else pk[q >> 2] |= two << 16;
-        }
+        const float neg = kLog2_448 - m_new;      // 2^(S c + neg) = 448 p
+        const float rs = full ? row_exp_pack<true>(sr, 32, c, neg, pk)
+                              : row_exp_pack<false>(sr, valid, c, neg, pk);
         l_part = alpha * l_part + rs;
         m_run = m_new;
       } else {
         tc_fence_before();
-        mbar_arrive(&ctl->s_free[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->s_free[b]);
 #pragma unroll
         for (int q = 0; q < 8; ++q) pk[q] = 0u;
       }
       // P(n) into buffer b once P.V(n-2) has read it
       if (n >= 2 && !wait_or_abort(&ctl->pv_done[b], ((n >> 1) - 1) & 1, ctl, status)) { ok = false; break; }
-      uint8_t* pb = smem + kOffP + b * kPBytes + (row >> 3) * 512 + (row & 7) * 16 + 2 * ch * 128;
+      uint8_t* pb = smem + kOffP + b * kPBytes + (row >> 3) * kPGroup + (row & 7) * 16 + 2 * kh * kPChunk;
       *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4*>(pb + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      *reinterpret_cast<uint4*>(pb + kPChunk) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       fence_proxy_async_smem();
-      // rescale this thread's 64 O columns once P.V(n-1) has landed (skipped when no row's
-      // max moved in this warp)
+      // rescale this row's O once P.V(n-1) has landed (skipped when no row of the warp moved
+      // its max); the two threads of a row each take 64 of the 128 columns
       if (n >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (!wait_or_abort(&ctl->pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
-          const uint32_t ta = tmem + lane_base + 64 * ch + 32 * cc;
-          tmem_ld32(ta, o);
+          tmem_ld16x64(tmem + lane16 + 64 * cc, o);
           tmem_ld_wait();
 #pragma unroll
           for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(ta, o);
+          tmem_st16x64(tmem + lane16 + 64 * cc, o);
         }
         tmem_st_wait();
       }
       tc_fence_before();
-      mbar_arrive(&ctl->p_full[b]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->p_full[b]);
     }
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);      // the row's total of 448 p
+    if (kh == 0) ctl->xf[0][row] = l_part;
 
     // ------------------------------------------------------------ epilogue
+    // Epilogue mapping (32x32b fragment): warp w holds row 32*(w&3) + lane and owns O columns
+    // 64*(w>>2) .. +63.
     if (ok) ok = wait_or_abort(&ctl->pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1, ctl, status);
     tc_fence_after();
-    // total row sum (of 448 p) from the two column halves
-    ctl->xf[ch][row] = l_part;
     pair_sync(bar_id);
-    const float l448 = l_part + ctl->xf[ch ^ 1][row];
-    const int tok = 128 * pair + row;            // token index within the head
+    const int erow = 32 * quad + lane;
+    const int ch = sub;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
+    const float l448 = ctl->xf[0][erow];
+    const int tok = 128 * pair + erow;           // token index within the head
     const bool store = ok && tok < prm.N;
     const int64_t b_ = bh / prm.q.H, h_ = bh % prm.q.H;
     float den = 0.f;
@@ -460,7 +496,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           dsum = fmaf(__low2float(p2), __uint_as_float(gw[z] << 16), dsum);
           dsum = fmaf(__high2float(p2), __uint_as_float(gw[z] & 0xFFFF0000u), dsum);
         }
-        const uint32_t off = ch * 16384u + sw128_offset(row, uu);
+        const uint32_t off = ch * 16384u + sw128_offset(erow, uu);
         *reinterpret_cast<uint4*>(smem + off) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
       fence_proxy_async_smem();
@@ -470,9 +506,9 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     // normalizer of the linear branch from the two column halves (executed by every softmax
     // thread exactly once, whatever path it took)
-    ctl->xd[ch][row] = den;
+    ctl->xd[ch][erow] = den;
     pair_sync(bar_id);
-    den += ctl->xd[ch ^ 1][row];
+    den += ctl->xd[ch ^ 1][erow];
     if (prm.linear && ok) {
       // wait for this half's phi(Q) . G (rows of a missing second block store nothing)
       if (half == 0 || has_b) {

@@ -330,7 +330,8 @@ k_quant(TensorArg Q, TensorArg K, TensorArg V, int N, int nb, int n_pad, int nbq
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
       const int r = g + 16 * s;
-      *reinterpret_cast<uint2*>(k8 + (row0 + r) * 128 + 8 * ch) = int8_codes(x[s], inv);
+      *reinterpret_cast<uint2*>(k8 + (row0 + k8_row_position(r)) * 128 + 8 * ch) =
+          int8_codes(x[s], inv);
     }
     if (t == 0) sk[bh * nbq + i] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 1.0f;
   }

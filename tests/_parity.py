@@ -60,8 +60,14 @@ def workspace_codes(res, bh: int):
     sk = _ws_slice(ws, lay["sk"] + bh * nbq * 4, nbq, torch.float32)
     s_v = _ws_slice(ws, lay["s_v"] + bh * 128 * 4, 128, torch.float32)
     mu = _ws_slice(ws, lay["mu"] + bh * 128 * 4, 128, torch.float32)
-    return {n: t.cpu().numpy() for n, t in
-            dict(q8=q8, k8=k8, v8=v8, sq=sq, sk=sk, s_v=s_v, mu=mu).items()}
+    res_np = {n: t.cpu().numpy() for n, t in
+              dict(q8=q8, k8=k8, v8=v8, sq=sq, sk=sk, s_v=s_v, mu=mu).items()}
+    # K8 rows are stored key-interleaved inside each 64-key block: key r at row 2(r%32)+r//32
+    r = np.arange(64)
+    perm = 2 * (r % 32) + r // 32
+    k8s = res_np["k8"].reshape(-1, 64, 128)
+    res_np["k8"] = k8s[:, perm, :].reshape(-1, 128)
+    return res_np
 
 
 def kept_sets_from_mask(mask_words: np.ndarray, nb: int) -> list:
@@ -115,14 +121,16 @@ def compare_head(q, k, v, ratio, res, b: int, h: int, rows=None, check_codes=Tru
         np.testing.assert_array_equal(wc["k8"][:N], prep.k8)
         np.testing.assert_array_equal(wc["v8"][:N], orc.e4m3_code(prep.v8))
         assert not wc["q8"][N:].any() and not wc["k8"][N:].any() and not wc["v8"][N:].any()
+    # err: max over elements of |gpu - oracle| minus the bound of what ambiguous P codes
+    # (values within the exp2 approximation error of an e4m3 midpoint) could change
     err = 0.0
     for i, r in out.items():
         sl = orc.block_rows(i, N)
         g = res["out"][b, h, sl].double().numpy()
         assert np.isfinite(g).all(), f"non-finite output in block {i}"
-        err = max(err, float(np.abs(g - r["o"]).max()))
+        err = max(err, float(np.max(np.abs(g - r["o"]) - r["o_s_ambig"])))
         if "sparse" in res:
             gs = res["sparse"][b, h, sl].double().numpy()
             assert np.isfinite(gs).all(), f"non-finite sparse-branch output in block {i}"
-            err = max(err, float(np.abs(gs - r["o_s"]).max()))
+            err = max(err, float(np.max(np.abs(gs - r["o_s"]) - r["o_s_ambig"])))
     return err, ambiguous

@@ -268,9 +268,9 @@ def test_p_code_decision_in_binary32_matches_float64_away_from_midpoints():
     checked = flips = 0
     for trial in range(40):
         s_int = rng.integers(-30000, 30000, size=(64, 64))
-        sq, sk = np.float32(rng.uniform(0.01, 0.05)), np.float32(rng.uniform(0.01, 0.05))
+        sq, sk = np.float32(rng.uniform(0.01, 0.5)), np.float32(rng.uniform(0.01, 0.5))
         m0 = np.full(64, -np.inf, dtype=np.float32)
-        p8, m32 = orc.p_codes_binary32(s_int, sq, sk, m0)
+        p8, m32, _ = orc.p_codes_binary32(s_int, sq, sk, m0)
         s = s_int * (float(sq) * float(sk)) / math.sqrt(128)
         y = 448.0 * np.exp(s - s.max(axis=1, keepdims=True))
         ref = orc.round_e4m3(y)
@@ -282,3 +282,13 @@ def test_p_code_decision_in_binary32_matches_float64_away_from_midpoints():
         # the running maximum is the binary32 image of the row maximum
         np.testing.assert_allclose(m32, s.max(axis=1) * math.log2(math.e), rtol=1e-6)
     assert flips < checked * 1e-3
+
+
+def test_e4m3_ambiguity_bound():
+    """Zero away from midpoints; exactly one grid step at a midpoint."""
+    grid = orc.e4m3_decode(np.arange(0, 127))
+    mids = (grid[:-1] + grid[1:]) / 2
+    amb = orc.e4m3_ambiguity(mids)
+    np.testing.assert_allclose(amb, np.diff(grid))
+    off = orc.e4m3_ambiguity(grid[1:])           # on the grid: unambiguous
+    assert not off.any()

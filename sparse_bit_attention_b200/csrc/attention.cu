@@ -10,26 +10,25 @@
 //     l = e^(m-m') l + sum p;   o = e^(m-m') o + e4m3(448 p) . V8;   m = m'
 //     out = o s_v / (448 l) + phi(q) G_i[:, :128] / phi(q) G_i[:, 128]
 //
-// B200 mapping. One CTA per PAIR of adjacent query blocks (128 rows = the tcgen05 M=128 tile)
-// walking the union of the two blocks' kept lists; rows of a block that does not keep the
-// current key block get P = 0 and skip their softmax work. Warp roles:
-//   warps 0-7  softmax / correction / epilogue: two threads per query row (TMEM lane = row),
-//              warp w exponentiates S columns 32*(w/4) .. +31 (both threads of a row read
-//              all 64 for the block maximum) and owns O columns 64*(w/4) .. +63
-//   warp 8     TMA producer: Q tile once, then K8/V8 tiles through a 4-stage ring
-//   warp 9     MMA issuer: S(n) = Q K_j^T (kind::i8, M128 N64 K128) into one of two S
-//              buffers, then O += P(n-1) V (kind::f8f6f4, M128 N128 K64) — S(n+1) overlaps
-//              the softmax of n.
-// TMEM (256 columns): O fp32 [0,128), S int32 [128,192) and [192,256); after the loop the S
-// columns hold phi(Q) . G for the linear branch. Two CTAs fit on an SM.
+// B200 mapping. One CTA holds two query blocks ("halves"). Each half runs its own pipeline
+// over its own k kept blocks with M=64 tcgen05 MMAs: an M=64 result occupies TMEM lanes
+// 0-15 of each 32-lane quadrant, and a lane offset of 16 in the D address puts the second
+// half in lanes 16-31, so both halves share the TMEM columns (O fp32 [0,128); S int32 in two
+// buffers [128,192), [192,256); the linear branch reuses the S columns at the end).
+//   warps 0-3 / 4-7  softmax, correction and epilogue of half 0 / half 1 (16 rows per warp,
+//                    two threads per row through the 16x64b TMEM fragment)
+//   warp 8           TMA producer for both halves (non-blocking event loop)
+//   warp 9           MMA issuer for both halves (non-blocking event loop)
+// Each half owns a private 52 KB of shared memory (its Q rows, a 2-stage K8/V8 ring and two
+// P tiles), reused for the linear-branch operands once its main loop is done.
 //
 // Softmax arithmetic per score: the int32 score becomes a float exactly through the 1.5*2^23
-// bias (integer add, float subtract: no conversion-pipe instruction); one FFMA forms the
-// base-2 exponent with the factor 448 of the P quantization folded in; 2^x comes from the
-// MUFU ex2 unit for most columns and, for the rest, from Cody-Waite range reduction (round
-// to nearest integer) plus a degree-5 polynomial fitted here by the Remez exchange algorithm
-// for minimax relative error on [-1/2, 1/2] (max relative error 2.3e-7 in fp32), so that the
-// FMA pipe takes part of the exponential load of the MUFU unit.
+// bias (integer add, then a packed f32x2 subtract: no conversion-pipe instruction); one packed
+// FFMA forms the base-2 exponent with the factor 448 of the P quantization folded in; 2^x
+// comes from the MUFU ex2 unit for most columns and, for the rest, from Cody-Waite range
+// reduction (round to nearest integer) plus a degree-5 polynomial fitted here by the Remez
+// exchange algorithm for minimax relative error on [-1/2, 1/2] (max relative error 2.3e-7 in
+// fp32), so that the FMA pipe takes part of the exponential load of the MUFU unit.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -39,24 +38,27 @@ namespace sagesla {
 
 namespace {
 
-constexpr int kNS = 4;                       // K/V ring stages
-constexpr int kSoftmaxWarps = 8;
+constexpr int kNS = 2;                       // K/V ring stages per half
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 320;
-constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-constexpr uint32_t kQBytes = 128 * 128;      // int8 Q tile
 constexpr uint32_t kKVBytes = 64 * 128;      // one K8 or V8 tile
 constexpr uint32_t kStageBytes = 2 * kKVBytes;
-// e4m3 P tile, K-major without swizzle: core matrices of 8 rows x 16 keys (128 B); K-chunks
-// 160 B apart and 8-row groups 672 B apart. The padding makes the 16-byte stores of the
-// softmax threads (lanes of one store phase hold rows r, r+8, r+1, r+9 and key halves 0, 1)
-// fall on eight distinct bank groups.
+// e4m3 P tile of one half (64 rows), K-major without swizzle: core matrices of 8 rows x 16
+// keys (128 B); K-chunks 160 B apart and 8-row groups 672 B apart. The padding makes the
+// 16-byte stores of the softmax threads (one store phase holds rows r, r+8, r+1, r+9 and key
+// halves 0, 1) fall on eight distinct bank groups.
 constexpr uint32_t kPChunk = 160, kPGroup = 672;
-constexpr uint32_t kPBytes = 16 * kPGroup;
-constexpr uint32_t kOffStages = kQBytes;
-constexpr uint32_t kOffP = kOffStages + kNS * kStageBytes;
-constexpr uint32_t kOffCtl = kOffP + 2 * kPBytes;
-static_assert(kOffCtl >= 96 * 1024, "the linear epilogue reuses [0, 96 KB) for its operands");
+constexpr uint32_t kPBytes = 8 * kPGroup;
+// Per-half private region.
+constexpr uint32_t kHQ = 0;                  // the half's 64 Q8 rows (SW128), 8 KB
+constexpr uint32_t kHStages = 8192;
+constexpr uint32_t kHP = kHStages + kNS * kStageBytes;
+constexpr uint32_t kHalfBytes = 53248;
+constexpr uint32_t kHLinA = 0;               // epilogue: phi(Q) bf16, 2 x [64][128 B]
+constexpr uint32_t kHLinG = 16384;           // epilogue: G_i bf16, 2 x [128][128 B]
+static_assert(kHP + 2 * kPBytes <= kHalfBytes, "half region");
+static_assert(kHLinG + 32768 <= kHalfBytes, "linear operands fit in the half region");
+constexpr uint32_t kOffCtl = 2 * kHalfBytes;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemS = 128;              // first S buffer column
 // Columns of each thread's 32 whose exponential uses the polynomial instead of MUFU ex2.
@@ -65,23 +67,24 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kInvSqrtD = 0.08838834764831845f;
 constexpr float kLog2_448 = 8.807354922057604f;
 
-struct Ctl {
+struct HalfCtl {
   uint64_t full[kNS], empty[kNS];
   uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
-  uint64_t q_full, g_full, a_full, la_done, la_free, lb_done, mma_done;
+  uint64_t q_full, g_full, a_full, l_done, mma_done;
+};
+
+struct Ctl {
+  HalfCtl hc[2];
   uint32_t tmem_base;
-  int list_len;
   volatile int abort;
   float s_v[128];
-  float xf[2][128];          // [column half][row]: epilogue exchanges
-  float xd[2][128];
 };
 
 struct AttnParams {
   const float* sq;            // [BH][nbq]
   const float* sk;            // [BH][nbq]
   const float* s_v;           // [BH][128]
-  const uint32_t* mask;       // [BH][nb][mask_words]
+  const int32_t* kept;        // [BH][nb][k]
   const __nv_bfloat16* gsum;  // [BH][nb_m_pad][129][128]
   TensorArg q;                // raw bf16 Q (for phi(q))
   void* out;
@@ -89,7 +92,7 @@ struct AttnParams {
   int32_t out_dtype;
   float* sparse_out;          // optional [BH][N][128]
   int* status;
-  int N, nb, nbq, n_pad, mask_words, nb_m_pad, n_last, list_cap;
+  int N, nb, nbq, n_pad, k, nb_m_pad, n_last;
   int linear;                 // 0 when every key block is kept
 };
 
@@ -103,11 +106,51 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ct
   return true;
 }
 
-// Named barrier for the two warps (64 threads) that share a group of 32 rows. Used only in
-// the epilogue, where both threads of a row execute it the same number of times on every
-// path (a named barrier cannot time out).
-__device__ __forceinline__ void pair_sync(int id) {
-  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+// Idle-time bookkeeping of the event loops: gives up (status TIMEOUT, abort) once no progress
+// was made for kSpinLimitNs.
+struct Watchdog {
+  unsigned long long since = 0;
+  int idle = 0;
+  __device__ __forceinline__ bool expired(Ctl* ctl, int* status) {
+    if (ctl->abort) return true;
+    if (++idle < 256) return false;
+    idle = 0;
+    const unsigned long long now = global_timer_ns();
+    if (since == 0) since = now;
+    if (now - since > kSpinLimitNs) {
+      record_error(status, SAGESLA_ERR_TIMEOUT);
+      ctl->abort = 1;
+      return true;
+    }
+    return false;
+  }
+  __device__ __forceinline__ void reset() { since = 0; idle = 0; }
+};
+
+// ---------------------------------------------------------------- packed f32x2 arithmetic
+__device__ __forceinline__ unsigned long long pk2(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void up2(unsigned long long v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
 // int32 -> float, exact for |s| < 2^22 (the INT8 product of a 128-channel row is < 2^21).
@@ -121,19 +164,28 @@ __device__ __forceinline__ float ex2_mufu(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe: x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f by a degree-5
-// minimax polynomial (coefficients from a Remez fit of relative error); 2^n added to the
-// exponent field. x is clamped below at -125 so that the result stays a normal float.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;              // rint(x) in the low mantissa bits
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.0013276472454890609f, f, 0.009675540961325169f);
-  p = fmaf(p, f, 0.05550713092088699f);
-  p = fmaf(p, f, 0.24022120237350464f);
-  p = fmaf(p, f, 0.6931469440460205f);
-  p = fmaf(p, f, 1.0000001192092896f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// 2^x on the FMA pipe for two values: x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f by a
+// degree-5 minimax polynomial (coefficients from a Remez fit of relative error); 2^n added
+// to the exponent field. x is clamped below at -125 so that the result stays a normal float.
+__device__ __forceinline__ unsigned long long ex2_poly2(unsigned long long x2) {
+  float x0, x1;
+  up2(x2, x0, x1);
+  x2 = pk2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const unsigned long long magic = pk2(12582912.0f, 12582912.0f);
+  const unsigned long long t = add2(x2, magic);                 // rint(x) in low mantissa bits
+  const unsigned long long f = fma2(add2(t, pk2(-12582912.0f, -12582912.0f)),
+                                    pk2(-1.0f, -1.0f), x2);     // x - rint(x)
+  unsigned long long p = fma2(pk2(0.0013276472454890609f, 0.0013276472454890609f), f,
+                              pk2(0.009675540961325169f, 0.009675540961325169f));
+  p = fma2(p, f, pk2(0.05550713092088699f, 0.05550713092088699f));
+  p = fma2(p, f, pk2(0.24022120237350464f, 0.24022120237350464f));
+  p = fma2(p, f, pk2(0.6931469440460205f, 0.6931469440460205f));
+  p = fma2(p, f, pk2(1.0000001192092896f, 1.0000001192092896f));
+  float p0, p1, t0, t1;
+  up2(p, p0, p1);
+  up2(t, t0, t1);
+  return pk2(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+             __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
 }
 
 // Maximum of this thread's valid scores (eight independent chains).
@@ -153,25 +205,40 @@ __device__ __forceinline__ int row_block_max(const uint32_t (&a)[32], int valid)
 template <bool kFull>
 __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int valid, float c,
                                               float neg, uint32_t (&pk)[8]) {
-  float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+  const unsigned long long c2 = pk2(c, c), neg2 = pk2(neg, neg);
+  const unsigned long long unbias = pk2(-12582912.0f, -12582912.0f);
+  unsigned long long acc0 = pk2(0.f, 0.f), acc1 = pk2(0.f, 0.f);
 #pragma unroll
   for (int q = 0; q < 32; q += 4) {
     float y[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const float x = fmaf(s32_to_f32(sr[q + t]), c, neg);
-      float v = (q + t < kPolyFrom) ? ex2_mufu(x) : ex2_poly(x);
-      if (!kFull && q + t >= valid) v = 0.f;
-      y[t] = v;
+    for (int t = 0; t < 4; t += 2) {
+      const unsigned long long f2 = add2(
+          pk2(__int_as_float(static_cast<int>(sr[q + t] + 0x4B400000u)),
+              __int_as_float(static_cast<int>(sr[q + t + 1] + 0x4B400000u))),
+          unbias);
+      const unsigned long long x2 = fma2(f2, c2, neg2);
+      if (q + t < kPolyFrom) {
+        float x0, x1;
+        up2(x2, x0, x1);
+        y[t] = ex2_mufu(x0);
+        y[t + 1] = ex2_mufu(x1);
+      } else {
+        up2(ex2_poly2(x2), y[t], y[t + 1]);
+      }
+      if (!kFull) {
+        if (q + t >= valid) y[t] = 0.f;
+        if (q + t + 1 >= valid) y[t + 1] = 0.f;
+      }
     }
-    r0 += y[0];
-    r1 += y[1];
-    r2 += y[2];
-    r3 += y[3];
+    acc0 = add2(acc0, pk2(y[0], y[1]));
+    acc1 = add2(acc1, pk2(y[2], y[3]));
     pk[q >> 2] = static_cast<uint32_t>(f32x2_to_e4m3x2(y[0], y[1])) |
                  (static_cast<uint32_t>(f32x2_to_e4m3x2(y[2], y[3])) << 16);
   }
-  return (r0 + r1) + (r2 + r3);
+  float a, b;
+  up2(add2(acc0, acc1), a, b);
+  return a + b;
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -182,66 +249,37 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + kOffCtl);
-  uint32_t* list = reinterpret_cast<uint32_t*>(smem + kOffCtl + sizeof(Ctl));
-  float* list_sk = reinterpret_cast<float*>(list + prm.list_cap);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x;
   const int64_t bh = blockIdx.y;
-  const int ia = 2 * pair, ib = 2 * pair + 1;     // the two query blocks
+  const int ia = 2 * pair;                        // first query block of the CTA
   int* status = prm.status;
+  int U[2];
+  U[0] = prm.k;
+  U[1] = (ia + 1 < prm.nb) ? prm.k : 0;           // the last pair may hold a single block
 
   if (warp == 0) {
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
-    // union of the two kept lists, ascending; flags bit0 = kept by ia, bit1 = kept by ib
-    const uint32_t* ma = prm.mask + (bh * prm.nb + ia) * prm.mask_words;
-    const uint32_t* mb = ib < prm.nb ? prm.mask + (bh * prm.nb + ib) * prm.mask_words : nullptr;
-    int base = 0;
-    for (int w0 = 0; w0 < prm.mask_words; w0 += 32) {
-      const int w = w0 + lane;
-      const uint32_t a = w < prm.mask_words ? ma[w] : 0u;
-      const uint32_t b = (w < prm.mask_words && mb) ? mb[w] : 0u;
-      uint32_t u = a | b;
-      const int cnt = __popc(u);
-      int incl = cnt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int nv = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += nv;
-      }
-      int pos = base + incl - cnt;
-      while (u) {
-        const int bit = __ffs(u) - 1;
-        u &= u - 1;
-        const int j = 32 * w + bit;
-        const uint32_t fl = ((a >> bit) & 1u) | (((b >> bit) & 1u) << 1);
-        if (pos < prm.list_cap) {
-          list[pos] = static_cast<uint32_t>(j) | (fl << 24);
-          list_sk[pos] = prm.sk[bh * prm.nbq + j];
-        }
-        ++pos;
-      }
-      base += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) ctl->list_len = min(base, prm.list_cap);
   } else if (warp == 1) {
     for (int c = lane; c < 128; c += 32) ctl->s_v[c] = prm.s_v[bh * 128 + c];
   } else if (threadIdx.x == 64) {
-    for (int s = 0; s < kNS; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&ctl->s_full[s], 1);
-      mbar_init(&ctl->s_free[s], kSoftmaxWarps);
-      mbar_init(&ctl->p_full[s], kSoftmaxWarps);
-      mbar_init(&ctl->pv_done[s], 1);
+    for (int h = 0; h < 2; ++h) {
+      HalfCtl& c = ctl->hc[h];
+      for (int s = 0; s < kNS; ++s) { mbar_init(&c.full[s], 1); mbar_init(&c.empty[s], 1); }
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(&c.s_full[s], 1);
+        mbar_init(&c.s_free[s], 4);
+        mbar_init(&c.p_full[s], 4);
+        mbar_init(&c.pv_done[s], 1);
+      }
+      mbar_init(&c.q_full, 1);
+      mbar_init(&c.g_full, 1);
+      mbar_init(&c.a_full, 4);
+      mbar_init(&c.l_done, 1);
+      mbar_init(&c.mma_done, 1);
     }
-    mbar_init(&ctl->q_full, 1);
-    mbar_init(&ctl->g_full, 1);
-    mbar_init(&ctl->a_full, kSoftmaxThreads);
-    mbar_init(&ctl->la_done, 1);
-    mbar_init(&ctl->la_free, kSoftmaxThreads / 2);
-    mbar_init(&ctl->lb_done, 1);
-    mbar_init(&ctl->mma_done, 1);
     ctl->abort = 0;
     fence_mbar_init();
   } else if (threadIdx.x == 96) {
@@ -251,217 +289,240 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const int U = ctl->list_len;
-  const bool has_b = ib < prm.nb;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int row_base = static_cast<int>(bh * prm.n_pad);
-      mbar_arrive_expect_tx(&ctl->q_full, kQBytes);
-      tma_load_2d(smem, &tm_q, &ctl->q_full, 0, row_base + 128 * pair);
-      for (int n = 0; n < U; ++n) {
-        const int s = n % kNS;
-        if (n >= kNS && !wait_or_abort(&ctl->empty[s], ((n / kNS) - 1) & 1, ctl, status)) break;
-        const int j = static_cast<int>(list[n] & 0xFFFFFFu);
-        uint8_t* st = smem + kOffStages + s * kStageBytes;
-        mbar_arrive_expect_tx(&ctl->full[s], kStageBytes);
-        tma_load_2d(st, &tm_k, &ctl->full[s], 0, row_base + 64 * j);
-        tma_load_2d(st + kKVBytes, &tm_v, &ctl->full[s], 0, row_base + 64 * j);
+      for (int h = 0; h < 2; ++h) {
+        if (U[h] == 0) continue;
+        mbar_arrive_expect_tx(&ctl->hc[h].q_full, 8192u);
+        tma_load_2d(smem + h * kHalfBytes + kHQ, &tm_q, &ctl->hc[h].q_full, 0,
+                    row_base + 128 * pair + 64 * h);
       }
-      // A parity wait only tells the last two phases apart, and this thread has not observed
-      // the earlier P.V phases, so it waits on the single-phase "all MMAs of the loop done".
-      if (prm.linear && wait_or_abort(&ctl->mma_done, 0, ctl, status)) {
-        // The whole operand area is free now: G_ia -> [32K, 64K), G_ib -> [64K, 96K).
-        const int gy = static_cast<int>((bh * prm.nb_m_pad + ia) * 129);
-        mbar_arrive_expect_tx(&ctl->g_full, has_b ? 65536u : 32768u);
-        tma_load_2d(smem + 32768, &tm_g, &ctl->g_full, 0, gy);
-        tma_load_2d(smem + 32768 + 16384, &tm_g, &ctl->g_full, 64, gy);
-        if (has_b) {
-          tma_load_2d(smem + 65536, &tm_g, &ctl->g_full, 0, gy + 129);
-          tma_load_2d(smem + 65536 + 16384, &tm_g, &ctl->g_full, 64, gy + 129);
+      int ld[2] = {0, 0};
+      bool gdone[2] = {U[0] == 0 || !prm.linear, U[1] == 0 || !prm.linear};
+      Watchdog wd;
+      while (true) {
+        bool pending = false, progress = false;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          HalfCtl& c = ctl->hc[h];
+          uint8_t* hb = smem + h * kHalfBytes;
+          if (ld[h] < U[h]) {
+            pending = true;
+            const int n = ld[h], s = n % kNS;
+            if (n < kNS || mbar_test(&c.empty[s], ((n / kNS) - 1) & 1)) {
+              const int j = __ldg(prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) + n);
+              uint8_t* st = hb + kHStages + s * kStageBytes;
+              mbar_arrive_expect_tx(&c.full[s], kStageBytes);
+              tma_load_2d(st, &tm_k, &c.full[s], 0, row_base + 64 * j);
+              tma_load_2d(st + kKVBytes, &tm_v, &c.full[s], 0, row_base + 64 * j);
+              ++ld[h];
+              progress = true;
+            }
+          } else if (!gdone[h]) {
+            // A parity wait only tells the last two phases apart and this thread has not
+            // observed the P.V phases, so it waits on the single-phase "loop MMAs done".
+            pending = true;
+            if (mbar_test(&c.mma_done, 0)) {
+              const int gy = static_cast<int>((bh * prm.nb_m_pad + ia + h) * 129);
+              mbar_arrive_expect_tx(&c.g_full, 32768u);
+              tma_load_2d(hb + kHLinG, &tm_g, &c.g_full, 0, gy);
+              tma_load_2d(hb + kHLinG + 16384, &tm_g, &c.g_full, 64, gy);
+              gdone[h] = true;
+              progress = true;
+            }
+          }
         }
+        if (!pending) break;
+        if (progress) wd.reset();
+        else if (wd.expired(ctl, status)) break;
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = make_idesc(kFmtS32, kFmtS8, kFmtS8, 0, 0, 128, 64);
-      constexpr uint32_t idesc_pv = make_idesc(kFmtF32, kFmtE4M3, kFmtE4M3, 0, 1, 128, 128);
-      const uint32_t q_addr = smem_u32(smem);
-      auto issue_pv = [&](int m) -> bool {
-        const int b = m & 1;
-        if (!wait_or_abort(&ctl->p_full[b], (m >> 1) & 1, ctl, status)) return false;
-        tc_fence_after();
-        const uint32_t p_addr = smem_u32(smem + kOffP + b * kPBytes);
-        const uint32_t v_addr = smem_u32(smem + kOffStages + (m % kNS) * kStageBytes + kKVBytes);
+      constexpr uint32_t idesc_s = make_idesc(kFmtS32, kFmtS8, kFmtS8, 0, 0, 64, 64);
+      constexpr uint32_t idesc_pv = make_idesc(kFmtF32, kFmtE4M3, kFmtE4M3, 0, 1, 64, 128);
+      constexpr uint32_t idesc_l = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 64, 128);
+      bool ok = true;
+      for (int h = 0; h < 2 && ok; ++h)
+        if (U[h] > 0) ok = wait_or_abort(&ctl->hc[h].q_full, 0, ctl, status);
+      int sn[2] = {0, 0}, pn[2] = {0, 0};
+      bool lin[2] = {U[0] == 0 || !prm.linear, U[1] == 0 || !prm.linear};
+      Watchdog wd;
+      while (ok) {
+        bool pending = false, progress = false;
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {   // 2 x K=32 keys
-          // P: K-major, no swizzle (layout above). V: MN-major (d contiguous), 128-byte
-          // swizzle, 8-key groups 1024 B apart.
-          const uint64_t ad = make_sdesc(p_addr + kk * 2 * kPChunk, kPChunk, kPGroup, kLayoutNone);
-          const uint64_t bd = make_sdesc(v_addr + kk * 4096, 8192, 1024, kLayoutSW128);
-          mma_f8(tmem, ad, bd, idesc_pv, (m > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&ctl->pv_done[b]);
-        mma_commit(&ctl->empty[m % kNS]);
-        return true;
-      };
-      bool ok = wait_or_abort(&ctl->q_full, 0, ctl, status);
-      for (int n = 0; n < U && ok; ++n) {
-        const int s = n % kNS, b = n & 1;
-        if (!wait_or_abort(&ctl->full[s], (n / kNS) & 1, ctl, status)) { ok = false; break; }
-        if (n >= 2 && !wait_or_abort(&ctl->s_free[b], ((n >> 1) - 1) & 1, ctl, status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + kOffStages + s * kStageBytes);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {   // 4 x K=32 channels
-          const uint64_t ad = make_sdesc(q_addr + kk * 32, 16, 1024, kLayoutSW128);
-          const uint64_t bd = make_sdesc(k_addr + kk * 32, 16, 1024, kLayoutSW128);
-          mma_i8(tmem + kTmemS + 64 * b, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&ctl->s_full[b]);
-        if (n >= 1 && !issue_pv(n - 1)) { ok = false; break; }
-      }
-      if (ok && U >= 1) ok = issue_pv(U - 1);
-      mma_commit(&ctl->mma_done);
-      if (ok && prm.linear) {
-        // phi(Q) . G_ia into the S columns, then (after rows 0-63 read it) phi(Q) . G_ib.
-        constexpr uint32_t idesc_l = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 128, 128);
-        ok = wait_or_abort(&ctl->a_full, 0, ctl, status) &&
-             wait_or_abort(&ctl->g_full, 0, ctl, status);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem);
-          for (int half = 0; half < (has_b ? 2 : 1) && ok; ++half) {
-            if (half == 1) {
-              ok = wait_or_abort(&ctl->la_free, 0, ctl, status);
-              if (!ok) break;
+        for (int h = 0; h < 2; ++h) {
+          HalfCtl& c = ctl->hc[h];
+          const uint32_t hb = smem_u32(smem + h * kHalfBytes);
+          const uint32_t dlane = static_cast<uint32_t>(16 * h) << 16;
+          if (pn[h] < U[h]) {
+            pending = true;
+            const int n = sn[h];
+            if (n < U[h] && mbar_test(&c.full[n % kNS], (n / kNS) & 1) &&
+                (n < 2 || mbar_test(&c.s_free[n & 1], ((n >> 1) - 1) & 1))) {
               tc_fence_after();
-            }
-            const uint32_t g_addr = smem_u32(smem + 32768 + half * 32768);
+              const uint32_t k_addr = hb + kHStages + (n % kNS) * kStageBytes;
 #pragma unroll
-            for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = make_sdesc(a_addr + kc * 16384 + kk * 32, 16, 1024, kLayoutSW128);
-                const uint64_t bd = make_sdesc(g_addr + kc * 16384 + kk * 32, 16, 1024, kLayoutSW128);
-                mma_bf16(tmem + kTmemS, ad, bd, idesc_l, (kc | kk) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {   // 4 x K=32 channels
+                const uint64_t ad = make_sdesc(hb + kHQ + kk * 32, 16, 1024, kLayoutSW128);
+                const uint64_t bd = make_sdesc(k_addr + kk * 32, 16, 1024, kLayoutSW128);
+                mma_i8(tmem + dlane + kTmemS + 64 * (n & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
               }
-            mma_commit(half == 0 ? &ctl->la_done : &ctl->lb_done);
+              mma_commit(&c.s_full[n & 1]);
+              ++sn[h];
+              progress = true;
+            }
+            const int m = pn[h];
+            if (m < sn[h] && mbar_test(&c.p_full[m & 1], (m >> 1) & 1)) {
+              tc_fence_after();
+              const uint32_t p_addr = hb + kHP + (m & 1) * kPBytes;
+              const uint32_t v_addr = hb + kHStages + (m % kNS) * kStageBytes + kKVBytes;
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk) {   // 2 x K=32 keys
+                // P: K-major, no swizzle (layout above). V: MN-major (d contiguous),
+                // 128-byte swizzle, 8-key groups 1024 B apart.
+                const uint64_t ad = make_sdesc(p_addr + kk * 2 * kPChunk, kPChunk, kPGroup, kLayoutNone);
+                const uint64_t bd = make_sdesc(v_addr + kk * 4096, 8192, 1024, kLayoutSW128);
+                mma_f8(tmem + dlane, ad, bd, idesc_pv, (m > 0 || kk > 0) ? 1u : 0u);
+              }
+              mma_commit(&c.pv_done[m & 1]);
+              mma_commit(&c.empty[m % kNS]);
+              ++pn[h];
+              if (pn[h] == U[h]) mma_commit(&c.mma_done);
+              progress = true;
+            }
+          } else if (!lin[h]) {
+            // phi(Q_i) . G_i into this half's S columns
+            pending = true;
+            if (mbar_test(&c.a_full, 0) && mbar_test(&c.g_full, 0)) {
+              tc_fence_after();
+#pragma unroll
+              for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t ad = make_sdesc(hb + kHLinA + kc * 8192 + kk * 32, 16, 1024, kLayoutSW128);
+                  const uint64_t bd = make_sdesc(hb + kHLinG + kc * 16384 + kk * 32, 16, 1024, kLayoutSW128);
+                  mma_bf16(tmem + dlane + kTmemS, ad, bd, idesc_l, (kc | kk) ? 1u : 0u);
+                }
+              mma_commit(&c.l_done);
+              lin[h] = true;
+              progress = true;
+            }
           }
         }
+        if (!pending) break;
+        if (progress) wd.reset();
+        else if (wd.expired(ctl, status)) break;
       }
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    // Loop mapping (16x64b TMEM fragment): warp w reads lanes 32*(w&3) + 16*(w>>2) + 0..15;
-    // lane t holds row lrow = t/4 + 8*(t&1) and key half p = (t>>1)&1, i.e. keys 32p..32p+31
-    // of the block (the K8 rows are stored key-interleaved). Lanes t and t^2 share a row.
+    // Warp w serves half h = w/4 and reads TMEM lanes 32*(w&3) + 16h + 0..15 (16x64b
+    // fragment): lane t holds row r = 16*(w&3) + t/4 + 8*(t&1) of the half's query block and
+    // key half kh = (t>>1)&1, i.e. keys 32kh..32kh+31 of the block (the K8 rows are stored
+    // key-interleaved). Lanes t and t^2 share a row.
+    const int h = warp >> 2;
     const int quad = warp & 3;
-    const int sub = warp >> 2;
-    const int row = 32 * quad + 16 * sub + (lane >> 2) + 8 * (lane & 1);   // 0..127
-    const int kh = (lane >> 1) & 1;              // key half
-    const int half = row >> 6;                   // 0: block ia, 1: block ib (warp-uniform)
-    const uint32_t my_bit = 1u << half;
-    const int qblock = ia + half;
-    const int bar_id = 1 + quad;                 // named barrier of warps quad, quad + 4
-    const float cs = prm.sq[bh * prm.nbq + qblock] * (kLog2e * kInvSqrtD);
-    const uint32_t lane16 = static_cast<uint32_t>(32 * quad + 16 * sub) << 16;
+    HalfCtl& c = ctl->hc[h];
+    uint8_t* hbase = smem + h * kHalfBytes;
+    const int r = 16 * quad + (lane >> 2) + 8 * (lane & 1);    // row within the block
+    const int kh = (lane >> 1) & 1;
+    const int qblock = ia + h;
+    const int Uh = U[h];
+    const uint32_t lane16 = static_cast<uint32_t>(32 * quad + 16 * h) << 16;
     const int valid = prm.n_last - 32 * kh;      // valid keys of this thread in the last block
+    bool ok = Uh > 0;
     float m_run = -INFINITY, l_part = 0.f;
-    bool ok = true;
-    for (int n = 0; n < U; ++n) {
-      const int b = n & 1;
-      const uint32_t e = list[n];
-      const int j = static_cast<int>(e & 0xFFFFFFu);
-      const bool mine = ((e >> 24) & my_bit) != 0;     // warp-uniform
-      if (!wait_or_abort(&ctl->s_full[b], (n >> 1) & 1, ctl, status)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t pk[8];
-      float alpha = 1.f;
-      if (mine) {
+    if (ok) {
+      const float cs = prm.sq[bh * prm.nbq + qblock] * (kLog2e * kInvSqrtD);
+      const int32_t* klist = prm.kept + (bh * prm.nb + qblock) * static_cast<int64_t>(prm.k);
+      const float* skh = prm.sk + bh * prm.nbq;
+      int j_next = __ldg(klist);
+      float sk_next = __ldg(skh + j_next);
+      for (int n = 0; n < Uh; ++n) {
+        const int b = n & 1;
+        const int j = j_next;
+        const float skj = sk_next;
+        if (n + 1 < Uh) {                        // prefetch the next kept block's scale
+          j_next = __ldg(klist + n + 1);
+          sk_next = __ldg(skh + j_next);
+        }
+        if (!wait_or_abort(&c.s_full[b], (n >> 1) & 1, ctl, status)) { ok = false; break; }
+        tc_fence_after();
         uint32_t sr[32];
         tmem_ld16x64(tmem + lane16 + kTmemS + 64 * b, sr);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->s_free[b]);
+        if (lane == 0) mbar_arrive(&c.s_free[b]);
         const bool full = j != prm.nb - 1 || prm.n_last == 64;   // no padded keys
         int mxi = full ? row_block_max<true>(sr, 32) : row_block_max<false>(sr, valid);
         mxi = max(mxi, __shfl_xor_sync(0xffffffffu, mxi, 2));
-        const float c = cs * list_sk[n];
-        const float m_new = fmaxf(m_run, s32_to_f32(static_cast<uint32_t>(mxi)) * c);
-        alpha = ex2_mufu(m_run - m_new);
-        const float neg = kLog2_448 - m_new;      // 2^(S c + neg) = 448 p
-        const float rs = full ? row_exp_pack<true>(sr, 32, c, neg, pk)
-                              : row_exp_pack<false>(sr, valid, c, neg, pk);
+        const float cst = cs * skj;
+        const float m_new = fmaxf(m_run, s32_to_f32(static_cast<uint32_t>(mxi)) * cst);
+        const float alpha = ex2_mufu(m_run - m_new);
+        const float neg = kLog2_448 - m_new;    // 2^(S c + neg) = 448 p
+        uint32_t pk[8];
+        const float rs = full ? row_exp_pack<true>(sr, 32, cst, neg, pk)
+                              : row_exp_pack<false>(sr, valid, cst, neg, pk);
         l_part = alpha * l_part + rs;
         m_run = m_new;
-      } else {
+        // P(n) into buffer b once P.V(n-2) has read it
+        if (n >= 2 && !wait_or_abort(&c.pv_done[b], ((n >> 1) - 1) & 1, ctl, status)) { ok = false; break; }
+        uint8_t* pb = hbase + kHP + b * kPBytes + (r >> 3) * kPGroup + (r & 7) * 16 + 2 * kh * kPChunk;
+        *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(pb + kPChunk) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        fence_proxy_async_smem();
+        // rescale this row's O once P.V(n-1) has landed (skipped when no row of the warp
+        // moved its max); the two threads of a row each take 64 of the 128 columns
+        if (n >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (!wait_or_abort(&c.pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status)) { ok = false; break; }
+          tc_fence_after();
+          const unsigned long long a2 = pk2(alpha, alpha);
+#pragma unroll 1
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t o[32];
+            tmem_ld16x64(tmem + lane16 + 64 * cc, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 32; q += 2) {
+              float x0, x1;
+              up2(mul2(pk2(__uint_as_float(o[q]), __uint_as_float(o[q + 1])), a2), x0, x1);
+              o[q] = __float_as_uint(x0);
+              o[q + 1] = __float_as_uint(x1);
+            }
+            tmem_st16x64(tmem + lane16 + 64 * cc, o);
+          }
+          tmem_st_wait();
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->s_free[b]);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) pk[q] = 0u;
+        if (lane == 0) mbar_arrive(&c.p_full[b]);
       }
-      // P(n) into buffer b once P.V(n-2) has read it
-      if (n >= 2 && !wait_or_abort(&ctl->pv_done[b], ((n >> 1) - 1) & 1, ctl, status)) { ok = false; break; }
-      uint8_t* pb = smem + kOffP + b * kPBytes + (row >> 3) * kPGroup + (row & 7) * 16 + 2 * kh * kPChunk;
-      *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4*>(pb + kPChunk) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-      fence_proxy_async_smem();
-      // rescale this row's O once P.V(n-1) has landed (skipped when no row of the warp moved
-      // its max); the two threads of a row each take 64 of the 128 columns
-      if (n >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!wait_or_abort(&ctl->pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t o[32];
-          tmem_ld16x64(tmem + lane16 + 64 * cc, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st16x64(tmem + lane16 + 64 * cc, o);
-        }
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->p_full[b]);
+      if (ok) ok = wait_or_abort(&c.pv_done[(Uh - 1) & 1], ((Uh - 1) >> 1) & 1, ctl, status);
+      tc_fence_after();
     }
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);      // the row's total of 448 p
-    if (kh == 0) ctl->xf[0][row] = l_part;
 
     // ------------------------------------------------------------ epilogue
-    // Epilogue mapping (32x32b fragment): warp w holds row 32*(w&3) + lane and owns O columns
-    // 64*(w>>2) .. +63.
-    if (ok) ok = wait_or_abort(&ctl->pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1, ctl, status);
-    tc_fence_after();
-    pair_sync(bar_id);
-    const int erow = 32 * quad + lane;
-    const int ch = sub;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
-    const float l448 = ctl->xf[0][erow];
-    const int tok = 128 * pair + erow;           // token index within the head
-    const bool store = ok && tok < prm.N;
+    const float l448 = l_part + __shfl_xor_sync(0xffffffffu, l_part, 2);   // row total of 448 p
+    const int tok = 64 * qblock + r;             // token index within the head
     const int64_t b_ = bh / prm.q.H, h_ = bh % prm.q.H;
     float den = 0.f;
     if (prm.linear && ok) {
-      // phi(q) for this row; this thread writes channels 64ch .. 64ch+63 of the A operand
-      // (bf16, K-major, 128-byte swizzle) and sums its part of the normalizer.
+      // phi(q) of this row: the thread writes channels 64kh .. 64kh+63 (chunk kh) of the A
+      // operand (bf16, K-major, 128-byte swizzle) and sums its part of the normalizer.
       const uint16_t* qrow = static_cast<const uint16_t*>(prm.q.data) + b_ * prm.q.stride_b +
                              h_ * prm.q.stride_h + static_cast<int64_t>(min(tok, prm.N - 1)) * prm.q.stride_n;
       const uint4* q4 = reinterpret_cast<const uint4*>(qrow);
       float mx = -INFINITY;
 #pragma unroll 4
       for (int u = 0; u < 16; ++u) {
-        const uint4 r = __ldg(q4 + u);
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+        const uint4 rr = __ldg(q4 + u);
+        const uint32_t w[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
         for (int z = 0; z < 4; ++z)
           mx = fmaxf(mx, fmaxf(__uint_as_float(w[z] << 16), __uint_as_float(w[z] & 0xFFFF0000u)));
@@ -469,8 +530,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       float sum = 0.f;
 #pragma unroll 4
       for (int u = 0; u < 16; ++u) {
-        const uint4 r = __ldg(q4 + u);
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+        const uint4 rr = __ldg(q4 + u);
+        const uint32_t w[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
         for (int z = 0; z < 4; ++z)
           sum += __expf(__uint_as_float(w[z] << 16) - mx) + __expf(__uint_as_float(w[z] & 0xFFFF0000u) - mx);
@@ -481,10 +542,10 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       float dsum = 0.f;
 #pragma unroll 2
       for (int uu = 0; uu < 8; ++uu) {
-        const int u = 8 * ch + uu;
-        const uint4 r = __ldg(q4 + u);
+        const int u = 8 * kh + uu;
+        const uint4 rr = __ldg(q4 + u);
         const uint4 gg = __ldg(g128 + u);
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+        const uint32_t w[4] = {rr.x, rr.y, rr.z, rr.w};
         const uint32_t gw[4] = {gg.x, gg.y, gg.z, gg.w};
         uint32_t packed[4];
 #pragma unroll
@@ -496,73 +557,68 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           dsum = fmaf(__low2float(p2), __uint_as_float(gw[z] << 16), dsum);
           dsum = fmaf(__high2float(p2), __uint_as_float(gw[z] & 0xFFFF0000u), dsum);
         }
-        const uint32_t off = ch * 16384u + sw128_offset(erow, uu);
-        *reinterpret_cast<uint4*>(smem + off) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        const uint32_t off = kHLinA + kh * 8192u + sw128_offset(r, uu);
+        *reinterpret_cast<uint4*>(hbase + off) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
+      den = dsum + __shfl_xor_sync(0xffffffffu, dsum, 2);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&ctl->a_full);
-      den = dsum;
-    }
-    // normalizer of the linear branch from the two column halves (executed by every softmax
-    // thread exactly once, whatever path it took)
-    ctl->xd[ch][erow] = den;
-    pair_sync(bar_id);
-    den += ctl->xd[ch ^ 1][erow];
-    if (prm.linear && ok) {
-      // wait for this half's phi(Q) . G (rows of a missing second block store nothing)
-      if (half == 0 || has_b) {
-        ok = wait_or_abort(half == 0 ? &ctl->la_done : &ctl->lb_done, 0, ctl, status);
-        tc_fence_after();
-      } else {
-        ok = false;
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.a_full);
+      ok = wait_or_abort(&c.l_done, 0, ctl, status);
+      tc_fence_after();
     }
     const float inv_l = 1.f / l448;
     const float inv_den = 1.f / den;
+    const bool store = ok && tok < prm.N;
     float* sp_row = (prm.sparse_out && store) ? prm.sparse_out + (bh * prm.N + tok) * 128 : nullptr;
     char* out_row = static_cast<char*>(prm.out) +
                     (b_ * prm.out_sb + h_ * prm.out_sh + static_cast<int64_t>(tok) * prm.out_sn) *
                         (prm.out_dtype == SAGESLA_F32 ? 4 : 2);
     if (ok) {
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int col0 = 64 * ch + 32 * cc;
+      for (int cb = 0; cb < 2; ++cb) {
+        // this thread holds columns 64cb + 2e + kh (e = 0..31) of its row
         uint32_t o[32], lin[32];
-        tmem_ld32(tmem + lane_base + col0, o);
-        if (prm.linear) tmem_ld32(tmem + lane_base + kTmemS + col0, lin);
+        tmem_ld16x64(tmem + lane16 + 64 * cb, o);
+        if (prm.linear) tmem_ld16x64(tmem + lane16 + kTmemS + 64 * cb, lin);
         tmem_ld_wait();
-        float res[32];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const float os = __uint_as_float(o[q]) * ctl->s_v[col0 + q] * inv_l;
-          if (sp_row) sp_row[col0 + q] = os;
-          res[q] = prm.linear ? os + __uint_as_float(lin[q]) * inv_den : os;
+        for (int e = 0; e < 32; ++e) {
+          const float os = __uint_as_float(o[e]) * ctl->s_v[64 * cb + 2 * e + kh] * inv_l;
+          o[e] = __float_as_uint(os);
+          lin[e] = __float_as_uint(prm.linear ? os + __uint_as_float(lin[e]) * inv_den : os);
         }
-        if (store) {
-          if (prm.out_dtype == SAGESLA_F32) {
-            float4* d = reinterpret_cast<float4*>(out_row) + col0 / 4;
+        // Pair exchange with lane ^ 2 so that each thread stores contiguous columns: kh = 0
+        // stores 64cb + 0..31 and kh = 1 stores 64cb + 32..63, four at a time.
+        const int col0 = 64 * cb + 32 * kh;
+        auto exchange_store = [&](const uint32_t (&v)[32], float* dst_f32, uint16_t* dst_bf16) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) d[q] = make_float4(res[4 * q], res[4 * q + 1], res[4 * q + 2], res[4 * q + 3]);
-          } else {
-            uint4* d = reinterpret_cast<uint4*>(out_row) + col0 / 8;
+          for (int e = 0; e < 16; e += 2) {
+            float w4[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t w[4];
-#pragma unroll
-              for (int z = 0; z < 4; ++z) {
-                __nv_bfloat162 v2 = __floats2bfloat162_rn(res[8 * q + 2 * z], res[8 * q + 2 * z + 1]);
-                w[z] = *reinterpret_cast<uint32_t*>(&v2);
-              }
-              d[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int u = 0; u < 2; ++u) {
+              const float mine0 = __uint_as_float(v[e + u]), mine1 = __uint_as_float(v[16 + e + u]);
+              const float recv = __shfl_xor_sync(0xffffffffu, kh ? mine0 : mine1, 2);
+              w4[2 * u] = kh ? recv : mine0;
+              w4[2 * u + 1] = kh ? mine1 : recv;
+            }
+            if (dst_f32) {
+              *reinterpret_cast<float4*>(dst_f32 + 2 * e) = make_float4(w4[0], w4[1], w4[2], w4[3]);
+            } else if (dst_bf16) {
+              __nv_bfloat162 a2 = __floats2bfloat162_rn(w4[0], w4[1]);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(w4[2], w4[3]);
+              *reinterpret_cast<uint2*>(dst_bf16 + 2 * e) =
+                  make_uint2(*reinterpret_cast<uint32_t*>(&a2), *reinterpret_cast<uint32_t*>(&b2));
             }
           }
-        }
+        };
+        if (prm.sparse_out) exchange_store(o, sp_row ? sp_row + col0 : nullptr, nullptr);
+        if (prm.out_dtype == SAGESLA_F32)
+          exchange_store(lin, store ? reinterpret_cast<float*>(out_row) + col0 : nullptr, nullptr);
+        else
+          exchange_store(lin, nullptr, store ? reinterpret_cast<uint16_t*>(out_row) + col0 : nullptr);
       }
-    }
-    if (prm.linear && half == 0) {
-      tc_fence_before();
-      mbar_arrive(&ctl->la_free);
     }
   }
   tc_fence_before();
@@ -578,7 +634,7 @@ cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32
   const auto& L = p.lay;
   CUtensorMap tq, tk, tv, tg;
   const uint64_t rows = static_cast<uint64_t>(p.BH * p.n_pad);
-  if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, ws + L.q8, 128, 128,
+  if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, ws + L.q8, 128, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, ws + L.k8, 128, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -592,7 +648,7 @@ cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32
   prm.sq = reinterpret_cast<const float*>(ws + L.sq);
   prm.sk = reinterpret_cast<const float*>(ws + L.sk);
   prm.s_v = reinterpret_cast<const float*>(ws + L.s_v);
-  prm.mask = reinterpret_cast<const uint32_t*>(ws + L.mask);
+  prm.kept = reinterpret_cast<const int32_t*>(ws + L.kept);
   prm.gsum = reinterpret_cast<const __nv_bfloat16*>(ws + L.gsum);
   prm.q = q;
   prm.out = out;
@@ -606,12 +662,11 @@ cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32
   prm.nb = static_cast<int>(p.nb);
   prm.nbq = static_cast<int>(2 * p.n_pairs);
   prm.n_pad = static_cast<int>(p.n_pad);
-  prm.mask_words = static_cast<int>(p.mask_words);
+  prm.k = static_cast<int>(p.k);
   prm.nb_m_pad = static_cast<int>(p.nb_m_pad);
   prm.n_last = p.n_last;
-  prm.list_cap = static_cast<int>(p.nb < 2 * p.k ? p.nb : 2 * p.k);
   prm.linear = p.linear_empty ? 0 : 1;
-  const size_t smem = 1024 + kOffCtl + sizeof(Ctl) + static_cast<size_t>(prm.list_cap) * 8;
+  const size_t smem = 1024 + kOffCtl + sizeof(Ctl);
   cudaError_t e = cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -18,7 +18,9 @@
 //   warps 0-3 / 4-7  softmax, correction and epilogue of half 0 / half 1 (16 rows per warp,
 //                    two threads per row through the 16x64b TMEM fragment)
 //   warp 8           TMA producer for both halves (non-blocking event loop)
-//   warp 9           MMA issuer for both halves (non-blocking event loop)
+//   warp 9           S = Q K^T MMA issuer for both halves (non-blocking event loop); the
+//                    P.V MMA of an iteration is issued by the last of the half's four softmax
+//                    warps to finish it (a shared-memory counter), with no polling hop
 // Each half owns a private 52 KB of shared memory (its Q rows, a 2-stage K8/V8 ring and two
 // P tiles), reused for the linear-branch operands once its main loop is done.
 //
@@ -61,6 +63,7 @@ static_assert(kHLinG + 32768 <= kHalfBytes, "linear operands fit in the half reg
 constexpr uint32_t kOffCtl = 2 * kHalfBytes;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemS = 128;              // first S buffer column
+constexpr uint32_t kIdescPV = make_idesc(kFmtF32, kFmtE4M3, kFmtE4M3, 0, 1, 64, 128);
 // Columns of each thread's 32 whose exponential uses the polynomial instead of MUFU ex2.
 constexpr int kPolyFrom = 28;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -69,8 +72,9 @@ constexpr float kLog2_448 = 8.807354922057604f;
 
 struct HalfCtl {
   uint64_t full[kNS], empty[kNS];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], s_free[2], pv_done[2];
   uint64_t q_full, g_full, a_full, l_done, mma_done;
+  unsigned int p_count;      // softmax warps done with their P tile: 4 per iteration
 };
 
 struct Ctl {
@@ -271,7 +275,6 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       for (int s = 0; s < 2; ++s) {
         mbar_init(&c.s_full[s], 1);
         mbar_init(&c.s_free[s], 4);
-        mbar_init(&c.p_full[s], 4);
         mbar_init(&c.pv_done[s], 1);
       }
       mbar_init(&c.q_full, 1);
@@ -279,6 +282,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       mbar_init(&c.a_full, 4);
       mbar_init(&c.l_done, 1);
       mbar_init(&c.mma_done, 1);
+      c.p_count = 0u;
     }
     ctl->abort = 0;
     fence_mbar_init();
@@ -341,15 +345,26 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (S and the
+    // linear branch; P.V is issued by the last softmax warp of each iteration)
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc(kFmtS32, kFmtS8, kFmtS8, 0, 0, 64, 64);
-      constexpr uint32_t idesc_pv = make_idesc(kFmtF32, kFmtE4M3, kFmtE4M3, 0, 1, 64, 128);
       constexpr uint32_t idesc_l = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 64, 128);
       bool ok = true;
       for (int h = 0; h < 2 && ok; ++h)
         if (U[h] > 0) ok = wait_or_abort(&ctl->hc[h].q_full, 0, ctl, status);
-      int sn[2] = {0, 0}, pn[2] = {0, 0};
+      // Descriptors of the Q rows and of the K tile of each stage, per half; the K-steps of
+      // 32 bytes add 2 to the start-address field.
+      uint64_t dq[2], dk[2][kNS];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t hb = smem_u32(smem + h * kHalfBytes);
+        dq[h] = make_sdesc(hb + kHQ, 16, 1024, kLayoutSW128);
+#pragma unroll
+        for (int st = 0; st < kNS; ++st)
+          dk[h][st] = make_sdesc(hb + kHStages + st * kStageBytes, 16, 1024, kLayoutSW128);
+      }
+      int sn[2] = {0, 0};
       bool lin[2] = {U[0] == 0 || !prm.linear, U[1] == 0 || !prm.linear};
       Watchdog wd;
       while (ok) {
@@ -357,49 +372,29 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           HalfCtl& c = ctl->hc[h];
-          const uint32_t hb = smem_u32(smem + h * kHalfBytes);
           const uint32_t dlane = static_cast<uint32_t>(16 * h) << 16;
-          if (pn[h] < U[h]) {
+          const int n = sn[h];
+          if (n < U[h]) {
             pending = true;
-            const int n = sn[h];
-            if (n < U[h] && mbar_test(&c.full[n % kNS], (n / kNS) & 1) &&
+            if (mbar_test(&c.full[n % kNS], (n / kNS) & 1) &&
                 (n < 2 || mbar_test(&c.s_free[n & 1], ((n >> 1) - 1) & 1))) {
               tc_fence_after();
-              const uint32_t k_addr = hb + kHStages + (n % kNS) * kStageBytes;
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {   // 4 x K=32 channels
-                const uint64_t ad = make_sdesc(hb + kHQ + kk * 32, 16, 1024, kLayoutSW128);
-                const uint64_t bd = make_sdesc(k_addr + kk * 32, 16, 1024, kLayoutSW128);
-                mma_i8(tmem + dlane + kTmemS + 64 * (n & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-              }
+              const uint32_t d = tmem + dlane + kTmemS + 64 * (n & 1);
+              const uint64_t bq = dq[h], bk = dk[h][n % kNS];
+              mma_i8(d, bq, bk, idesc_s, 0u);
+              mma_i8(d, bq + 2, bk + 2, idesc_s, 1u);
+              mma_i8(d, bq + 4, bk + 4, idesc_s, 1u);
+              mma_i8(d, bq + 6, bk + 6, idesc_s, 1u);
               mma_commit(&c.s_full[n & 1]);
               ++sn[h];
               progress = true;
             }
-            const int m = pn[h];
-            if (m < sn[h] && mbar_test(&c.p_full[m & 1], (m >> 1) & 1)) {
-              tc_fence_after();
-              const uint32_t p_addr = hb + kHP + (m & 1) * kPBytes;
-              const uint32_t v_addr = hb + kHStages + (m % kNS) * kStageBytes + kKVBytes;
-#pragma unroll
-              for (int kk = 0; kk < 2; ++kk) {   // 2 x K=32 keys
-                // P: K-major, no swizzle (layout above). V: MN-major (d contiguous),
-                // 128-byte swizzle, 8-key groups 1024 B apart.
-                const uint64_t ad = make_sdesc(p_addr + kk * 2 * kPChunk, kPChunk, kPGroup, kLayoutNone);
-                const uint64_t bd = make_sdesc(v_addr + kk * 4096, 8192, 1024, kLayoutSW128);
-                mma_f8(tmem + dlane, ad, bd, idesc_pv, (m > 0 || kk > 0) ? 1u : 0u);
-              }
-              mma_commit(&c.pv_done[m & 1]);
-              mma_commit(&c.empty[m % kNS]);
-              ++pn[h];
-              if (pn[h] == U[h]) mma_commit(&c.mma_done);
-              progress = true;
-            }
           } else if (!lin[h]) {
-            // phi(Q_i) . G_i into this half's S columns
+            // phi(Q_i) . G_i into this half's S columns, once the loop's P.V are done
             pending = true;
-            if (mbar_test(&c.a_full, 0) && mbar_test(&c.g_full, 0)) {
+            if (mbar_test(&c.mma_done, 0) && mbar_test(&c.a_full, 0) && mbar_test(&c.g_full, 0)) {
               tc_fence_after();
+              const uint32_t hb = smem_u32(smem + h * kHalfBytes);
 #pragma unroll
               for (int kc = 0; kc < 2; ++kc)
 #pragma unroll
@@ -471,17 +466,17 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                               : row_exp_pack<false>(sr, valid, cst, neg, pk);
         l_part = alpha * l_part + rs;
         m_run = m_new;
-        // P(n) into buffer b once P.V(n-2) has read it
-        if (n >= 2 && !wait_or_abort(&c.pv_done[b], ((n >> 1) - 1) & 1, ctl, status)) { ok = false; break; }
+        // P.V(n-1) must be done: it frees P buffer b (read by P.V(n-2) before it), makes O
+        // stable for the rescale, and orders the P.V MMAs issued from different warps.
+        if (n >= 1 && !wait_or_abort(&c.pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status)) { ok = false; break; }
+        tc_fence_after();
         uint8_t* pb = hbase + kHP + b * kPBytes + (r >> 3) * kPGroup + (r & 7) * 16 + 2 * kh * kPChunk;
         *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4*>(pb + kPChunk) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         fence_proxy_async_smem();
-        // rescale this row's O once P.V(n-1) has landed (skipped when no row of the warp
-        // moved its max); the two threads of a row each take 64 of the 128 columns
+        // rescale this row's O (skipped when no row of the warp moved its max); the two
+        // threads of a row each take 64 of the 128 columns
         if (n >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!wait_or_abort(&c.pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status)) { ok = false; break; }
-          tc_fence_after();
           const unsigned long long a2 = pk2(alpha, alpha);
 #pragma unroll 1
           for (int cc = 0; cc < 2; ++cc) {
@@ -501,7 +496,28 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&c.p_full[b]);
+        if (lane == 0) {
+          // the last of the half's four warps to get here issues P.V(n)
+          __threadfence_block();
+          const unsigned int prior = atomicAdd(&c.p_count, 1u);
+          __threadfence_block();
+          if ((prior & 3u) == 3u) {
+            tc_fence_after();
+            const uint32_t hb = smem_u32(hbase);
+            const uint32_t p_addr = hb + kHP + b * kPBytes;
+            const uint32_t v_addr = hb + kHStages + (n % kNS) * kStageBytes + kKVBytes;
+            const uint32_t d = tmem + (static_cast<uint32_t>(16 * h) << 16);
+            // P: K-major, no swizzle (layout above). V: MN-major (d contiguous), 128-byte
+            // swizzle, 8-key groups 1024 B apart.
+            mma_f8(d, make_sdesc(p_addr, kPChunk, kPGroup, kLayoutNone),
+                   make_sdesc(v_addr, 8192, 1024, kLayoutSW128), kIdescPV, n > 0 ? 1u : 0u);
+            mma_f8(d, make_sdesc(p_addr + 2 * kPChunk, kPChunk, kPGroup, kLayoutNone),
+                   make_sdesc(v_addr + 4096, 8192, 1024, kLayoutSW128), kIdescPV, 1u);
+            mma_commit(&c.pv_done[b]);
+            mma_commit(&c.empty[n % kNS]);
+            if (n == Uh - 1) mma_commit(&c.mma_done);
+          }
+        }
       }
       if (ok) ok = wait_or_abort(&c.pv_done[(Uh - 1) & 1], ((Uh - 1) >> 1) & 1, ctl, status);
       tc_fence_after();

@@ -157,6 +157,29 @@ sagesla_status sagesla_forward_host(const uint16_t* q_host, const uint16_t* k_ho
                                     int32_t out_dtype, void* workspace, size_t workspace_bytes,
                                     void* stream);
 
+/* Size of the fixed scratch area used by sagesla_forward_no_alloc (64 MiB). */
+#define SAGESLA_NO_ALLOC_SCRATCH_BYTES (64ull << 20)
+
+/* Forward for callers that cannot allocate device memory (for example a host integration
+ * that only hands over input and output buffers, code inside a memory pool that may not
+ * grow, or a process that must not call cudaMalloc once loaded). The paper has no counterpart
+ * of this call: it exists for such integrations.
+ *   - Same arguments and result as sagesla_forward, without the workspace: the forward's
+ *     scratch lives in a device array of SAGESLA_NO_ALLOC_SCRATCH_BYTES that is part of this
+ *     library; every GPU that loads the library holds it until the process exits.
+ *   - Problems whose sagesla_workspace_size() exceeds SAGESLA_NO_ALLOC_SCRATCH_BYTES are
+ *     rejected with SAGESLA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents; calls whose GPU
+ *     work overlaps (different streams, or threads without ordering) race on it.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - Asynchronous on `stream`; device-side timeouts are not reported back (there is no
+ *     workspace to pass to sagesla_stream_status). */
+sagesla_status sagesla_forward_no_alloc(const sagesla_tensor* q, const sagesla_tensor* k,
+                                        const sagesla_tensor* v, double topk_ratio, int block,
+                                        sagesla_tensor* out, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device status word of `workspace`
  * (the one used by the last forward on that workspace). Returns SAGESLA_OK, TIMEOUT,
  * DEVICE_CHECK, or CUDA if the stream reported an error. */

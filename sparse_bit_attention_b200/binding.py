@@ -80,7 +80,11 @@ _SIGNATURES = {
         ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
         ctypes.c_size_t, ctypes.c_void_p]),
     "sagesla_stream_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "sagesla_forward_no_alloc": (ctypes.c_int, [ctypes.POINTER(SageslaTensor)] * 3 + [
+        ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaTensor), ctypes.c_void_p]),
 }
+
+NO_ALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -229,3 +233,17 @@ def sagesla_stream_status(stream=None, workspace: torch.Tensor | None = None) ->
     """Synchronizes the stream and returns (and clears) the workspace's device status word."""
     wp = None if workspace is None else ctypes.c_void_p(workspace.data_ptr())
     return int(load_library().sagesla_stream_status(ctypes.c_void_p(_stream_ptr(stream)), wp))
+
+
+def sagesla_forward_no_alloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                             topk_ratio: float = 0.1, block: int = BLOCK, stream=None) -> torch.Tensor:
+    """Forward for callers that cannot allocate device memory: the library's built-in scratch
+    area replaces the workspace (problems needing more than NO_ALLOC_SCRATCH_BYTES raise).
+    Calls whose GPU work overlaps race on that shared area."""
+    lib = load_library()
+    vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
+    _check(lib.sagesla_forward_no_alloc(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv),
+                                        float(topk_ratio), int(block), ctypes.byref(vo),
+                                        ctypes.c_void_p(_stream_ptr(stream))),
+           "sagesla_forward_no_alloc")
+    return out

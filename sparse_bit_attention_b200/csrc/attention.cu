@@ -13,24 +13,26 @@
 // B200 mapping. One CTA holds two query blocks ("halves"). Each half runs its own pipeline
 // over its own k kept blocks with M=64 tcgen05 MMAs: an M=64 result occupies TMEM lanes
 // 0-15 of each 32-lane quadrant, and a lane offset of 16 in the D address puts the second
-// half in lanes 16-31, so both halves share the TMEM columns (O fp32 [0,128); S int32 in two
-// buffers [128,192), [192,256); the linear branch reuses the S columns at the end).
+// half in lanes 16-31, so both halves share the TMEM columns (O fp32 [0,128); S int32 of a
+// pair of kept blocks [128,256); the linear branch reuses the S columns at the end).
 //   warps 0-3 / 4-7  softmax, correction and epilogue of half 0 / half 1 (16 rows per warp,
 //                    two threads per row through the 16x64b TMEM fragment)
-//   warp 8           TMA producer for both halves (non-blocking event loop)
-//   warp 9           S = Q K^T MMA issuer for both halves (non-blocking event loop); the
-//                    P.V MMA of an iteration is issued by the last of the half's four softmax
-//                    warps to finish it (a shared-memory counter), with no polling hop
-// Each half owns a private 52 KB of shared memory (its Q rows, a 2-stage K8/V8 ring and two
-// P tiles), reused for the linear-branch operands once its main loop is done.
+//   warp 8           TMA producer: Q rows, K8 tiles of pairs of kept blocks, V8 ring, G_i
+//   warp 9           S = Q K^T issuer for both halves: one M=64 N=128 MMA group (4 K-steps)
+//                    per pair of kept blocks, whose K8 tiles sit side by side in shared memory
+//   warps 10 / 11    P.V issuer of half 0 / half 1
+// A tcgen05.mma blocks its issuing thread for about 100 cycles whatever its shape (measured
+// on B200), while MMAs from different threads overlap: the N=128 pairs halve the S MMA count
+// and the issue work is spread over three threads. The helper warpgroup (8-11) hands
+// registers to the softmax warpgroups with setmaxnreg.
+// Each half owns 48 KB of shared memory (its Q rows, the K8 pair, a 3-stage V8 ring), reused
+// for the linear-branch operands once its main loop is done; its P tile sits after both halves.
 //
 // Softmax arithmetic per score: the int32 score becomes a float exactly through the 1.5*2^23
 // bias (integer add, then a packed f32x2 subtract: no conversion-pipe instruction); one packed
 // FFMA forms the base-2 exponent with the factor 448 of the P quantization folded in; 2^x
-// comes from the MUFU ex2 unit for most columns and, for the rest, from Cody-Waite range
-// reduction (round to nearest integer) plus a degree-5 polynomial fitted here by the Remez
-// exchange algorithm for minimax relative error on [-1/2, 1/2] (max relative error 2.3e-7 in
-// fp32), so that the FMA pipe takes part of the exponential load of the MUFU unit.
+// comes from the MUFU ex2 unit (measured faster here than moving part of the exponentials to
+// a polynomial on the FMA pipe: the loop is bound by latency, not by MUFU throughput).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -40,11 +42,13 @@ namespace sagesla {
 
 namespace {
 
-constexpr int kNS = 2;                       // K/V ring stages per half
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kNV = 3;                       // V ring stages per half
+constexpr int kProducerWarp = 8, kSWarp = 9, kPVWarp0 = 10;
+constexpr int kThreads = 384;
+// setmaxnreg split: 256 x 88 + 128 x 56 = 29696 registers, within the 384 x 80 a CTA is
+// launched with (checked on the host before the launch).
+constexpr uint32_t kSoftmaxRegs = 88, kHelperRegs = 56;
 constexpr uint32_t kKVBytes = 64 * 128;      // one K8 or V8 tile
-constexpr uint32_t kStageBytes = 2 * kKVBytes;
 // e4m3 P tile of one half (64 rows), K-major without swizzle: core matrices of 8 rows x 16
 // keys (128 B); K-chunks 160 B apart and 8-row groups 672 B apart. The padding makes the
 // 16-byte stores of the softmax threads (one store phase holds rows r, r+8, r+1, r+9 and key
@@ -53,28 +57,30 @@ constexpr uint32_t kPChunk = 160, kPGroup = 672;
 constexpr uint32_t kPBytes = 8 * kPGroup;
 // Per-half private region.
 constexpr uint32_t kHQ = 0;                  // the half's 64 Q8 rows (SW128), 8 KB
-constexpr uint32_t kHStages = 8192;
-constexpr uint32_t kHP = kHStages + kNS * kStageBytes;
-constexpr uint32_t kHalfBytes = 53248;
+constexpr uint32_t kHK = 8192;               // K8 tiles of a pair of kept blocks, 16 KB
+constexpr uint32_t kHV = kHK + 2 * kKVBytes; // V8 ring, kNV x 8 KB
+constexpr uint32_t kHalfBytes = kHV + kNV * kKVBytes;
 constexpr uint32_t kHLinA = 0;               // epilogue: phi(Q) bf16, 2 x [64][128 B]
 constexpr uint32_t kHLinG = 16384;           // epilogue: G_i bf16, 2 x [128][128 B]
-static_assert(kHP + 2 * kPBytes <= kHalfBytes, "half region");
 static_assert(kHLinG + 32768 <= kHalfBytes, "linear operands fit in the half region");
-constexpr uint32_t kOffCtl = 2 * kHalfBytes;
+static_assert(kHalfBytes % 1024 == 0, "half regions keep the 1024-byte swizzle atoms aligned");
+constexpr uint32_t kOffP = 2 * kHalfBytes;   // the two halves' P tiles
+constexpr uint32_t kOffCtl = kOffP + 2 * kPBytes;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemS = 128;              // first S buffer column
 constexpr uint32_t kIdescPV = make_idesc(kFmtF32, kFmtE4M3, kFmtE4M3, 0, 1, 64, 128);
-// Columns of each thread's 32 whose exponential uses the polynomial instead of MUFU ex2.
-constexpr int kPolyFrom = 28;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kInvSqrtD = 0.08838834764831845f;
 constexpr float kLog2_448 = 8.807354922057604f;
 
+// Every barrier is waited on by parity, which is safe because none can complete a phase
+// twice ahead of any of its waiters: each next phase needs an action that only follows the
+// waiter's own wait (for p_full: the softmax warps wait for P.V(n-1) before writing P(n)).
 struct HalfCtl {
-  uint64_t full[kNS], empty[kNS];
-  uint64_t s_full[2], s_free[2], pv_done[2];
+  uint64_t k_full, s_full, s_free;          // one phase per pair of kept blocks
+  uint64_t v_full[kNV], v_empty[kNV];
+  uint64_t p_full, pv_done[2];              // one phase per kept block
   uint64_t q_full, g_full, a_full, l_done, mma_done;
-  unsigned int p_count;      // softmax warps done with their P tile: 4 per iteration
 };
 
 struct Ctl {
@@ -109,27 +115,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ct
   }
   return true;
 }
-
-// Idle-time bookkeeping of the event loops: gives up (status TIMEOUT, abort) once no progress
-// was made for kSpinLimitNs.
-struct Watchdog {
-  unsigned long long since = 0;
-  int idle = 0;
-  __device__ __forceinline__ bool expired(Ctl* ctl, int* status) {
-    if (ctl->abort) return true;
-    if (++idle < 256) return false;
-    idle = 0;
-    const unsigned long long now = global_timer_ns();
-    if (since == 0) since = now;
-    if (now - since > kSpinLimitNs) {
-      record_error(status, SAGESLA_ERR_TIMEOUT);
-      ctl->abort = 1;
-      return true;
-    }
-    return false;
-  }
-  __device__ __forceinline__ void reset() { since = 0; idle = 0; }
-};
 
 // ---------------------------------------------------------------- packed f32x2 arithmetic
 __device__ __forceinline__ unsigned long long pk2(float a, float b) {
@@ -168,30 +153,6 @@ __device__ __forceinline__ float ex2_mufu(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe for two values: x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f by a
-// degree-5 minimax polynomial (coefficients from a Remez fit of relative error); 2^n added
-// to the exponent field. x is clamped below at -125 so that the result stays a normal float.
-__device__ __forceinline__ unsigned long long ex2_poly2(unsigned long long x2) {
-  float x0, x1;
-  up2(x2, x0, x1);
-  x2 = pk2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const unsigned long long magic = pk2(12582912.0f, 12582912.0f);
-  const unsigned long long t = add2(x2, magic);                 // rint(x) in low mantissa bits
-  const unsigned long long f = fma2(add2(t, pk2(-12582912.0f, -12582912.0f)),
-                                    pk2(-1.0f, -1.0f), x2);     // x - rint(x)
-  unsigned long long p = fma2(pk2(0.0013276472454890609f, 0.0013276472454890609f), f,
-                              pk2(0.009675540961325169f, 0.009675540961325169f));
-  p = fma2(p, f, pk2(0.05550713092088699f, 0.05550713092088699f));
-  p = fma2(p, f, pk2(0.24022120237350464f, 0.24022120237350464f));
-  p = fma2(p, f, pk2(0.6931469440460205f, 0.6931469440460205f));
-  p = fma2(p, f, pk2(1.0000001192092896f, 1.0000001192092896f));
-  float p0, p1, t0, t1;
-  up2(p, p0, p1);
-  up2(t, t0, t1);
-  return pk2(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
-             __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
-}
-
 // Maximum of this thread's valid scores (eight independent chains).
 template <bool kFull>
 __device__ __forceinline__ int row_block_max(const uint32_t (&a)[32], int valid) {
@@ -221,15 +182,10 @@ __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int vali
           pk2(__int_as_float(static_cast<int>(sr[q + t] + 0x4B400000u)),
               __int_as_float(static_cast<int>(sr[q + t + 1] + 0x4B400000u))),
           unbias);
-      const unsigned long long x2 = fma2(f2, c2, neg2);
-      if (q + t < kPolyFrom) {
-        float x0, x1;
-        up2(x2, x0, x1);
-        y[t] = ex2_mufu(x0);
-        y[t + 1] = ex2_mufu(x1);
-      } else {
-        up2(ex2_poly2(x2), y[t], y[t + 1]);
-      }
+      float x0, x1;
+      up2(fma2(f2, c2, neg2), x0, x1);
+      y[t] = ex2_mufu(x0);
+      y[t + 1] = ex2_mufu(x1);
       if (!kFull) {
         if (q + t >= valid) y[t] = 0.f;
         if (q + t + 1 >= valid) y[t + 1] = 0.f;
@@ -271,18 +227,18 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   } else if (threadIdx.x == 64) {
     for (int h = 0; h < 2; ++h) {
       HalfCtl& c = ctl->hc[h];
-      for (int s = 0; s < kNS; ++s) { mbar_init(&c.full[s], 1); mbar_init(&c.empty[s], 1); }
-      for (int s = 0; s < 2; ++s) {
-        mbar_init(&c.s_full[s], 1);
-        mbar_init(&c.s_free[s], 4);
-        mbar_init(&c.pv_done[s], 1);
-      }
+      mbar_init(&c.k_full, 1);
+      mbar_init(&c.s_full, 1);
+      mbar_init(&c.s_free, 4);
+      for (int s = 0; s < kNV; ++s) { mbar_init(&c.v_full[s], 1); mbar_init(&c.v_empty[s], 1); }
+      mbar_init(&c.p_full, 4);
+      mbar_init(&c.pv_done[0], 1);
+      mbar_init(&c.pv_done[1], 1);
       mbar_init(&c.q_full, 1);
       mbar_init(&c.g_full, 1);
       mbar_init(&c.a_full, 4);
       mbar_init(&c.l_done, 1);
       mbar_init(&c.mma_done, 1);
-      c.p_count = 0u;
     }
     ctl->abort = 0;
     fence_mbar_init();
@@ -294,6 +250,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
+  if (warp >= kProducerWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegs));
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -304,117 +262,128 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tma_load_2d(smem + h * kHalfBytes + kHQ, &tm_q, &ctl->hc[h].q_full, 0,
                     row_base + 128 * pair + 64 * h);
       }
-      int ld[2] = {0, 0};
-      bool gdone[2] = {U[0] == 0 || !prm.linear, U[1] == 0 || !prm.linear};
-      Watchdog wd;
-      while (true) {
-        bool pending = false, progress = false;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+      bool ok = true;
+      const int Umax = max(U[0], U[1]);
+      for (int n0 = 0; n0 < Umax && ok; n0 += 2) {
+        // K8 of the pair (n0, n0 + 1): the stage is free once S of the previous pair is done
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (n0 >= U[h]) continue;
           HalfCtl& c = ctl->hc[h];
-          uint8_t* hb = smem + h * kHalfBytes;
-          if (ld[h] < U[h]) {
-            pending = true;
-            const int n = ld[h], s = n % kNS;
-            if (n < kNS || mbar_test(&c.empty[s], ((n / kNS) - 1) & 1)) {
-              const int j = __ldg(prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) + n);
-              uint8_t* st = hb + kHStages + s * kStageBytes;
-              mbar_arrive_expect_tx(&c.full[s], kStageBytes);
-              tma_load_2d(st, &tm_k, &c.full[s], 0, row_base + 64 * j);
-              tma_load_2d(st + kKVBytes, &tm_v, &c.full[s], 0, row_base + 64 * j);
-              ++ld[h];
-              progress = true;
-            }
-          } else if (!gdone[h]) {
-            // A parity wait only tells the last two phases apart and this thread has not
-            // observed the P.V phases, so it waits on the single-phase "loop MMAs done".
-            pending = true;
-            if (mbar_test(&c.mma_done, 0)) {
-              const int gy = static_cast<int>((bh * prm.nb_m_pad + ia + h) * 129);
-              mbar_arrive_expect_tx(&c.g_full, 32768u);
-              tma_load_2d(hb + kHLinG, &tm_g, &c.g_full, 0, gy);
-              tma_load_2d(hb + kHLinG + 16384, &tm_g, &c.g_full, 64, gy);
-              gdone[h] = true;
-              progress = true;
-            }
-          }
+          if (n0 > 0 && !(ok = wait_or_abort(&c.s_full, ((n0 >> 1) - 1) & 1, ctl, status))) break;
+          const int32_t* klist = prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k);
+          const int two = n0 + 1 < U[h] ? 2 : 1;
+          mbar_arrive_expect_tx(&c.k_full, two * kKVBytes);
+          uint8_t* kst = smem + h * kHalfBytes + kHK;
+          tma_load_2d(kst, &tm_k, &c.k_full, 0, row_base + 64 * __ldg(klist + n0));
+          if (two == 2) tma_load_2d(kst + kKVBytes, &tm_k, &c.k_full, 0, row_base + 64 * __ldg(klist + n0 + 1));
         }
-        if (!pending) break;
-        if (progress) wd.reset();
-        else if (wd.expired(ctl, status)) break;
+        // V8 of blocks n0 and n0 + 1: stage n % kNV is free once P.V(n - kNV) is done
+        for (int n = n0; n < n0 + 2 && ok; ++n)
+          for (int h = 0; h < 2 && ok; ++h) {
+            if (n >= U[h]) continue;
+            HalfCtl& c = ctl->hc[h];
+            const int s = n % kNV;
+            if (n >= kNV && !(ok = wait_or_abort(&c.v_empty[s], ((n / kNV) - 1) & 1, ctl, status))) break;
+            const int32_t* klist = prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k);
+            mbar_arrive_expect_tx(&c.v_full[s], kKVBytes);
+            tma_load_2d(smem + h * kHalfBytes + kHV + s * kKVBytes, &tm_v, &c.v_full[s], 0,
+                        row_base + 64 * __ldg(klist + n));
+          }
+      }
+      // G_i once the half's loop MMAs are done (its tile overlaps the K and V stages)
+      for (int h = 0; h < 2 && ok && prm.linear; ++h) {
+        if (U[h] == 0) continue;
+        HalfCtl& c = ctl->hc[h];
+        if (!(ok = wait_or_abort(&c.mma_done, 0, ctl, status))) break;
+        const int gy = static_cast<int>((bh * prm.nb_m_pad + ia + h) * 129);
+        uint8_t* hb = smem + h * kHalfBytes;
+        mbar_arrive_expect_tx(&c.g_full, 32768u);
+        tma_load_2d(hb + kHLinG, &tm_g, &c.g_full, 0, gy);
+        tma_load_2d(hb + kHLinG + 16384, &tm_g, &c.g_full, 64, gy);
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer (S and the
-    // linear branch; P.V is issued by the last softmax warp of each iteration)
+  } else if (warp == kSWarp) {
+    // ------------------------------------------------------------ S = Q K^T issuer (both
+    // halves, one M=64 N=128 group per pair of kept blocks) and the linear-branch MMA
     if (lane == 0) {
-      constexpr uint32_t idesc_s = make_idesc(kFmtS32, kFmtS8, kFmtS8, 0, 0, 64, 64);
+      constexpr uint32_t idesc_s = make_idesc(kFmtS32, kFmtS8, kFmtS8, 0, 0, 64, 128);
       constexpr uint32_t idesc_l = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 64, 128);
       bool ok = true;
       for (int h = 0; h < 2 && ok; ++h)
         if (U[h] > 0) ok = wait_or_abort(&ctl->hc[h].q_full, 0, ctl, status);
-      // Descriptors of the Q rows and of the K tile of each stage, per half; the K-steps of
-      // 32 bytes add 2 to the start-address field.
-      uint64_t dq[2], dk[2][kNS];
+      // Q rows and K pair descriptors; the K-steps of 32 bytes add 2 to the address field.
+      uint64_t dq[2], dk[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t hb = smem_u32(smem + h * kHalfBytes);
         dq[h] = make_sdesc(hb + kHQ, 16, 1024, kLayoutSW128);
-#pragma unroll
-        for (int st = 0; st < kNS; ++st)
-          dk[h][st] = make_sdesc(hb + kHStages + st * kStageBytes, 16, 1024, kLayoutSW128);
+        dk[h] = make_sdesc(hb + kHK, 16, 1024, kLayoutSW128);
       }
-      int sn[2] = {0, 0};
-      bool lin[2] = {U[0] == 0 || !prm.linear, U[1] == 0 || !prm.linear};
-      Watchdog wd;
-      while (ok) {
-        bool pending = false, progress = false;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+      const int Umax = max(U[0], U[1]);
+      for (int n0 = 0; n0 < Umax && ok; n0 += 2) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (n0 >= U[h]) continue;
           HalfCtl& c = ctl->hc[h];
-          const uint32_t dlane = static_cast<uint32_t>(16 * h) << 16;
-          const int n = sn[h];
-          if (n < U[h]) {
-            pending = true;
-            if (mbar_test(&c.full[n % kNS], (n / kNS) & 1) &&
-                (n < 2 || mbar_test(&c.s_free[n & 1], ((n >> 1) - 1) & 1))) {
-              tc_fence_after();
-              const uint32_t d = tmem + dlane + kTmemS + 64 * (n & 1);
-              const uint64_t bq = dq[h], bk = dk[h][n % kNS];
-              mma_i8(d, bq, bk, idesc_s, 0u);
-              mma_i8(d, bq + 2, bk + 2, idesc_s, 1u);
-              mma_i8(d, bq + 4, bk + 4, idesc_s, 1u);
-              mma_i8(d, bq + 6, bk + 6, idesc_s, 1u);
-              mma_commit(&c.s_full[n & 1]);
-              ++sn[h];
-              progress = true;
-            }
-          } else if (!lin[h]) {
-            // phi(Q_i) . G_i into this half's S columns, once the loop's P.V are done
-            pending = true;
-            if (mbar_test(&c.mma_done, 0) && mbar_test(&c.a_full, 0) && mbar_test(&c.g_full, 0)) {
-              tc_fence_after();
-              const uint32_t hb = smem_u32(smem + h * kHalfBytes);
-#pragma unroll
-              for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t ad = make_sdesc(hb + kHLinA + kc * 8192 + kk * 32, 16, 1024, kLayoutSW128);
-                  const uint64_t bd = make_sdesc(hb + kHLinG + kc * 16384 + kk * 32, 16, 1024, kLayoutSW128);
-                  mma_bf16(tmem + dlane + kTmemS, ad, bd, idesc_l, (kc | kk) ? 1u : 0u);
-                }
-              mma_commit(&c.l_done);
-              lin[h] = true;
-              progress = true;
-            }
-          }
+          const int p = n0 >> 1;
+          if (!(ok = wait_or_abort(&c.k_full, p & 1, ctl, status))) break;
+          if (p > 0 && !(ok = wait_or_abort(&c.s_free, (p - 1) & 1, ctl, status))) break;
+          tc_fence_after();
+          const uint32_t d = tmem + (static_cast<uint32_t>(16 * h) << 16) + kTmemS;
+          mma_i8(d, dq[h], dk[h], idesc_s, 0u);
+          mma_i8(d, dq[h] + 2, dk[h] + 2, idesc_s, 1u);
+          mma_i8(d, dq[h] + 4, dk[h] + 4, idesc_s, 1u);
+          mma_i8(d, dq[h] + 6, dk[h] + 6, idesc_s, 1u);
+          mma_commit(&c.s_full);
         }
-        if (!pending) break;
-        if (progress) wd.reset();
-        else if (wd.expired(ctl, status)) break;
+      }
+      for (int h = 0; h < 2 && ok && prm.linear; ++h) {
+        // phi(Q_i) . G_i into this half's S columns, once the loop's P.V are done
+        if (U[h] == 0) continue;
+        HalfCtl& c = ctl->hc[h];
+        if (!(ok = wait_or_abort(&c.mma_done, 0, ctl, status) && wait_or_abort(&c.a_full, 0, ctl, status) &&
+                   wait_or_abort(&c.g_full, 0, ctl, status))) break;
+        tc_fence_after();
+        const uint32_t dlane = static_cast<uint32_t>(16 * h) << 16;
+        const uint32_t hb = smem_u32(smem + h * kHalfBytes);
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_sdesc(hb + kHLinA + kc * 8192 + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bd = make_sdesc(hb + kHLinG + kc * 16384 + kk * 32, 16, 1024, kLayoutSW128);
+            mma_bf16(tmem + dlane + kTmemS, ad, bd, idesc_l, (kc | kk) ? 1u : 0u);
+          }
+        mma_commit(&c.l_done);
       }
     }
+  } else if (warp >= kPVWarp0) {
+    // ------------------------------------------------------------ P.V issuer of one half
+    if (lane == 0) {
+      const int h = warp - kPVWarp0;
+      HalfCtl& c = ctl->hc[h];
+      const uint32_t p_addr = smem_u32(smem) + kOffP + h * kPBytes;
+      const uint64_t dp0 = make_sdesc(p_addr, kPChunk, kPGroup, kLayoutNone);
+      const uint64_t dp1 = make_sdesc(p_addr + 2 * kPChunk, kPChunk, kPGroup, kLayoutNone);
+      const uint32_t vb = smem_u32(smem + h * kHalfBytes) + kHV;
+      const uint32_t d = tmem + (static_cast<uint32_t>(16 * h) << 16);
+      for (int n = 0; n < U[h]; ++n) {
+        const int s = n % kNV;
+        if (!wait_or_abort(&c.p_full, n & 1, ctl, status)) break;
+        if (!wait_or_abort(&c.v_full[s], (n / kNV) & 1, ctl, status)) break;
+        tc_fence_after();
+        // P: K-major, no swizzle (layout above). V: MN-major (d contiguous), 128-byte
+        // swizzle, 8-key groups 1024 B apart.
+        const uint32_t v_addr = vb + s * kKVBytes;
+        mma_f8(d, dp0, make_sdesc(v_addr, 8192, 1024, kLayoutSW128), kIdescPV, n > 0 ? 1u : 0u);
+        mma_f8(d, dp1, make_sdesc(v_addr + 4096, 8192, 1024, kLayoutSW128), kIdescPV, 1u);
+        mma_commit(&c.pv_done[n & 1]);
+        mma_commit(&c.v_empty[s]);
+        if (n == U[h] - 1) mma_commit(&c.mma_done);
+      }
+    }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ------------------------------------------------------------ softmax / epilogue
     // Warp w serves half h = w/4 and reads TMEM lanes 32*(w&3) + 16h + 0..15 (16x64b
     // fragment): lane t holds row r = 16*(w&3) + t/4 + 8*(t&1) of the half's query block and
@@ -446,14 +415,16 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           j_next = __ldg(klist + n + 1);
           sk_next = __ldg(skh + j_next);
         }
-        if (!wait_or_abort(&c.s_full[b], (n >> 1) & 1, ctl, status)) { ok = false; break; }
+        if (b == 0 && !wait_or_abort(&c.s_full, (n >> 1) & 1, ctl, status)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[32];
         tmem_ld16x64(tmem + lane16 + kTmemS + 64 * b, sr);
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c.s_free[b]);
+        if (b == 1) {                            // both blocks of the pair are read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.s_free);
+        }
         const bool full = j != prm.nb - 1 || prm.n_last == 64;   // no padded keys
         int mxi = full ? row_block_max<true>(sr, 32) : row_block_max<false>(sr, valid);
         mxi = max(mxi, __shfl_xor_sync(0xffffffffu, mxi, 2));
@@ -470,7 +441,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // stable for the rescale, and orders the P.V MMAs issued from different warps.
         if (n >= 1 && !wait_or_abort(&c.pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status)) { ok = false; break; }
         tc_fence_after();
-        uint8_t* pb = hbase + kHP + b * kPBytes + (r >> 3) * kPGroup + (r & 7) * 16 + 2 * kh * kPChunk;
+        uint8_t* pb = smem + kOffP + h * kPBytes + (r >> 3) * kPGroup + (r & 7) * 16 + 2 * kh * kPChunk;
         *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4*>(pb + kPChunk) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         fence_proxy_async_smem();
@@ -496,28 +467,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          // the last of the half's four warps to get here issues P.V(n)
-          __threadfence_block();
-          const unsigned int prior = atomicAdd(&c.p_count, 1u);
-          __threadfence_block();
-          if ((prior & 3u) == 3u) {
-            tc_fence_after();
-            const uint32_t hb = smem_u32(hbase);
-            const uint32_t p_addr = hb + kHP + b * kPBytes;
-            const uint32_t v_addr = hb + kHStages + (n % kNS) * kStageBytes + kKVBytes;
-            const uint32_t d = tmem + (static_cast<uint32_t>(16 * h) << 16);
-            // P: K-major, no swizzle (layout above). V: MN-major (d contiguous), 128-byte
-            // swizzle, 8-key groups 1024 B apart.
-            mma_f8(d, make_sdesc(p_addr, kPChunk, kPGroup, kLayoutNone),
-                   make_sdesc(v_addr, 8192, 1024, kLayoutSW128), kIdescPV, n > 0 ? 1u : 0u);
-            mma_f8(d, make_sdesc(p_addr + 2 * kPChunk, kPChunk, kPGroup, kLayoutNone),
-                   make_sdesc(v_addr + 4096, 8192, 1024, kLayoutSW128), kIdescPV, 1u);
-            mma_commit(&c.pv_done[b]);
-            mma_commit(&c.empty[n % kNS]);
-            if (n == Uh - 1) mma_commit(&c.mma_done);
-          }
-        }
+        if (lane == 0) mbar_arrive(&c.p_full);
       }
       if (ok) ok = wait_or_abort(&c.pv_done[(Uh - 1) & 1], ((Uh - 1) >> 1) & 1, ctl, status);
       tc_fence_after();
@@ -682,6 +632,16 @@ cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32
   prm.nb_m_pad = static_cast<int>(p.nb_m_pad);
   prm.n_last = p.n_last;
   prm.linear = p.linear_empty ? 0 : 1;
+  // The register split (setmaxnreg) must fit the registers the CTA is launched with, or the
+  // softmax warps would wait for registers forever.
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, k_attention) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+    regs = fa.numRegs;
+  }
+  if (static_cast<uint32_t>(regs) * kThreads < 256 * kSoftmaxRegs + 128 * kHelperRegs)
+    return cudaErrorInvalidConfiguration;
   const size_t smem = 1024 + kOffCtl + sizeof(Ctl);
   cudaError_t e = cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

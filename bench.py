@@ -14,6 +14,11 @@ reported.
 
 --impl reference times the CPU oracle (test infrastructure, float64) on the host cores, on a
 bounded sample of the same workload per step, extrapolated to the whole forward.
+
+--sweep (one GPU) prints one JSON line per point instead: the forward on the 14B-720P random
+workload and on the smoothed-field locality workload over Top-K ratios 0.05-0.2 and the dense
+mode (ratio 1: every block kept, selection and linear branch skipped), and a dense BF16
+attention of the same shape through torch's scaled_dot_product_attention for comparison.
 """
 from __future__ import annotations
 
@@ -50,9 +55,21 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="another named workload (smaller cases for ncu captures)")
+    ap.add_argument("--topk-ratio", type=float, default=None,
+                    help="Top-K ratio (default: 0.1; 1.0 is the dense SageAttention mode)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="Top-K ratio sweep and dense BF16 comparison, one JSON line per point")
     args = ap.parse_args()
     globals()["WORKLOAD"] = args.workload
+    if args.topk_ratio is not None:
+        globals()["RATIO"] = args.topk_ratio
     return args
+
+
+def kernel_launches(dense: bool) -> int:
+    """Kernels of one forward: stats, finalize, quant, scores, top-k, complement GEMM and
+    attention; with every block kept only stats, finalize, quant and attention run."""
+    return 4 if dense else 7
 
 
 def measured_peaks():
@@ -346,7 +363,8 @@ def run_cuda(args):
                 "dense_equiv_tops": 4.0 * B * H * N * N * D / fwd_s / 1e12,
                 "stage_ms": stage_ms, "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": e2e,
-                "gpu_launches": binding.N_STAGES * args.steps, "clocks": clock_info}
+                "gpu_launches": kernel_launches(lay["k"] == lay["nb"]) * args.steps,
+                "clocks": clock_info}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -354,8 +372,93 @@ def run_cuda(args):
     return 0
 
 
+def _time_forward(sba, binding, torch, q, k, v, ratio, steps, warmup):
+    B, H, N, D = q.shape
+    lay = sba.sagesla_get_workspace_layout(B, H, N, D, ratio)
+    ws = sba.alloc_workspace(lay["total_bytes"], q.device)
+    out = torch.empty((B, H, N, D), dtype=torch.float32, device=q.device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        sba.sagesla_forward(q, k, v, ratio, out=out, workspace=ws)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(binding.N_STAGES + 1)]
+          for _ in range(steps)]
+    for s in range(steps):
+        sba.sagesla_forward(q, k, v, ratio, out=out, workspace=ws, stage_events=ev[s])
+    torch.cuda.synchronize()
+    st = sba.sagesla_stream_status(stream, ws)
+    if st != 0:
+        raise RuntimeError(f"device status: {sba.sagesla_status_string(st)}")
+    stage = {name: statistics.median(e[i].elapsed_time(e[i + 1]) for e in ev)
+             for i, name in enumerate(binding.STAGE_NAMES)}
+    total = statistics.median(e[0].elapsed_time(e[-1]) for e in ev)
+    del ws, out
+    torch.cuda.empty_cache()
+    return lay, total, stage
+
+
+def _time_sdpa(torch, q, k, v, steps, warmup):
+    """Dense BF16 attention of the same shape through torch (a library kernel, for context)."""
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    for backend in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION,
+                    SDPBackend.EFFICIENT_ATTENTION):
+        try:
+            with sdpa_kernel([backend]):
+                for _ in range(warmup):
+                    F.scaled_dot_product_attention(q, k, v)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(steps):
+                    F.scaled_dot_product_attention(q, k, v)
+                e1.record()
+                torch.cuda.synchronize()
+            return backend.name, e0.elapsed_time(e1) / steps
+        except RuntimeError:
+            continue
+    return None, None
+
+
+def run_sweep(args):
+    import torch
+    import sparse_bit_attention_b200 as sba
+    from sparse_bit_attention_b200 import binding, inputs
+    from sparse_bit_attention_b200.build import build
+    build()
+    sba.load_library()
+    dev = torch.device("cuda", 0)
+    steps = max(3, min(args.steps, 10))
+    for name, ratios in (("wan21_14b_720p", (0.05, 0.1, 0.15, 0.2, 1.0)),
+                         ("locality_14b_720p", (0.05, 0.1, 0.15, 0.2))):
+        q, k, v = (x.to(dev) for x in inputs.make_qkv(name))
+        B, H, N, D = q.shape
+        dense_ops = 4.0 * B * H * N * N * D
+        for ratio in ratios:
+            lay, ms, stage = _time_forward(sba, binding, torch, q, k, v, ratio, steps, args.warmup)
+            ops = attention_tensor_ops(B, H, lay["nb"], lay["k"])
+            print(json.dumps({
+                "sweep": name, "topk_ratio": ratio, "k": lay["k"], "nb": lay["nb"],
+                "ms_per_forward": ms, "tokens_per_s": B * N / (ms / 1e3),
+                "attention_ms": stage["attention"],
+                "attention_tops": ops / (stage["attention"] / 1e3) / 1e12,
+                "dense_equiv_tops": dense_ops / (ms / 1e3) / 1e12,
+                "stage_ms": stage}), flush=True)
+        if name == "wan21_14b_720p":
+            backend, ms = _time_sdpa(torch, q, k, v, max(2, steps // 2), 1)
+            print(json.dumps({
+                "sweep": name, "baseline": "torch scaled_dot_product_attention, bf16 dense",
+                "backend": backend, "ms_per_forward": ms,
+                "tokens_per_s": B * N / (ms / 1e3) if ms else None,
+                "dense_tflops": dense_ops / (ms / 1e3) / 1e12 if ms else None}), flush=True)
+        del q, k, v
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.sweep:
+        return run_sweep(args)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

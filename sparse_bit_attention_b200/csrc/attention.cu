@@ -90,11 +90,17 @@ struct Ctl {
   float s_v[128];
 };
 
+// n-th kept key block of a query block: its kept list, or block n itself when every block is
+// kept (no list).
+__device__ __forceinline__ int kept_block(const int32_t* klist, int n) {
+  return klist ? __ldg(klist + n) : n;
+}
+
 struct AttnParams {
   const float* sq;            // [BH][nbq]
   const float* sk;            // [BH][nbq]
   const float* s_v;           // [BH][128]
-  const int32_t* kept;        // [BH][nb][k]
+  const int32_t* kept;        // [BH][nb][k], or null when every block is kept
   const __nv_bfloat16* gsum;  // [BH][nb_m_pad][129][128]
   TensorArg q;                // raw bf16 Q (for phi(q))
   void* out;
@@ -270,12 +276,12 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           if (n0 >= U[h]) continue;
           HalfCtl& c = ctl->hc[h];
           if (n0 > 0 && !(ok = wait_or_abort(&c.s_full, ((n0 >> 1) - 1) & 1, ctl, status))) break;
-          const int32_t* klist = prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k);
+          const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) : nullptr;
           const int two = n0 + 1 < U[h] ? 2 : 1;
           mbar_arrive_expect_tx(&c.k_full, two * kKVBytes);
           uint8_t* kst = smem + h * kHalfBytes + kHK;
-          tma_load_2d(kst, &tm_k, &c.k_full, 0, row_base + 64 * __ldg(klist + n0));
-          if (two == 2) tma_load_2d(kst + kKVBytes, &tm_k, &c.k_full, 0, row_base + 64 * __ldg(klist + n0 + 1));
+          tma_load_2d(kst, &tm_k, &c.k_full, 0, row_base + 64 * kept_block(klist, n0));
+          if (two == 2) tma_load_2d(kst + kKVBytes, &tm_k, &c.k_full, 0, row_base + 64 * kept_block(klist, n0 + 1));
         }
         // V8 of blocks n0 and n0 + 1: stage n % kNV is free once P.V(n - kNV) is done
         for (int n = n0; n < n0 + 2 && ok; ++n)
@@ -284,10 +290,10 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             HalfCtl& c = ctl->hc[h];
             const int s = n % kNV;
             if (n >= kNV && !(ok = wait_or_abort(&c.v_empty[s], ((n / kNV) - 1) & 1, ctl, status))) break;
-            const int32_t* klist = prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k);
+            const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) : nullptr;
             mbar_arrive_expect_tx(&c.v_full[s], kKVBytes);
             tma_load_2d(smem + h * kHalfBytes + kHV + s * kKVBytes, &tm_v, &c.v_full[s], 0,
-                        row_base + 64 * __ldg(klist + n));
+                        row_base + 64 * kept_block(klist, n));
           }
       }
       // G_i once the half's loop MMAs are done (its tile overlaps the K and V stages)
@@ -403,16 +409,16 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     float m_run = -INFINITY, l_part = 0.f;
     if (ok) {
       const float cs = prm.sq[bh * prm.nbq + qblock] * (kLog2e * kInvSqrtD);
-      const int32_t* klist = prm.kept + (bh * prm.nb + qblock) * static_cast<int64_t>(prm.k);
+      const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + qblock) * static_cast<int64_t>(prm.k) : nullptr;
       const float* skh = prm.sk + bh * prm.nbq;
-      int j_next = __ldg(klist);
+      int j_next = kept_block(klist, 0);
       float sk_next = __ldg(skh + j_next);
       for (int n = 0; n < Uh; ++n) {
         const int b = n & 1;
         const int j = j_next;
         const float skj = sk_next;
         if (n + 1 < Uh) {                        // prefetch the next kept block's scale
-          j_next = __ldg(klist + n + 1);
+          j_next = kept_block(klist, n + 1);
           sk_next = __ldg(skh + j_next);
         }
         if (b == 0 && !wait_or_abort(&c.s_full, (n >> 1) & 1, ctl, status)) { ok = false; break; }
@@ -614,7 +620,7 @@ cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32
   prm.sq = reinterpret_cast<const float*>(ws + L.sq);
   prm.sk = reinterpret_cast<const float*>(ws + L.sk);
   prm.s_v = reinterpret_cast<const float*>(ws + L.s_v);
-  prm.kept = reinterpret_cast<const int32_t*>(ws + L.kept);
+  prm.kept = p.linear_empty ? nullptr : reinterpret_cast<const int32_t*>(ws + L.kept);
   prm.gsum = reinterpret_cast<const __nv_bfloat16*>(ws + L.gsum);
   prm.q = q;
   prm.out = out;

@@ -47,6 +47,7 @@ cudaError_t launch_quant(const ForwardPlan& p, TensorArg q, TensorArg k, TensorA
                          cudaStream_t stream);
 cudaError_t launch_scores(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_topk(const ForwardPlan& p, char* ws, cudaStream_t stream);
+cudaError_t launch_fill_all_kept(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_complement_gemm(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32_t out_dtype,
                              int64_t out_sb, int64_t out_sh, int64_t out_sn, float* sparse_out,

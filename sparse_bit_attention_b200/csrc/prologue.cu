@@ -59,6 +59,9 @@ constexpr int kStatsThreads = 128;
 // CTAs on an SM, so four 128-column TMEM allocations always fit in the 512 columns.
 constexpr int kStatsSmem = 52 * 1024;
 
+// kLinear = false (every key block kept, no linear branch): only the K sums, V amax and
+// pooled K are needed, so phi, H_j and its MMA are skipped.
+template <bool kLinear>
 __global__ void __launch_bounds__(kStatsThreads)
 k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restrict__ ksum_part,
         float* __restrict__ vmax_part, float* __restrict__ kbar, __nv_bfloat16* __restrict__ hflat,
@@ -80,15 +83,16 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
   __nv_bfloat16* hrow = hflat + (bh * nb_k_pad + j) * static_cast<int64_t>(kHFlat);
 
   if (j >= nb) {  // zero padding rows of the complement-sum GEMM operand
-    for (int e = t; e < kHFlat; e += kStatsThreads) hrow[e] = __float2bfloat16_rn(0.f);
+    if (kLinear)
+      for (int e = t; e < kHFlat; e += kStatsThreads) hrow[e] = __float2bfloat16_rn(0.f);
     return;
   }
 
-  if (warp == 0) {
+  if (kLinear && warp == 0) {
     tmem_alloc(tmem_slot, 128);
     tmem_relinquish();
   }
-  if (t == 0) {
+  if (kLinear && t == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
   }
@@ -125,6 +129,7 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
       vmax[e] = fmaxf(vmax[e], fabsf(vf[e]));
       mx = fmaxf(mx, kf[e]);
     }
+    if (!kLinear) continue;
     // phi = softmax over the 128 channels of this token; the row lives in 16 lanes.
 #pragma unroll
     for (int o = 8; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -156,8 +161,8 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
   fence_proxy_async_smem();
   __syncthreads();
 
-  const uint32_t tmem = *tmem_slot;
-  if (t == 0) {
+  const uint32_t tmem = kLinear ? *tmem_slot : 0u;
+  if (kLinear && t == 0) {
     tc_fence_after();
     constexpr uint32_t idesc = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 1, 1, 128, 128);
 #pragma unroll
@@ -182,8 +187,9 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
     ksum_part[o] = ks;
     vmax_part[o] = vm;
     kbar[o] = static_cast<float>(ks / static_cast<double>(nj));
-    hrow[128 * 128 + c] = __float2bfloat16_rn(ps);
+    if (kLinear) hrow[128 * 128 + c] = __float2bfloat16_rn(ps);
   }
+  if (!kLinear) return;
 
   const bool ok = mbar_wait(bar, 0, status);
   tc_fence_after();
@@ -365,14 +371,18 @@ cudaError_t launch_stats(const ForwardPlan& p, TensorArg k, TensorArg v, char* w
                          cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_stats, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kStatsSmem);
-    if (e != cudaSuccess) return e;
+    for (const void* f : {reinterpret_cast<const void*>(k_stats<true>),
+                          reinterpret_cast<const void*>(k_stats<false>)}) {
+      cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kStatsSmem);
+      if (e != cudaSuccess) return e;
+    }
     configured = true;
   }
   const auto& L = p.lay;
   dim3 grid(static_cast<unsigned>(p.nb_k_pad), static_cast<unsigned>(p.BH));
-  k_stats<<<grid, kStatsThreads, kStatsSmem, stream>>>(
+  auto kern = p.linear_empty ? k_stats<false> : k_stats<true>;
+  kern<<<grid, kStatsThreads, kStatsSmem, stream>>>(
       k, v, static_cast<int>(p.N), static_cast<int>(p.nb), static_cast<int>(p.nb_k_pad),
       reinterpret_cast<double*>(ws + L.ksum_part), reinterpret_cast<float*>(ws + L.vmax_part),
       reinterpret_cast<float*>(ws + L.kbar), reinterpret_cast<__nv_bfloat16*>(ws + L.hflat),

@@ -265,9 +265,13 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
   SAGESLA_LAUNCH(mark(2));
   SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
   SAGESLA_LAUNCH(mark(3));
-  SAGESLA_LAUNCH(launch_scores(p, ws, stream));
+  // With every key block kept (k == nb) the selection is the identity: the scores are only
+  // computed when asked for, and the kept lists and masks only written when asked for.
+  const bool want_lists = opt && (opt->kept_idx_out || opt->mask_out);
+  if (!p.linear_empty || (opt && opt->scores_out)) SAGESLA_LAUNCH(launch_scores(p, ws, stream));
   SAGESLA_LAUNCH(mark(4));
-  SAGESLA_LAUNCH(launch_topk(p, ws, stream));
+  if (!p.linear_empty) SAGESLA_LAUNCH(launch_topk(p, ws, stream));
+  else if (want_lists) SAGESLA_LAUNCH(launch_fill_all_kept(p, ws, stream));
   SAGESLA_LAUNCH(mark(5));
   if (!p.linear_empty) SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
   SAGESLA_LAUNCH(mark(6));

@@ -172,6 +172,18 @@ k_topk(int nb, int k, int mask_words, int nb_k_pad, const float* __restrict__ sc
   }
 }
 
+// Every key block kept (k == nb): kept lists 0..nb-1 and full masks. Written only when a
+// caller asks for them; the attention kernel then walks the key blocks in order without a list.
+__global__ void k_fill_all_kept(int nb, int mask_words, int32_t* __restrict__ kept,
+                                uint32_t* __restrict__ mask) {
+  const int64_t row = blockIdx.x;
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) kept[row * nb + j] = j;
+  for (int w = threadIdx.x; w < mask_words; w += blockDim.x) {
+    const int rem = nb - 32 * w;
+    mask[row * mask_words + w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+  }
+}
+
 __global__ void k_scale_scores(int64_t n, const float* __restrict__ src, float* __restrict__ dst) {
   const int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (e < n) dst[e] = src[e] * 0.08838834764831845f;   // 1/sqrt(128)
@@ -207,6 +219,13 @@ cudaError_t launch_topk(const ForwardPlan& p, char* ws, cudaStream_t stream) {
       static_cast<int>(p.nb_k_pad), reinterpret_cast<const float*>(ws + L.scores),
       reinterpret_cast<int32_t*>(ws + L.kept), reinterpret_cast<uint32_t*>(ws + L.mask),
       reinterpret_cast<__nv_bfloat16*>(ws + L.amask), static_cast<int>(p.nb_m_pad));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_all_kept(const ForwardPlan& p, char* ws, cudaStream_t stream) {
+  k_fill_all_kept<<<static_cast<unsigned>(p.BH * p.nb), 256, 0, stream>>>(
+      static_cast<int>(p.nb), static_cast<int>(p.mask_words),
+      reinterpret_cast<int32_t*>(ws + p.lay.kept), reinterpret_cast<uint32_t*>(ws + p.lay.mask));
   return cudaGetLastError();
 }
 

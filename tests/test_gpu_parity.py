@@ -94,6 +94,32 @@ def test_repeatable():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("n,seed", [(1025, 26), (4096, 27), (700, 28)])
+def test_dense_mode(n, seed):
+    """r = 1 keeps every key block: no selection, no linear branch, the attention kernel walks
+    the blocks in order (odd block counts leave a single-block last pair)."""
+    q, k, v = inputs.make_random(1, 2, n, seed, k_offset_std=1.0)
+    res = gpu_run(q, k, v, 1.0)
+    nb = res["layout"]["nb"]
+    assert res["layout"]["k"] == nb
+    assert (res["kept"] == np.arange(nb, dtype=np.int32)[None, None, :]).all()
+    err, _ = _all_heads(q, k, v, 1.0, res)
+    assert err <= OUT_TOL, err
+    # without the optional outputs the lists are never written; the output is the same
+    plain = gpu_run(q, k, v, 1.0, extras=False)
+    assert torch.equal(plain["out"], res["out"])
+
+
+def test_dense_mode_full_size_sampled():
+    """r = 1 on the Wan2.1-1.3B-480P shape (512 kept blocks per query block), sampled rows."""
+    q, k, v = inputs.make_qkv("wan21_1p3b_480p", heads=2)
+    res = gpu_run(q, k, v, 1.0)
+    nb = res["layout"]["nb"]
+    for h in range(2):
+        err, _ = compare_head(q, k, v, 1.0, res, 0, h, rows=_sampled_rows(nb, 30 + h, count=3))
+        assert err <= OUT_TOL, (h, err)
+
+
 def _sampled_rows(nb, seed, count=6):
     rng = np.random.default_rng(seed)
     return sorted(set([0, 1, nb - 2, nb - 1] + list(rng.integers(0, nb, count))))

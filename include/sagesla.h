@@ -97,7 +97,7 @@ typedef struct {
   size_t qbar, kbar;  /* float [B*H][nb][128] block means */
   size_t ksum_part;   /* double [B*H][nb][128] per-block K channel sums */
   size_t vmax_part;   /* float [B*H][nb][128] per-block V channel amax */
-  size_t scores;      /* float [B*H][nb][nb] raw block dot products */
+  size_t scores;      /* float [B*H][nb][ld] raw block dot products, ld = nb rounded up to 4 */
   size_t kept;        /* int32 [B*H][nb][k] */
   size_t mask;        /* uint32 [B*H][nb][mask_words] */
   size_t amask;       /* bf16 [B*H][nb_m_pad][nb_k_pad] complement mask (1 = not kept) */

@@ -24,6 +24,7 @@ struct ForwardPlan {
   int64_t n_pairs;     // ceil(nb / 2)
   int64_t n_pad;       // 128 * n_pairs token rows per head in the code buffers
   int64_t mask_words;  // ceil(nb / 32)
+  int64_t scores_ld;   // row stride of the block scores: nb rounded up to a multiple of 4
   int64_t nb_k_pad;    // nb rounded up to 64 (K extent of the complement-sum GEMM)
   int64_t nb_m_pad;    // nb rounded up to 128 (M extent of the complement-sum GEMM)
   int32_t n_last;      // tokens in the last block

@@ -51,6 +51,7 @@ bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* 
   p->n_pairs = ceil_div(p->nb, 2);
   p->n_pad = 128 * p->n_pairs;
   p->mask_words = ceil_div(p->nb, 32);
+  p->scores_ld = ceil_div(p->nb, 4) * 4;
   p->nb_k_pad = ceil_div(p->nb, 64) * 64;
   p->nb_m_pad = ceil_div(p->nb, 128) * 128;
   p->n_last = static_cast<int32_t>(N - kBlock * (p->nb - 1));
@@ -87,7 +88,7 @@ bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* 
   L.kbar = take(static_cast<size_t>(BH * nb * 128) * 4);
   L.ksum_part = take(static_cast<size_t>(BH * nb * 128) * 8);
   L.vmax_part = take(static_cast<size_t>(BH * nb * 128) * 4);
-  L.scores = take(static_cast<size_t>(BH * nb * nb) * 4);
+  L.scores = take(static_cast<size_t>(BH * nb * p->scores_ld) * 4);
   L.kept = take(static_cast<size_t>(BH * nb * p->k) * 4);
   L.mask = take(static_cast<size_t>(BH * nb * p->mask_words) * 4);
   L.amask = take(static_cast<size_t>(BH * p->nb_m_pad * p->nb_k_pad) * 2);

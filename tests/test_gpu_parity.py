@@ -110,6 +110,28 @@ def test_dense_mode(n, seed):
     assert torch.equal(plain["out"], res["out"])
 
 
+@pytest.mark.parametrize("n", [4096, 2050 * 64])
+def test_equal_scores_keep_the_lowest_blocks(n):
+    """Constant K makes every score of a row equal: the selection keeps blocks 0..k-1."""
+    q, _, v = inputs.make_random(1, 1, n, 31)
+    k = torch.full_like(q, 0.5)
+    res = gpu_run(q, k, v, 0.05)
+    nb, kk = res["layout"]["nb"], res["layout"]["k"]
+    assert (res["kept"][0] == np.arange(kk, dtype=np.int32)[None, :]).all()
+    err, _ = compare_head(q, k, v, 0.05, res, 0, 0, rows=_sampled_rows(nb, 31, count=2))
+    assert err <= OUT_TOL, err
+
+
+def test_long_rows_block_topk():
+    """More than 2048 key blocks per row: the selection takes the one-CTA-per-row path."""
+    q, k, v = inputs.make_random(1, 1, 2050 * 64 - 10, 29, k_offset_std=0.5)
+    res = gpu_run(q, k, v, 0.02, extras=True)
+    nb = res["layout"]["nb"]
+    assert nb == 2050
+    err, _ = compare_head(q, k, v, 0.02, res, 0, 0, rows=_sampled_rows(nb, 29, count=4))
+    assert err <= OUT_TOL, err
+
+
 def test_dense_mode_full_size_sampled():
     """r = 1 on the Wan2.1-1.3B-480P shape (512 kept blocks per query block), sampled rows."""
     q, k, v = inputs.make_qkv("wan21_1p3b_480p", heads=2)

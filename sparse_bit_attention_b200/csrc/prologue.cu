@@ -110,15 +110,23 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
 #pragma unroll
   for (int e = 0; e < 8; ++e) { ksum[e] = 0.0; vmax[e] = 0.f; psum[e] = 0.f; }
 
-#pragma unroll 2
+  // all of this thread's K and V chunks in flight at once (8 + 8 x 16 bytes)
+  uint4 kreg[8], vreg[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int r = g + 8 * s;
+    kreg[s] = make_uint4(0, 0, 0, 0);
+    vreg[s] = make_uint4(0, 0, 0, 0);
+    if (r < nj) {
+      kreg[s] = ld_row_chunk(kb, (n0 + r) * K.stride_n + 8 * ch);
+      vreg[s] = ld_row_chunk(vb, (n0 + r) * V.stride_n + 8 * ch);
+    }
+  }
+#pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int r = g + 8 * s;
     const bool valid = r < nj;
-    uint4 kraw = make_uint4(0, 0, 0, 0), vraw = make_uint4(0, 0, 0, 0);
-    if (valid) {
-      kraw = ld_row_chunk(kb, (n0 + r) * K.stride_n + 8 * ch);
-      vraw = ld_row_chunk(vb, (n0 + r) * V.stride_n + 8 * ch);
-    }
+    const uint4 kraw = kreg[s], vraw = vreg[s];
     float kf[8], vf[8];
     unpack_bf16x8(kraw, kf);
     unpack_bf16x8(vraw, vf);
@@ -193,8 +201,11 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
 
   const bool ok = mbar_wait(bar, 0, status);
   tc_fence_after();
+  // H_j[c][n] (TMEM lane c, column n) -> bf16 tile [n][c] in the freed operand tiles, then
+  // 16-byte stores of the contiguous 32 KB of the row.
+  uint16_t* stage = reinterpret_cast<uint16_t*>(smem);
   if (ok) {
-    const int c = 32 * warp + lane;   // TMEM lane = channel
+    const int c = 32 * warp + lane;
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t r[32];
@@ -202,11 +213,17 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
       tmem_ld_wait();
 #pragma unroll
       for (int e = 0; e < 32; ++e)
-        hrow[(32 * cc + e) * 128 + c] = __float2bfloat16_rn(__uint_as_float(r[e]));
+        stage[(32 * cc + e) * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[e])));
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (ok) {
+    const uint4* src = reinterpret_cast<const uint4*>(stage);
+    uint4* dst = reinterpret_cast<uint4*>(hrow);
+#pragma unroll 4
+    for (int e = t; e < 128 * 128 / 8; e += kStatsThreads) dst[e] = src[e];
+  }
   if (warp == 0) tmem_dealloc(tmem, 128);
 }
 

@@ -4,3 +4,4 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of ``benc
 import this package. The product path never does.
 """
 from .sagesla_oracle import *  # noqa: F401,F403
+from . import norm_oracle  # noqa: F401,E402

@@ -419,6 +419,30 @@ def _time_sdpa(torch, q, k, v, steps, warmup):
     return None, None
 
 
+def _time_norm(sba, torch, steps, warmup):
+    """Fused LayerNorm + AdaLN modulation + per-token INT8 codes on the 14B-720P token rows
+    (75600 x 5120 bf16): device time per call and HBM bytes per call."""
+    M, K = 75600, 5120
+    g = torch.Generator().manual_seed(11)
+    x = (torch.randn(M, K, generator=g) * 1.5).to(torch.bfloat16).cuda()
+    scale = (torch.randn(1, K, generator=g) * 0.2).to(torch.bfloat16).cuda()
+    shift = (torch.randn(1, K, generator=g) * 0.5).to(torch.bfloat16).cuda()
+    for _ in range(warmup):
+        sba.sagesla_norm_quant(x, sba.SAGESLA_LAYER_NORM, 1e-6, None, None, scale, shift,
+                               rows_per_sample=M, want_codes=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        sba.sagesla_norm_quant(x, sba.SAGESLA_LAYER_NORM, 1e-6, None, None, scale, shift,
+                               rows_per_sample=M, want_codes=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    nbytes = M * K * 2 + M * K * 2 + M * K + M * 4      # x in, bf16 y out, codes out, scales
+    return M, K, ms, nbytes
+
+
 def run_sweep(args):
     import torch
     import sparse_bit_attention_b200 as sba
@@ -452,6 +476,14 @@ def run_sweep(args):
                 "dense_tflops": dense_ops / (ms / 1e3) / 1e12 if ms else None}), flush=True)
         del q, k, v
         torch.cuda.empty_cache()
+    M, K, ms, nbytes = _time_norm(sba, torch, steps, args.warmup)
+    peaks, src = measured_peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    print(json.dumps({
+        "sweep": "fused_norm", "op": "LayerNorm + AdaLN modulation + bf16 out + per-token INT8",
+        "M": M, "K": K, "ms_per_call": ms, "hbm_bytes": nbytes, "achieved_gbs": gbs,
+        "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"], "peak_source": src}),
+        flush=True)
     return 0
 
 

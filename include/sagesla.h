@@ -180,6 +180,48 @@ sagesla_status sagesla_forward_no_alloc(const sagesla_tensor* q, const sagesla_t
                                         const sagesla_tensor* v, double topk_ratio, int block,
                                         sagesla_tensor* out, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Fused normalization, modulation and INT8 activation quantization: the LayerNorm / RMSNorm
+ * of a DiT block feeding an 8-bit linear layer. News.qq.com TurboDiffusion article, section
+ * 第四把钥匙 (LayerNorm and RMSNorm rewritten and fused with neighbouring operations so that
+ * data crosses memory fewer times) and section 第三把钥匙 (activations quantized to INT8 on
+ * the fly). Per token row x (bf16, K channels):
+ *   LayerNorm: y = (x - mean) / sqrt(var + eps), then y * gamma + beta   (biased variance)
+ *   RMSNorm:   y = x / sqrt(mean(x^2) + eps), then y * gamma
+ *   modulation, if given: y = y * (1 + scale[b]) + shift[b], b = row / rows_per_sample
+ *   y_out = bf16(y) (round to nearest even)
+ *   INT8, if asked: a = max |y_out| over the row; code = clamp(rne(y_out * fl32(127 / a)),
+ *   -127, 127) and code_scale = fl32(a / 127); a = 0 gives scale 1 and zero codes.
+ * The arithmetic is fp32 (fp32 sums over the row), so y_out can differ by one bf16 ulp from
+ * the real-number y rounded to bf16; the codes are exact functions of y_out. */
+typedef enum { SAGESLA_LAYER_NORM = 0, SAGESLA_RMS_NORM = 1 } sagesla_norm_kind;
+
+typedef struct {
+  const uint16_t* x;       /* bf16 [M][K] device (read only), row stride x_stride elements */
+  int64_t M, K, x_stride;
+  int32_t kind;            /* sagesla_norm_kind */
+  float eps;               /* >= 0, finite */
+  const uint16_t* gamma;   /* bf16 [K] or NULL (1) */
+  const uint16_t* beta;    /* bf16 [K] or NULL (0); LayerNorm only */
+  const uint16_t* scale;   /* bf16 [ceil(M / rows_per_sample)][K] or NULL (0) */
+  const uint16_t* shift;   /* same shape as scale, or NULL (0) */
+  int64_t rows_per_sample; /* >= 1 when scale or shift is given */
+  uint16_t* y;             /* bf16 [M][K] out, row stride y_stride elements, or NULL */
+  int64_t y_stride;
+  int8_t* codes;           /* int8 [M][K] out, row stride codes_stride bytes, or NULL */
+  int64_t codes_stride;
+  float* code_scale;       /* float [M] out, given exactly when codes is given */
+} sagesla_norm_args;
+
+/* Runs the fused normalization asynchronously on `stream` (cudaStream_t as void*); all
+ * pointers are device pointers owned by the caller. Requirements: M >= 1; 8 <= K <= 16384
+ * and K a multiple of 8; x and y rows 16-byte aligned (strides multiples of 8 elements, at
+ * least K), codes rows 8-byte aligned (stride a multiple of 8, at least K); gamma, beta,
+ * scale, shift 16-byte aligned; at least one of y and codes; the outputs must not overlap x.
+ * Errors: INVALID_ARG (bad pointers, strides, kind, eps), UNSUPPORTED (K out of range),
+ * CUDA, NO_DEVICE (nothing launched in every case). */
+sagesla_status sagesla_norm_quant(const sagesla_norm_args* args, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device status word of `workspace`
  * (the one used by the last forward on that workspace). Returns SAGESLA_OK, TIMEOUT,
  * DEVICE_CHECK, or CUDA if the stream reported an error. */

@@ -4,5 +4,6 @@ from .binding import (  # noqa: F401
     SAGESLA_BF16, SAGESLA_F32, SageslaError, alloc_workspace, load_library,
     sagesla_forward, sagesla_forward_host, sagesla_get_workspace_layout,
     sagesla_host_workspace_size, sagesla_status_string, sagesla_stream_status,
-    sagesla_topk_count, sagesla_workspace_size,
+    sagesla_topk_count, sagesla_workspace_size, SAGESLA_LAYER_NORM, SAGESLA_RMS_NORM,
+    sagesla_norm_quant,
 )

@@ -61,6 +61,19 @@ class SageslaWorkspaceLayout(ctypes.Structure):
                 [(n, ctypes.c_size_t) for n in _LAYOUT_FIELDS])
 
 
+SAGESLA_LAYER_NORM = 0
+SAGESLA_RMS_NORM = 1
+
+
+class SageslaNormArgs(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("M", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("x_stride", ctypes.c_int64), ("kind", ctypes.c_int32), ("eps", ctypes.c_float),
+                ("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("scale", ctypes.c_void_p),
+                ("shift", ctypes.c_void_p), ("rows_per_sample", ctypes.c_int64),
+                ("y", ctypes.c_void_p), ("y_stride", ctypes.c_int64), ("codes", ctypes.c_void_p),
+                ("codes_stride", ctypes.c_int64), ("code_scale", ctypes.c_void_p)]
+
+
 # Every symbol the header declares, with its signature.
 _SIGNATURES = {
     "sagesla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -82,6 +95,7 @@ _SIGNATURES = {
     "sagesla_stream_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "sagesla_forward_no_alloc": (ctypes.c_int, [ctypes.POINTER(SageslaTensor)] * 3 + [
         ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaTensor), ctypes.c_void_p]),
+    "sagesla_norm_quant": (ctypes.c_int, [ctypes.POINTER(SageslaNormArgs), ctypes.c_void_p]),
 }
 
 NO_ALLOC_SCRATCH_BYTES = 64 << 20
@@ -247,3 +261,31 @@ def sagesla_forward_no_alloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
                                         ctypes.c_void_p(_stream_ptr(stream))),
            "sagesla_forward_no_alloc")
     return out
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def sagesla_norm_quant(x: torch.Tensor, kind: int = SAGESLA_LAYER_NORM, eps: float = 1e-6,
+                       gamma=None, beta=None, scale=None, shift=None, rows_per_sample: int = 0,
+                       want_y: bool = True, want_codes: bool = False, stream=None):
+    """Fused LayerNorm / RMSNorm (+ modulation) of the rows of a bf16 [M, K] device tensor
+    (last dimension contiguous). Returns (y bf16 [M, K] or None, codes int8 [M, K] or None,
+    code_scale float32 [M] or None)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [M, K] tensor with contiguous rows")
+    M, K = x.shape
+    y = torch.empty((M, K), dtype=torch.bfloat16, device=x.device) if want_y else None
+    codes = torch.empty((M, K), dtype=torch.int8, device=x.device) if want_codes else None
+    cs = torch.empty((M,), dtype=torch.float32, device=x.device) if want_codes else None
+    for v in (gamma, beta, scale, shift):
+        if v is not None and (v.dtype != torch.bfloat16 or not v.is_contiguous()):
+            raise ValueError("gamma, beta, scale, shift must be contiguous bf16 tensors")
+    args = SageslaNormArgs(x.data_ptr(), M, K, x.stride(0), kind, eps, _ptr(gamma), _ptr(beta),
+                           _ptr(scale), _ptr(shift), rows_per_sample, _ptr(y), K, _ptr(codes), K,
+                           _ptr(cs))
+    _check(load_library().sagesla_norm_quant(ctypes.byref(args),
+                                             ctypes.c_void_p(_stream_ptr(stream))),
+           "sagesla_norm_quant")
+    return y, codes, cs

@@ -48,6 +48,10 @@ cudaError_t launch_quant(const ForwardPlan& p, TensorArg q, TensorArg k, TensorA
                          cudaStream_t stream);
 cudaError_t launch_scores(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_topk(const ForwardPlan& p, char* ws, cudaStream_t stream);
+// SAGESLA_OK when the current device is a compute-capability-10.0 part (B200), else
+// SAGESLA_ERR_NO_DEVICE.
+sagesla_status require_b200();
+
 cudaError_t launch_fill_all_kept(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_complement_gemm(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32_t out_dtype,

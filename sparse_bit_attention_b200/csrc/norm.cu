@@ -1,0 +1,257 @@
+// Fused LayerNorm / RMSNorm + AdaLN modulation + per-token INT8 quantization.
+//
+// News.qq.com TurboDiffusion article, section 第四把钥匙: LayerNorm and RMSNorm are rewritten
+// and fused with their neighbouring operations so that the data crosses memory fewer times;
+// section 第三把钥匙: the activations of the 8-bit linear layers are quantized to INT8 on the
+// fly. Here one pass over a token row reads the bf16 row once and writes the normalized,
+// modulated row (bf16) and/or its INT8 codes with one scale per row.
+//
+// B200 mapping: one 128-thread CTA per row. Each thread holds its chunks of 8 channels
+// (16-byte loads; up to 16 chunks, K <= 16384; the count is a template parameter so that the
+// registers, and with them the occupancy, follow K) in registers, so the row is read from HBM exactly once; the
+// mean / variance (or mean square) and the row's absolute maximum are block reductions
+// (warp shuffles, then 4 warp partials in shared memory). The kernel is bound by HBM
+// bandwidth: per row 2K bytes in, 2K bytes of bf16 and K bytes of codes out.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sagesla {
+
+namespace {
+
+constexpr int kNormThreads = 128;
+constexpr int kMaxChunks = 16;              // 16 x 8 x 128 = 16384 channels
+
+struct NormParams {
+  const uint16_t* x;
+  int64_t x_stride;
+  int K, kind;
+  float eps;
+  const uint16_t *gamma, *beta, *scale, *shift;
+  int64_t rows_per_sample;
+  uint16_t* y;
+  int64_t y_stride;
+  int8_t* codes;
+  int64_t codes_stride;
+  float* code_scale;
+};
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Sum over the CTA of one float per thread (every thread gets the total).
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  return (red[0] + red[1]) + (red[2] + red[3]);
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+}
+
+// kCh = chunks of 8 channels per thread (K <= 8 * 128 * kCh): the row stays in registers.
+template <int kCh>
+__global__ void __launch_bounds__(kNormThreads)
+k_norm_quant(NormParams p) {
+  __shared__ float red[4];
+  const int64_t row = blockIdx.x;
+  const int t = threadIdx.x;
+  const int nch = p.K >> 3;                   // 8-channel chunks; thread t takes t + 128 i
+  const uint4* xr = reinterpret_cast<const uint4*>(p.x + row * p.x_stride);
+
+  uint4 raw[kCh];
+#pragma unroll
+  for (int i = 0; i < kCh; ++i)
+    raw[i] = (t + kNormThreads * i < nch) ? __ldg(xr + t + kNormThreads * i) : make_uint4(0, 0, 0, 0);
+
+  // statistics (fp32 sums; padded chunks hold zeros and are left out of the LayerNorm
+  // deviations)
+  const float inv_k = 1.0f / static_cast<float>(p.K);
+  float mu = 0.f, rstd;
+  if (p.kind == SAGESLA_LAYER_NORM) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kCh; ++i) {
+      float f[8];
+      unpack8(raw[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += f[e];
+    }
+    mu = block_sum(s, red) * inv_k;
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < kCh; ++i) {
+      if (t + kNormThreads * i >= nch) continue;
+      float f[8];
+      unpack8(raw[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = f[e] - mu;
+        q = fmaf(d, d, q);
+      }
+    }
+    rstd = 1.0f / sqrtf(block_sum(q, red) * inv_k + p.eps);
+  } else {
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < kCh; ++i) {
+      float f[8];
+      unpack8(raw[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) q = fmaf(f[e], f[e], q);
+    }
+    rstd = 1.0f / sqrtf(block_sum(q, red) * inv_k + p.eps);
+  }
+
+  // normalize, affine, modulate, round to bf16 (kept in raw[] for the quantization)
+  const int64_t b = p.rows_per_sample > 0 ? row / p.rows_per_sample : 0;
+  const uint4* g4 = reinterpret_cast<const uint4*>(p.gamma);
+  const uint4* be4 = reinterpret_cast<const uint4*>(p.beta);
+  const uint4* sc4 = p.scale ? reinterpret_cast<const uint4*>(p.scale + b * p.K) : nullptr;
+  const uint4* sh4 = p.shift ? reinterpret_cast<const uint4*>(p.shift + b * p.K) : nullptr;
+  uint4* yr = p.y ? reinterpret_cast<uint4*>(p.y + row * p.y_stride) : nullptr;
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kCh; ++i) {
+    const int c = t + kNormThreads * i;
+    if (c >= nch) continue;
+    float f[8], g[8], be[8], sc[8], sh[8];
+    unpack8(raw[i], f);
+    if (g4) unpack8(__ldg(g4 + c), g);
+    if (be4) unpack8(__ldg(be4 + c), be);
+    if (sc4) unpack8(__ldg(sc4 + c), sc);
+    if (sh4) unpack8(__ldg(sh4 + c), sh);
+    uint32_t packed[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      float v[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float y = (f[e + u] - mu) * rstd;
+        if (g4) y *= g[e + u];
+        if (be4) y += be[e + u];
+        if (sc4) y *= 1.0f + sc[e + u];
+        if (sh4) y += sh[e + u];
+        v[u] = y;
+      }
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[0], v[1]);
+      packed[e >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+      amax = fmaxf(amax, fmaxf(fabsf(__low2float(h2)), fabsf(__high2float(h2))));
+    }
+    raw[i] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    if (yr) yr[c] = raw[i];
+  }
+  if (!p.codes) return;
+
+  // per-row INT8 codes of the bf16 row: inv = fl32(127 / a), code = rne(fl32(y * inv))
+  const float a = block_max(amax, red);
+  const float inv = a > 0.f ? 127.0f / a : 0.f;
+  uint2* cr = reinterpret_cast<uint2*>(p.codes + row * p.codes_stride);
+#pragma unroll
+  for (int i = 0; i < kCh; ++i) {
+    const int c = t + kNormThreads * i;
+    if (c >= nch) continue;
+    float f[8];
+    unpack8(raw[i], f);
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float q = fminf(fmaxf(rintf(f[e] * inv), -127.f), 127.f);
+      w[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(q)) & 0xFFu) << (8 * (e & 3));
+    }
+    cr[c] = make_uint2(w[0], w[1]);
+  }
+  if (t == 0) p.code_scale[row] = a > 0.f ? a / 127.0f : 1.0f;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool overlaps(const void* a0, size_t na, const void* b0, size_t nb) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(a0), b = reinterpret_cast<uintptr_t>(b0);
+  return a < b + nb && b < a + na;
+}
+
+}  // namespace
+}  // namespace sagesla
+
+extern "C" sagesla_status sagesla_norm_quant(const sagesla_norm_args* a, void* stream) {
+  using namespace sagesla;
+  if (!a || !a->x) return SAGESLA_ERR_INVALID_ARG;
+  if (a->M < 1 || a->K < 1) return SAGESLA_ERR_INVALID_ARG;
+  if (a->K < 8 || a->K > 8 * kNormThreads * kMaxChunks || a->K % 8 != 0) return SAGESLA_ERR_UNSUPPORTED;
+  if (a->M > 0x7FFFFFFF) return SAGESLA_ERR_UNSUPPORTED;
+  if (a->kind != SAGESLA_LAYER_NORM && a->kind != SAGESLA_RMS_NORM) return SAGESLA_ERR_INVALID_ARG;
+  if (!(a->eps >= 0.f) || !std::isfinite(a->eps)) return SAGESLA_ERR_INVALID_ARG;
+  if (a->beta && a->kind != SAGESLA_LAYER_NORM) return SAGESLA_ERR_INVALID_ARG;
+  if (!a->y && !a->codes) return SAGESLA_ERR_INVALID_ARG;
+  if ((a->codes == nullptr) != (a->code_scale == nullptr)) return SAGESLA_ERR_INVALID_ARG;
+  if ((a->scale || a->shift) && a->rows_per_sample < 1) return SAGESLA_ERR_INVALID_ARG;
+  if (a->x_stride < a->K || a->x_stride % 8 != 0 || !aligned(a->x, 16)) return SAGESLA_ERR_INVALID_ARG;
+  for (const void* v : {static_cast<const void*>(a->gamma), static_cast<const void*>(a->beta),
+                        static_cast<const void*>(a->scale), static_cast<const void*>(a->shift)})
+    if (v && !aligned(v, 16)) return SAGESLA_ERR_INVALID_ARG;
+  const size_t x_bytes = static_cast<size_t>((a->M - 1) * a->x_stride + a->K) * 2;
+  if (a->y) {
+    if (a->y_stride < a->K || a->y_stride % 8 != 0 || !aligned(a->y, 16)) return SAGESLA_ERR_INVALID_ARG;
+    if (overlaps(a->y, static_cast<size_t>((a->M - 1) * a->y_stride + a->K) * 2, a->x, x_bytes))
+      return SAGESLA_ERR_INVALID_ARG;
+  }
+  if (a->codes) {
+    if (a->codes_stride < a->K || a->codes_stride % 8 != 0 || !aligned(a->codes, 8) ||
+        !aligned(a->code_scale, 4))
+      return SAGESLA_ERR_INVALID_ARG;
+    if (overlaps(a->codes, static_cast<size_t>((a->M - 1) * a->codes_stride + a->K), a->x, x_bytes) ||
+        overlaps(a->code_scale, static_cast<size_t>(a->M) * 4, a->x, x_bytes))
+      return SAGESLA_ERR_INVALID_ARG;
+  }
+  sagesla_status st = require_b200();
+  if (st != SAGESLA_OK) return st;
+  NormParams p;
+  p.x = a->x;
+  p.x_stride = a->x_stride;
+  p.K = static_cast<int>(a->K);
+  p.kind = a->kind;
+  p.eps = a->eps;
+  p.gamma = a->gamma;
+  p.beta = a->beta;
+  p.scale = a->scale;
+  p.shift = a->shift;
+  p.rows_per_sample = (a->scale || a->shift) ? a->rows_per_sample : 0;
+  p.y = a->y;
+  p.y_stride = a->y_stride;
+  p.codes = a->codes;
+  p.codes_stride = a->codes_stride;
+  p.code_scale = a->code_scale;
+  const int ch = static_cast<int>((a->K / 8 + kNormThreads - 1) / kNormThreads);
+  const dim3 grid(static_cast<unsigned>(a->M));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ch <= 1) k_norm_quant<1><<<grid, kNormThreads, 0, s>>>(p);
+  else if (ch <= 2) k_norm_quant<2><<<grid, kNormThreads, 0, s>>>(p);
+  else if (ch <= 3) k_norm_quant<3><<<grid, kNormThreads, 0, s>>>(p);
+  else if (ch <= 4) k_norm_quant<4><<<grid, kNormThreads, 0, s>>>(p);
+  else if (ch <= 5) k_norm_quant<5><<<grid, kNormThreads, 0, s>>>(p);
+  else if (ch <= 6) k_norm_quant<6><<<grid, kNormThreads, 0, s>>>(p);
+  else if (ch <= 8) k_norm_quant<8><<<grid, kNormThreads, 0, s>>>(p);
+  else if (ch <= 12) k_norm_quant<12><<<grid, kNormThreads, 0, s>>>(p);
+  else k_norm_quant<kMaxChunks><<<grid, kNormThreads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SAGESLA_OK : SAGESLA_ERR_CUDA;
+}

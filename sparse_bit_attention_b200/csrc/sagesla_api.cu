@@ -163,8 +163,17 @@ TensorArg to_arg(const sagesla_tensor* t) {
   return a;
 }
 
+sagesla_status check_device() { return require_b200(); }
+
+#define SAGESLA_LAUNCH(call)                            \
+  do {                                                  \
+    if ((call) != cudaSuccess) return SAGESLA_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
 // The current device must be a compute-capability-10.0 part (B200).
-sagesla_status check_device() {
+sagesla_status require_b200() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return SAGESLA_ERR_NO_DEVICE;
   int major = 0, minor = 0;
@@ -174,13 +183,6 @@ sagesla_status check_device() {
   if (major != 10 || minor != 0) return SAGESLA_ERR_NO_DEVICE;
   return SAGESLA_OK;
 }
-
-#define SAGESLA_LAUNCH(call)                            \
-  do {                                                  \
-    if ((call) != cudaSuccess) return SAGESLA_ERR_CUDA; \
-  } while (0)
-
-}  // namespace
 
 }  // namespace sagesla
 

@@ -25,6 +25,7 @@ from .sagesla_oracle import quant_int8_block, round_bf16
 
 LAYER_NORM = 0
 RMS_NORM = 1
+NO_NORM = 2        # the row itself (per-token quantization of any activation row)
 
 
 def normalize_rows(x, kind: int, eps: float, gamma=None, beta=None):
@@ -47,6 +48,8 @@ def normalize_rows(x, kind: int, eps: float, gamma=None, beta=None):
         if gamma is not None:
             y = y * np.asarray(gamma, dtype=np.float64)
         return y
+    if kind == NO_NORM:
+        return x.copy()
     raise ValueError(f"unknown normalization kind {kind}")
 
 

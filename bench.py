@@ -443,6 +443,34 @@ def _time_norm(sba, torch, steps, warmup):
     return M, K, ms, nbytes
 
 
+def _time_w8a8(sba, torch, steps, warmup, M=75600, K=5120, N=5120):
+    """W8A8 projection of the 14B-720P token rows (M x K int8 codes, N x K block-quantized
+    weights, bf16 output with bias) and the same layer in bf16 through torch.matmul."""
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(M, K, generator=g) * 1.5).to(torch.bfloat16).cuda()
+    w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).cuda()
+    bias = (torch.randn(N, generator=g) * 0.1).to(torch.bfloat16).cuda()
+    _, x8, s_x = sba.sagesla_norm_quant(x, sba.SAGESLA_NO_NORM, 0.0, want_y=False, want_codes=True)
+    w8, s_w = sba.sagesla_w8a8_quantize_weight(w)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    ms_w8 = timed(lambda: sba.sagesla_w8a8_gemm(x8, s_x, w8, s_w, bias, out=y))
+    ms_bf16 = timed(lambda: torch.addmm(bias, x, w.t()))
+    return M, K, N, ms_w8, ms_bf16
+
+
 def run_sweep(args):
     import torch
     import sparse_bit_attention_b200 as sba
@@ -484,6 +512,16 @@ def run_sweep(args):
         "M": M, "K": K, "ms_per_call": ms, "hbm_bytes": nbytes, "achieved_gbs": gbs,
         "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"], "peak_source": src}),
         flush=True)
+    M, K, N, ms_w8, ms_bf16 = _time_w8a8(sba, torch, steps, args.warmup)
+    ops = 2.0 * M * N * K
+    peak_int8 = 2.0 * peaks["bf16_tflops_sustained"]
+    print(json.dumps({
+        "sweep": "w8a8_linear", "M": M, "K": K, "N": N, "ms_per_call": ms_w8,
+        "tops": ops / (ms_w8 / 1e3) / 1e12, "peak_tops": peak_int8,
+        "frac": ops / (ms_w8 / 1e3) / 1e12 / peak_int8,
+        "peak_source": f"{src}: 2 x bf16_tflops_sustained",
+        "bf16_torch_ms": ms_bf16, "bf16_torch_tflops": ops / (ms_bf16 / 1e3) / 1e12,
+        "speedup_vs_bf16": ms_bf16 / ms_w8}), flush=True)
     return 0
 
 

@@ -188,20 +188,21 @@ sagesla_status sagesla_forward_no_alloc(const sagesla_tensor* q, const sagesla_t
  * the fly). Per token row x (bf16, K channels):
  *   LayerNorm: y = (x - mean) / sqrt(var + eps), then y * gamma + beta   (biased variance)
  *   RMSNorm:   y = x / sqrt(mean(x^2) + eps), then y * gamma
+ *   none:      y = x (the per-token INT8 quantizer of any activation row)
  *   modulation, if given: y = y * (1 + scale[b]) + shift[b], b = row / rows_per_sample
  *   y_out = bf16(y) (round to nearest even)
  *   INT8, if asked: a = max |y_out| over the row; code = clamp(rne(y_out * fl32(127 / a)),
  *   -127, 127) and code_scale = fl32(a / 127); a = 0 gives scale 1 and zero codes.
  * The arithmetic is fp32 (fp32 sums over the row), so y_out can differ by one bf16 ulp from
  * the real-number y rounded to bf16; the codes are exact functions of y_out. */
-typedef enum { SAGESLA_LAYER_NORM = 0, SAGESLA_RMS_NORM = 1 } sagesla_norm_kind;
+typedef enum { SAGESLA_LAYER_NORM = 0, SAGESLA_RMS_NORM = 1, SAGESLA_NO_NORM = 2 } sagesla_norm_kind;
 
 typedef struct {
   const uint16_t* x;       /* bf16 [M][K] device (read only), row stride x_stride elements */
   int64_t M, K, x_stride;
   int32_t kind;            /* sagesla_norm_kind */
   float eps;               /* >= 0, finite */
-  const uint16_t* gamma;   /* bf16 [K] or NULL (1) */
+  const uint16_t* gamma;   /* bf16 [K] or NULL (1); not with SAGESLA_NO_NORM */
   const uint16_t* beta;    /* bf16 [K] or NULL (0); LayerNorm only */
   const uint16_t* scale;   /* bf16 [ceil(M / rows_per_sample)][K] or NULL (0) */
   const uint16_t* shift;   /* same shape as scale, or NULL (0) */
@@ -221,6 +222,43 @@ typedef struct {
  * Errors: INVALID_ARG (bad pointers, strides, kind, eps), UNSUPPORTED (K out of range),
  * CUDA, NO_DEVICE (nothing launched in every case). */
 sagesla_status sagesla_norm_quant(const sagesla_norm_args* args, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * W8A8 linear layer: INT8 weights in 128x128 blocks with one scale per block, INT8
+ * activations with one scale per token row, the GEMM on the INT8 tensor cores.
+ * News.qq.com TurboDiffusion article, section 第三把钥匙 (weights and activations both in
+ * 8-bit integers so that the whole linear layer runs in the integer domain; block-wise weight
+ * quantization with 128x128 blocks; activations quantized on the fly). The activation codes
+ * come from sagesla_norm_quant (any kind, including SAGESLA_NO_NORM). */
+
+/* Offline weight quantization. w: bf16 [N][K] device, row stride w_stride elements (a
+ * multiple of 8, at least K, 16-byte aligned base); K a multiple of 128 (<= 2^20), N >= 1.
+ * For each block of rows 128*bn.. (the last block may hold fewer rows) and columns
+ * 128*bk..128*bk+127: a = max |w|; a = 0 gives scale 1 and zero codes, else code =
+ * clamp(rne(w * fl32(127 / a)), -127, 127), w_scale[bn][bk] = fl32(a / 127).
+ * Outputs: w8 int8 [N][K] (contiguous, 16-byte aligned), w_scale float [ceil(N/128)][K/128].
+ * Asynchronous on `stream`. Errors: INVALID_ARG, UNSUPPORTED (K not a multiple of 128),
+ * CUDA, NO_DEVICE (nothing launched). */
+sagesla_status sagesla_w8a8_quantize_weight(const uint16_t* w, int64_t N, int64_t K,
+                                            int64_t w_stride, int8_t* w8, float* w_scale,
+                                            void* stream);
+
+/* y[m][n] = x_scale[m] * sum_bk w_scale[n/128][bk] * sum_{k in block bk} x8[m][k] w8[n][k]
+ *           (+ bias[n]), summed over the K blocks in fp32 from exact int32 block products.
+ *   x8      int8 [M][K] contiguous, x_scale float [M] (per token row)
+ *   w8      int8 [N][K] contiguous, w_scale float [ceil(N/128)][K/128]
+ *   bias    bf16 [N] or NULL
+ *   y       bf16 (y_dtype SAGESLA_BF16, round to nearest even) or float (SAGESLA_F32)
+ *           [M][N], row stride y_stride elements (16-byte aligned rows)
+ *   status  device int32 or NULL: a device-side timeout of the kernel's bounded waits writes
+ *           SAGESLA_ERR_TIMEOUT there (the caller zeroes it)
+ * Requirements: M, N >= 1 (< 2^31); K a multiple of 128; N a multiple of 8; all buffers
+ * 16-byte aligned; y must not overlap the inputs. Asynchronous on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA, NO_DEVICE (nothing launched). */
+sagesla_status sagesla_w8a8_gemm(const int8_t* x8, const float* x_scale, int64_t M, int64_t K,
+                                 const int8_t* w8, const float* w_scale, int64_t N,
+                                 const uint16_t* bias, void* y, int32_t y_dtype,
+                                 int64_t y_stride, int32_t* status, void* stream);
 
 /* Synchronizes `stream`, then reads and clears the device status word of `workspace`
  * (the one used by the last forward on that workspace). Returns SAGESLA_OK, TIMEOUT,

@@ -5,5 +5,5 @@ from .binding import (  # noqa: F401
     sagesla_forward, sagesla_forward_host, sagesla_get_workspace_layout,
     sagesla_host_workspace_size, sagesla_status_string, sagesla_stream_status,
     sagesla_topk_count, sagesla_workspace_size, SAGESLA_LAYER_NORM, SAGESLA_RMS_NORM,
-    sagesla_norm_quant,
+    sagesla_norm_quant, SAGESLA_NO_NORM, sagesla_w8a8_quantize_weight, sagesla_w8a8_gemm,
 )

@@ -63,6 +63,8 @@ class SageslaWorkspaceLayout(ctypes.Structure):
 
 SAGESLA_LAYER_NORM = 0
 SAGESLA_RMS_NORM = 1
+SAGESLA_NO_NORM = 2
+W8A8_BLOCK = 128
 
 
 class SageslaNormArgs(ctypes.Structure):
@@ -96,6 +98,14 @@ _SIGNATURES = {
     "sagesla_forward_no_alloc": (ctypes.c_int, [ctypes.POINTER(SageslaTensor)] * 3 + [
         ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaTensor), ctypes.c_void_p]),
     "sagesla_norm_quant": (ctypes.c_int, [ctypes.POINTER(SageslaNormArgs), ctypes.c_void_p]),
+    "sagesla_w8a8_quantize_weight": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                    ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                                    ctypes.c_void_p]),
+    "sagesla_w8a8_gemm": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                         ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p,
+                                         ctypes.c_void_p]),
 }
 
 NO_ALLOC_SCRATCH_BYTES = 64 << 20
@@ -289,3 +299,43 @@ def sagesla_norm_quant(x: torch.Tensor, kind: int = SAGESLA_LAYER_NORM, eps: flo
                                              ctypes.c_void_p(_stream_ptr(stream))),
            "sagesla_norm_quant")
     return y, codes, cs
+
+
+def sagesla_w8a8_quantize_weight(w: torch.Tensor, stream=None):
+    """Block-wise (128 x 128) INT8 quantization of a bf16 [N, K] weight (rows contiguous).
+    Returns (w8 int8 [N, K], w_scale float32 [ceil(N/128), K/128])."""
+    if w.dtype != torch.bfloat16 or w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be a bf16 [N, K] tensor with contiguous rows")
+    N, K = w.shape
+    w8 = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    ws = torch.empty(((N + W8A8_BLOCK - 1) // W8A8_BLOCK, K // W8A8_BLOCK), dtype=torch.float32,
+                     device=w.device)
+    _check(load_library().sagesla_w8a8_quantize_weight(
+        ctypes.c_void_p(w.data_ptr()), N, K, w.stride(0), ctypes.c_void_p(w8.data_ptr()),
+        ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(_stream_ptr(stream))),
+        "sagesla_w8a8_quantize_weight")
+    return w8, ws
+
+
+def sagesla_w8a8_gemm(x8: torch.Tensor, x_scale: torch.Tensor, w8: torch.Tensor,
+                      w_scale: torch.Tensor, bias=None, out_dtype=torch.bfloat16, out=None,
+                      status=None, stream=None):
+    """y[m, n] = x_scale[m] * sum_bk w_scale[n/128, bk] * (x8[m, block bk] . w8[n, block bk])
+    (+ bias[n]) on the INT8 tensor cores; x8 [M, K] and w8 [N, K] contiguous int8."""
+    M, K = x8.shape
+    N = w8.shape[0]
+    for t, dt in ((x8, torch.int8), (w8, torch.int8), (x_scale, torch.float32),
+                  (w_scale, torch.float32)):
+        if t.dtype != dt or not t.is_contiguous():
+            raise ValueError("x8, w8 (int8) and x_scale, w_scale (float32) must be contiguous")
+    if bias is not None and (bias.dtype != torch.bfloat16 or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous bf16 vector")
+    y_dtype = SAGESLA_F32 if out_dtype == torch.float32 else SAGESLA_BF16
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x8.device)
+    _check(load_library().sagesla_w8a8_gemm(
+        ctypes.c_void_p(x8.data_ptr()), ctypes.c_void_p(x_scale.data_ptr()), M, K,
+        ctypes.c_void_p(w8.data_ptr()), ctypes.c_void_p(w_scale.data_ptr()), N,
+        ctypes.c_void_p(_ptr(bias)), ctypes.c_void_p(out.data_ptr()), y_dtype, out.stride(0),
+        ctypes.c_void_p(_ptr(status)), ctypes.c_void_p(_stream_ptr(stream))), "sagesla_w8a8_gemm")
+    return out

@@ -87,7 +87,9 @@ k_norm_quant(NormParams p) {
   // deviations)
   const float inv_k = 1.0f / static_cast<float>(p.K);
   float mu = 0.f, rstd;
-  if (p.kind == SAGESLA_LAYER_NORM) {
+  if (p.kind == SAGESLA_NO_NORM) {
+    rstd = 1.0f;
+  } else if (p.kind == SAGESLA_LAYER_NORM) {
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < kCh; ++i) {
@@ -199,7 +201,9 @@ extern "C" sagesla_status sagesla_norm_quant(const sagesla_norm_args* a, void* s
   if (a->M < 1 || a->K < 1) return SAGESLA_ERR_INVALID_ARG;
   if (a->K < 8 || a->K > 8 * kNormThreads * kMaxChunks || a->K % 8 != 0) return SAGESLA_ERR_UNSUPPORTED;
   if (a->M > 0x7FFFFFFF) return SAGESLA_ERR_UNSUPPORTED;
-  if (a->kind != SAGESLA_LAYER_NORM && a->kind != SAGESLA_RMS_NORM) return SAGESLA_ERR_INVALID_ARG;
+  if (a->kind != SAGESLA_LAYER_NORM && a->kind != SAGESLA_RMS_NORM && a->kind != SAGESLA_NO_NORM)
+    return SAGESLA_ERR_INVALID_ARG;
+  if (a->kind == SAGESLA_NO_NORM && a->gamma) return SAGESLA_ERR_INVALID_ARG;
   if (!(a->eps >= 0.f) || !std::isfinite(a->eps)) return SAGESLA_ERR_INVALID_ARG;
   if (a->beta && a->kind != SAGESLA_LAYER_NORM) return SAGESLA_ERR_INVALID_ARG;
   if (!a->y && !a->codes) return SAGESLA_ERR_INVALID_ARG;

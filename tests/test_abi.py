@@ -22,7 +22,7 @@ def built_library():
 
 def _header_functions():
     text = open(os.path.join(ROOT, "include", "sagesla.h")).read()
-    return sorted(set(re.findall(r"\b(sagesla_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(sagesla_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported():

@@ -142,15 +142,19 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
                                   sagesla_tensor* out, void* workspace, size_t workspace_bytes,
                                   void* stream, const sagesla_options* opt);
 
-/* Bytes of device workspace sagesla_forward_host needs (the forward workspace plus device
- * copies of Q, K, V and the output); 0 for invalid arguments. */
+/* Bytes of device workspace sagesla_forward_host needs: the forward workspace for a chunk
+ * of ceil(B*H / min(B*H, 16)) heads, two slots of that chunk's Q, K, V and output, and one
+ * status word per chunk; 0 for invalid arguments. */
 size_t sagesla_host_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                    double topk_ratio, int block, int32_t out_dtype);
 
 /* Forward on HOST buffers: contiguous [B,H,N,128] bf16 inputs (uint16 bit patterns) and a
  * contiguous bf16/f32 output in host memory (page-locked memory gives asynchronous copies).
- * Copies the inputs into `workspace`, runs the forward there, copies the output back and
- * synchronizes `stream` before returning. Also returns device-side errors (TIMEOUT). */
+ * Works through the heads in up to 16 chunks: the host->device copy of one chunk (its own
+ * stream), the forward of the previous chunk (on `stream`) and the device->host copy of the
+ * one before (its own stream) overlap. The copies start after the work already queued on
+ * `stream`; the call synchronizes `stream` before returning and also returns device-side
+ * errors (TIMEOUT) of any chunk. */
 sagesla_status sagesla_forward_host(const uint16_t* q_host, const uint16_t* k_host,
                                     const uint16_t* v_host, int64_t B, int64_t H, int64_t N,
                                     int64_t D, double topk_ratio, int block, void* out_host,

@@ -303,13 +303,49 @@ sagesla_status sagesla_forward(const sagesla_tensor* q, const sagesla_tensor* k,
                             nullptr);
 }
 
+}  // extern "C"
+
+namespace sagesla {
+namespace {
+// The host entry point works through the heads in chunks so that the host->device copy of
+// one chunk, the forward of the previous one and the device->host copy of the one before
+// overlap (three streams). Device memory: one forward workspace for a chunk of heads, two
+// slots of chunk inputs and outputs, and one status word per chunk.
+constexpr int64_t kHostChunks = 16;
+
+int64_t host_chunk_heads(int64_t BH) { return ceil_div(BH, BH < kHostChunks ? BH : kHostChunks); }
+
+struct HostPlan {
+  int64_t hc, nchunks;
+  size_t fw, in_bytes, out_bytes, slot_bytes, status_off, total;
+};
+
+bool host_plan(int64_t B, int64_t H, int64_t N, int64_t D, double topk_ratio, int block,
+               int32_t out_dtype, HostPlan* hp) {
+  if (out_dtype != SAGESLA_BF16 && out_dtype != SAGESLA_F32) return false;
+  if (B < 1 || H < 1 || sagesla_workspace_size(B, H, N, D, topk_ratio, block) == 0) return false;
+  const int64_t BH = B * H;
+  hp->hc = host_chunk_heads(BH);
+  hp->nchunks = ceil_div(BH, hp->hc);
+  hp->fw = sagesla_workspace_size(1, hp->hc, N, D, topk_ratio, block);
+  if (hp->fw == 0) return false;
+  const size_t elems = static_cast<size_t>(hp->hc * N * D);
+  hp->in_bytes = align_up(elems * 2, kAlign);
+  hp->out_bytes = align_up(elems * elem_bytes(out_dtype), kAlign);
+  hp->slot_bytes = 3 * hp->in_bytes + hp->out_bytes;
+  hp->status_off = hp->fw + 2 * hp->slot_bytes;
+  hp->total = hp->status_off + align_up(static_cast<size_t>(hp->nchunks) * 4, kAlign);
+  return true;
+}
+}  // namespace
+}  // namespace sagesla
+
+extern "C" {
+
 size_t sagesla_host_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
                                    double topk_ratio, int block, int32_t out_dtype) {
-  if (out_dtype != SAGESLA_BF16 && out_dtype != SAGESLA_F32) return 0;
-  const size_t fw = sagesla_workspace_size(B, H, N, D, topk_ratio, block);
-  if (fw == 0) return 0;
-  const size_t elems = static_cast<size_t>(B * H * N * D);
-  return fw + 3 * align_up(elems * 2, kAlign) + align_up(elems * elem_bytes(out_dtype), kAlign);
+  HostPlan hp;
+  return host_plan(B, H, N, D, topk_ratio, block, out_dtype, &hp) ? hp.total : 0;
 }
 
 sagesla_status sagesla_stream_status(void* stream_ptr, void* workspace) {
@@ -333,46 +369,102 @@ sagesla_status sagesla_forward_host(const uint16_t* q_host, const uint16_t* k_ho
                                     int32_t out_dtype, void* workspace, size_t workspace_bytes,
                                     void* stream_ptr) {
   if (!q_host || !k_host || !v_host || !out_host) return SAGESLA_ERR_INVALID_ARG;
-  const size_t need = sagesla_host_workspace_size(B, H, N, D, topk_ratio, block, out_dtype);
-  if (need == 0) {
+  HostPlan hp;
+  if (!host_plan(B, H, N, D, topk_ratio, block, out_dtype, &hp)) {
     if (D != kHeadDim || block != kBlock) return SAGESLA_ERR_UNSUPPORTED;
     return SAGESLA_ERR_INVALID_ARG;
   }
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
-      workspace_bytes < need)
+      workspace_bytes < hp.total)
     return SAGESLA_ERR_WORKSPACE;
-  const size_t fw = sagesla_workspace_size(B, H, N, D, topk_ratio, block);
-  const size_t elems = static_cast<size_t>(B * H * N * D);
-  const size_t in_bytes = elems * 2, out_bytes = elems * elem_bytes(out_dtype);
-  char* base = static_cast<char*>(workspace);
-  char* dq = base + fw;
-  char* dk = dq + align_up(in_bytes, kAlign);
-  char* dv = dk + align_up(in_bytes, kAlign);
-  char* dout = dv + align_up(in_bytes, kAlign);
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   sagesla_status st = check_device();
   if (st != SAGESLA_OK) return st;
-  if (cudaMemcpyAsync(dq, q_host, in_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k_host, in_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v_host, in_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
-    return SAGESLA_ERR_CUDA;
-  auto view = [&](void* data, int32_t dt) {
-    sagesla_tensor t;
-    t.data = data;
-    t.dtype = dt;
-    t.B = B; t.H = H; t.N = N; t.D = D;
-    t.stride_n = D;
-    t.stride_h = N * D;
-    t.stride_b = H * N * D;
-    return t;
+  char* base = static_cast<char*>(workspace);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  const int64_t BH = B * H;
+  const size_t head_elems = static_cast<size_t>(N * D);
+  const size_t out_esz = elem_bytes(out_dtype);
+
+  // Copy streams and the events that order the three stages (per call, so that concurrent
+  // calls with their own workspaces stay independent).
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t in_ready[2] = {}, computed[2] = {}, out_free[2] = {};
+  auto cleanup = [&]() {
+    for (int s = 0; s < 2; ++s) {
+      if (in_ready[s]) cudaEventDestroy(in_ready[s]);
+      if (computed[s]) cudaEventDestroy(computed[s]);
+      if (out_free[s]) cudaEventDestroy(out_free[s]);
+    }
+    if (h2d) cudaStreamDestroy(h2d);
+    if (d2h) cudaStreamDestroy(d2h);
   };
-  sagesla_tensor tq = view(dq, SAGESLA_BF16), tk = view(dk, SAGESLA_BF16),
-                 tv = view(dv, SAGESLA_BF16), to = view(dout, out_dtype);
-  st = sagesla_forward(&tq, &tk, &tv, topk_ratio, block, &to, base, fw, stream_ptr);
-  if (st != SAGESLA_OK) return st;
-  if (cudaMemcpyAsync(out_host, dout, out_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+  bool ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess;
+  for (int s = 0; s < 2 && ok; ++s)
+    ok = cudaEventCreateWithFlags(&in_ready[s], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&computed[s], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&out_free[s], cudaEventDisableTiming) == cudaSuccess;
+  // the copies start after whatever the caller queued on `stream` before this call
+  cudaEvent_t start = nullptr;
+  if (ok) ok = cudaEventCreateWithFlags(&start, cudaEventDisableTiming) == cudaSuccess &&
+               cudaEventRecord(start, stream) == cudaSuccess &&
+               cudaStreamWaitEvent(h2d, start, 0) == cudaSuccess;
+  if (start) cudaEventDestroy(start);
+  if (!ok) { cleanup(); return SAGESLA_ERR_CUDA; }
+
+  for (int64_t c = 0; c < hp.nchunks && ok; ++c) {
+    const int s = static_cast<int>(c & 1);
+    const int64_t h0 = c * hp.hc, hn = (h0 + hp.hc <= BH) ? hp.hc : BH - h0;
+    char* slot = base + hp.fw + s * hp.slot_bytes;
+    char* dq = slot;
+    char* dk = dq + hp.in_bytes;
+    char* dv = dk + hp.in_bytes;
+    char* dout = dv + hp.in_bytes;
+    const size_t in_b = static_cast<size_t>(hn) * head_elems * 2;
+    const size_t off = static_cast<size_t>(h0) * head_elems;
+    // inputs of chunk c into slot s once the forward of chunk c - 2 has read that slot
+    if (c >= 2) ok = cudaStreamWaitEvent(h2d, computed[s], 0) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dq, q_host + off, in_b, cudaMemcpyHostToDevice, h2d) == cudaSuccess &&
+         cudaMemcpyAsync(dk, k_host + off, in_b, cudaMemcpyHostToDevice, h2d) == cudaSuccess &&
+         cudaMemcpyAsync(dv, v_host + off, in_b, cudaMemcpyHostToDevice, h2d) == cudaSuccess &&
+         cudaEventRecord(in_ready[s], h2d) == cudaSuccess;
+    // the forward of chunk c once its inputs are in and the output slot has been copied out
+    ok = ok && cudaStreamWaitEvent(stream, in_ready[s], 0) == cudaSuccess;
+    if (ok && c >= 2) ok = cudaStreamWaitEvent(stream, out_free[s], 0) == cudaSuccess;
+    if (!ok) break;
+    sagesla_tensor tq, tk, tv, to;
+    for (sagesla_tensor* t : {&tq, &tk, &tv, &to}) {
+      t->B = 1; t->H = hn; t->N = N; t->D = D;
+      t->stride_n = D; t->stride_h = N * D; t->stride_b = hn * N * D;
+    }
+    tq.data = dq; tk.data = dk; tv.data = dv; to.data = dout;
+    tq.dtype = tk.dtype = tv.dtype = SAGESLA_BF16;
+    to.dtype = out_dtype;
+    st = sagesla_forward(&tq, &tk, &tv, topk_ratio, block, &to, base, hp.fw, stream_ptr);
+    if (st != SAGESLA_OK) { cleanup(); return st; }
+    // keep this chunk's device status word (the next forward clears the workspace's)
+    ok = cudaMemcpyAsync(base + hp.status_off + 4 * c, base, 4, cudaMemcpyDeviceToDevice, stream) ==
+             cudaSuccess &&
+         cudaEventRecord(computed[s], stream) == cudaSuccess &&
+         cudaStreamWaitEvent(d2h, computed[s], 0) == cudaSuccess &&
+         cudaMemcpyAsync(static_cast<char*>(out_host) + off * out_esz, dout,
+                         static_cast<size_t>(hn) * head_elems * out_esz, cudaMemcpyDeviceToHost,
+                         d2h) == cudaSuccess &&
+         cudaEventRecord(out_free[s], d2h) == cudaSuccess;
+  }
+  // `stream` ends after the last output copy, as a single-stream call would
+  for (int s = 0; s < 2 && ok; ++s) ok = cudaStreamWaitEvent(stream, out_free[s], 0) == cudaSuccess;
+  const bool synced = cudaStreamSynchronize(stream) == cudaSuccess;
+  cleanup();
+  if (!ok || !synced) return SAGESLA_ERR_CUDA;
+  // the first device-side error of any chunk
+  int32_t words[kHostChunks] = {};
+  if (cudaMemcpy(words, base + hp.status_off, static_cast<size_t>(hp.nchunks) * 4,
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
     return SAGESLA_ERR_CUDA;
-  return sagesla_stream_status(stream_ptr, base);
+  for (int64_t c = 0; c < hp.nchunks; ++c)
+    if (words[c] != 0) return static_cast<sagesla_status>(words[c]);
+  return SAGESLA_OK;
 }
 
 }  // extern "C"

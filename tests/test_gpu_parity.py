@@ -87,6 +87,18 @@ def test_host_entry_point_matches_device_entry_point():
     assert torch.equal(out, dev)
 
 
+@pytest.mark.parametrize("B,H,out_dtype", [(1, 11, torch.float32), (2, 5, torch.bfloat16)])
+def test_host_entry_point_chunks_heads(B, H, out_dtype):
+    """The host entry point pipelines copies and forwards over chunks of heads (the last
+    chunk may be short); its output equals the device entry point's."""
+    q, k, v = inputs.make_random(B, H, 700, 33 + H, k_offset_std=0.5)
+    dev = gpu_run(q, k, v, 0.2, out_dtype=out_dtype, extras=False)["out"]
+    out = torch.empty(q.shape, dtype=out_dtype).pin_memory()
+    sba.sagesla_forward_host(q.contiguous().pin_memory(), k.contiguous().pin_memory(),
+                             v.contiguous().pin_memory(), out, 0.2)
+    assert torch.equal(out.float(), dev)
+
+
 def test_repeatable():
     q, k, v = inputs.make_random(1, 2, 2048, 25)
     a = gpu_run(q, k, v, 0.1, extras=False)["out"]

@@ -66,6 +66,23 @@ def parse_args():
     return args
 
 
+def rank_env():
+    """(rank, local rank, world size) from the torchrun environment (1 process if absent)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The maximum of a per-rank time over all ranks (every rank gets it). The tensor lives on
+    `device`: the GPU for NCCL, the CPU for gloo."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def kernel_launches(dense: bool) -> int:
     """Kernels of one forward: stats, finalize, quant, scores, top-k, complement GEMM and
     attention; with every block kept only stats, finalize, quant and attention run."""
@@ -194,8 +211,8 @@ def blas_threads():
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    rank, _, _ = rank_env()
+    if rank != 0:          # under torchrun, rank 0 alone times the oracle
         return 0
     from sparse_bit_attention_b200 import inputs
     w, cfg = workload_config()
@@ -245,11 +262,7 @@ def run_e2e(args, sba, torch, dist, q_cpu, k_cpu, v_cpu, ws, dev, stream, barrie
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dist, dev)
     h2d = 3 * B * H * N * D * 2
     d2h = B * H * N * D * 4
 
@@ -264,9 +277,7 @@ def run_cuda(args):
     from sparse_bit_attention_b200 import binding, inputs
     from sparse_bit_attention_b200.build import build
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, local, world = rank_env()
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     torch.cuda.set_device(local)
@@ -314,10 +325,7 @@ def run_cuda(args):
     ms_total = t_begin.elapsed_time(t_end)
     stage_ms = {name: statistics.mean(ev[i].elapsed_time(ev[i + 1]) for ev in stage_ev)
                 for i, name in enumerate(binding.STAGE_NAMES)}
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dist, dev)
     ms_step = ms_total / args.steps
     value = B * N * world / (ms_step / 1e3)
 

@@ -59,6 +59,8 @@ def parse_args():
                     help="Top-K ratio (default: 0.1; 1.0 is the dense SageAttention mode)")
     ap.add_argument("--sweep", action="store_true",
                     help="Top-K ratio sweep and dense BF16 comparison, one JSON line per point")
+    ap.add_argument("--kernel-case", choices=["norm", "w8a8"], default=None,
+                    help="run a small case of one next-row kernel a few times (for ncu captures)")
     args = ap.parse_args()
     globals()["WORKLOAD"] = args.workload
     if args.topk_ratio is not None:
@@ -533,8 +535,41 @@ def run_sweep(args):
     return 0
 
 
+def run_kernel_case(args):
+    """A few calls of one next-row kernel on a case sized for ncu captures (well above the
+    126 MB L2, a few hundred MB on the device)."""
+    import torch
+    import sparse_bit_attention_b200 as sba
+    from sparse_bit_attention_b200.build import build
+    build()
+    sba.load_library()
+    g = torch.Generator().manual_seed(5)
+    if args.kernel_case == "norm":
+        M, K = 24000, 5120
+        x = (torch.randn(M, K, generator=g) * 1.5).to(torch.bfloat16).cuda()
+        scale = (torch.randn(1, K, generator=g) * 0.2).to(torch.bfloat16).cuda()
+        shift = (torch.randn(1, K, generator=g) * 0.5).to(torch.bfloat16).cuda()
+        for _ in range(3):
+            sba.sagesla_norm_quant(x, sba.SAGESLA_LAYER_NORM, 1e-6, None, None, scale, shift,
+                                   rows_per_sample=M, want_codes=True)
+    else:
+        M, K, N = 16384, 5120, 5120
+        x = (torch.randn(M, K, generator=g) * 1.5).to(torch.bfloat16).cuda()
+        w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).cuda()
+        _, x8, s_x = sba.sagesla_norm_quant(x, sba.SAGESLA_NO_NORM, 0.0, want_y=False,
+                                            want_codes=True)
+        w8, s_w = sba.sagesla_w8a8_quantize_weight(w)
+        for _ in range(3):
+            sba.sagesla_w8a8_gemm(x8, s_x, w8, s_w)
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel_case": args.kernel_case, "ok": True}))
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.kernel_case:
+        return run_kernel_case(args)
     if args.sweep:
         return run_sweep(args)
     if args.warmup < 3:

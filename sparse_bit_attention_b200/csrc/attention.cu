@@ -17,7 +17,9 @@
 // pair of kept blocks [128,256); the linear branch reuses the S columns at the end).
 //   warps 0-3 / 4-7  softmax, correction and epilogue of half 0 / half 1 (16 rows per warp,
 //                    two threads per row through the 16x64b TMEM fragment)
-//   warp 8           TMA producer: Q rows, K8 tiles of pairs of kept blocks, V8 ring, G_i
+//   warp 8           TMA producer: Q rows, K8 tiles of pairs of kept blocks, V8 ring, G_i;
+//                    the kept lists are staged in shared memory when the CTA starts, so no
+//                    tile load waits for a global read of its block index
 //   warp 9           S = Q K^T issuer for both halves: one M=64 N=128 MMA group (4 K-steps)
 //                    per pair of kept blocks, whose K8 tiles sit side by side in shared memory
 //   warps 10 / 11    P.V issuer of half 0 / half 1
@@ -83,12 +85,28 @@ struct HalfCtl {
   uint64_t q_full, g_full, a_full, l_done, mma_done;
 };
 
+// Entries of each half's kept list staged in shared memory (block indices < 2^15 fit 16 bits);
+// entries past this come from global memory.
+constexpr int kListCap = 768;
+
 struct Ctl {
   HalfCtl hc[2];
   uint32_t tmem_base;
   volatile int abort;
   float s_v[128];
+  uint16_t klist[2][kListCap];
 };
+
+// Two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA, and 1 KB of
+// alignment slack in each CTA's request.
+static_assert(2 * (1024 + kOffCtl + sizeof(Ctl) + 1024) <= 228 * 1024, "two CTAs fit on an SM");
+
+// n-th kept key block of half h's query block: its kept list (shared-memory copy first), or
+// block n itself when every block is kept (no list).
+__device__ __forceinline__ int kept_at(const Ctl* ctl, int h, const int32_t* klist, int n) {
+  if (!klist) return n;
+  return n < kListCap ? static_cast<int>(ctl->klist[h][n]) : __ldg(klist + n);
+}
 
 // n-th kept key block of a query block: its kept list, or block n itself when every block is
 // kept (no list).
@@ -250,6 +268,15 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     fence_mbar_init();
   } else if (threadIdx.x == 96) {
     prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_g);
+  } else if (warp >= 4 && warp < 8 && prm.kept) {
+    // both halves' kept lists into shared memory
+    for (int h = 0; h < 2; ++h) {
+      if (U[h] == 0) continue;
+      const int32_t* kl = prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k);
+      const int n = min(U[h], kListCap);
+      for (int e = threadIdx.x - 128; e < n; e += 128)
+        ctl->klist[h][e] = static_cast<uint16_t>(__ldg(kl + e));
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -280,8 +307,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           const int two = n0 + 1 < U[h] ? 2 : 1;
           mbar_arrive_expect_tx(&c.k_full, two * kKVBytes);
           uint8_t* kst = smem + h * kHalfBytes + kHK;
-          tma_load_2d(kst, &tm_k, &c.k_full, 0, row_base + 64 * kept_block(klist, n0));
-          if (two == 2) tma_load_2d(kst + kKVBytes, &tm_k, &c.k_full, 0, row_base + 64 * kept_block(klist, n0 + 1));
+          tma_load_2d(kst, &tm_k, &c.k_full, 0, row_base + 64 * kept_at(ctl, h, klist, n0));
+          if (two == 2) tma_load_2d(kst + kKVBytes, &tm_k, &c.k_full, 0, row_base + 64 * kept_at(ctl, h, klist, n0 + 1));
         }
         // V8 of blocks n0 and n0 + 1: stage n % kNV is free once P.V(n - kNV) is done
         for (int n = n0; n < n0 + 2 && ok; ++n)
@@ -293,7 +320,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) : nullptr;
             mbar_arrive_expect_tx(&c.v_full[s], kKVBytes);
             tma_load_2d(smem + h * kHalfBytes + kHV + s * kKVBytes, &tm_v, &c.v_full[s], 0,
-                        row_base + 64 * kept_block(klist, n));
+                        row_base + 64 * kept_at(ctl, h, klist, n));
           }
       }
       // G_i once the half's loop MMAs are done (its tile overlaps the K and V stages)
@@ -411,15 +438,19 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       const float cs = prm.sq[bh * prm.nbq + qblock] * (kLog2e * kInvSqrtD);
       const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + qblock) * static_cast<int64_t>(prm.k) : nullptr;
       const float* skh = prm.sk + bh * prm.nbq;
-      int j_next = kept_block(klist, 0);
-      float sk_next = __ldg(skh + j_next);
+      // kept indices are read two blocks ahead and scales one block ahead, so that no load
+      // of the loop waits for another one
+      int j_cur = kept_block(klist, 0);
+      int j_ahead = Uh > 1 ? kept_block(klist, 1) : 0;
+      float sk_next = __ldg(skh + j_cur);
       for (int n = 0; n < Uh; ++n) {
         const int b = n & 1;
-        const int j = j_next;
+        const int j = j_cur;
         const float skj = sk_next;
-        if (n + 1 < Uh) {                        // prefetch the next kept block's scale
-          j_next = kept_block(klist, n + 1);
-          sk_next = __ldg(skh + j_next);
+        if (n + 1 < Uh) {
+          sk_next = __ldg(skh + j_ahead);
+          j_cur = j_ahead;
+          if (n + 2 < Uh) j_ahead = kept_block(klist, n + 2);
         }
         if (b == 0 && !wait_or_abort(&c.s_full, (n >> 1) & 1, ctl, status)) { ok = false; break; }
         tc_fence_after();

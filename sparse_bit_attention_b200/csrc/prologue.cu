@@ -54,27 +54,41 @@ __device__ __forceinline__ float double_to_bf16_rne(double x) {
   return static_cast<float>(__longlong_as_double(static_cast<long long>(b)));
 }
 
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 fills the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
 constexpr int kStatsThreads = 128;
-// 48 KB of operands and reductions + alignment slack; this size also keeps at most four
-// CTAs on an SM, so four 128-column TMEM allocations always fit in the 512 columns.
-constexpr int kStatsSmem = 52 * 1024;
+// Two 16 KB operand tiles + alignment slack. Four CTAs per SM, each holding 128 TMEM columns
+// from its start (measured on B200: allocating TMEM only around the MMA, to let six CTAs
+// share an SM, made the kernel almost twice as slow).
+constexpr int kStatsSmem = 33 * 1024;
 
 // kLinear = false (every key block kept, no linear branch): only the K sums, V amax and
 // pooled K are needed, so phi, H_j and its MMA are skipped.
+//
+// Thread t serves the 8-channel chunk ch = t & 15 of rows g, g+8, ..., g+56 (g = t >> 4); the
+// 16 chunks of a row sit in 16 lanes of one warp. K and V arrive by cp.async directly in the
+// layout the MMA reads (128-byte-swizzled, MN-major: row r, chunk ch at
+// (ch / 8) * 8 KB + sw128(r, ch % 8)), so each thread turns its own K chunks into phi in place.
 template <bool kLinear>
-__global__ void __launch_bounds__(kStatsThreads)
+__global__ void __launch_bounds__(kStatsThreads, 4)
 k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restrict__ ksum_part,
         float* __restrict__ vmax_part, float* __restrict__ kbar, __nv_bfloat16* __restrict__ hflat,
         int* status) {
   extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_slot;
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* a_tile = smem;               // phi(K_j) as [token][channel], 2 x 8 KB, MN-major
-  uint8_t* b_tile = smem + 16384;       // V_j as [token][column], 2 x 8 KB, MN-major
-  double* red_k = reinterpret_cast<double*>(smem + 32768);        // [8][128]
-  float* red_v = reinterpret_cast<float*>(smem + 32768 + 8192);   // [8][128]
+  uint8_t* a_tile = smem;               // K_j, then phi(K_j) as [token][channel], 2 x 8 KB
+  uint8_t* b_tile = smem + 16384;       // V_j as [token][column], 2 x 8 KB
+  // per-row-group partial sums, in the operand tiles once the MMA has read them
+  double* red_k = reinterpret_cast<double*>(smem);                // [8][128]
+  float* red_v = reinterpret_cast<float*>(smem + 8192);           // [8][128]
   float* red_p = red_v + 8 * 128;                                 // [8][128]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(red_p + 8 * 128);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
 
   const int j = blockIdx.x;
   const int64_t bh = blockIdx.y;
@@ -88,15 +102,6 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
     return;
   }
 
-  if (kLinear && warp == 0) {
-    tmem_alloc(tmem_slot, 128);
-    tmem_relinquish();
-  }
-  if (kLinear && t == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-  }
-
   const int64_t b = bh / K.H, h = bh % K.H;
   const uint16_t* kb = static_cast<const uint16_t*>(K.data) + b * K.stride_b + h * K.stride_h;
   const uint16_t* vb = static_cast<const uint16_t*>(V.data) + b * V.stride_b + h * V.stride_h;
@@ -105,31 +110,41 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
   const int ch = t & 15;   // 8-channel chunk
   const int g = t >> 4;    // row group: rows g, g+8, ..., g+56
 
+  if (kLinear && warp == 0) {
+    tmem_alloc(&tmem_slot, 128);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  // all of this thread's K and V chunks in flight at once (rows past the end read as zeros)
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int r = g + 8 * s;
+    const bool in = r < nj;
+    const int64_t row = n0 + (in ? r : 0);
+    const uint32_t off = (ch >> 3) * 8192u + sw128_offset(r, ch & 7);
+    cp_async16(a_tile + off, kb + row * K.stride_n + 8 * ch, in ? 16u : 0u);
+    cp_async16(b_tile + off, vb + row * V.stride_n + 8 * ch, in ? 16u : 0u);
+  }
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  if (kLinear && t == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
   double ksum[8];
   float vmax[8], psum[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) { ksum[e] = 0.0; vmax[e] = 0.f; psum[e] = 0.f; }
 
-  // all of this thread's K and V chunks in flight at once (8 + 8 x 16 bytes)
-  uint4 kreg[8], vreg[8];
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int r = g + 8 * s;
-    kreg[s] = make_uint4(0, 0, 0, 0);
-    vreg[s] = make_uint4(0, 0, 0, 0);
-    if (r < nj) {
-      kreg[s] = ld_row_chunk(kb, (n0 + r) * K.stride_n + 8 * ch);
-      vreg[s] = ld_row_chunk(vb, (n0 + r) * V.stride_n + 8 * ch);
-    }
-  }
-#pragma unroll
+#pragma unroll 2
   for (int s = 0; s < 8; ++s) {
     const int r = g + 8 * s;
     const bool valid = r < nj;
-    const uint4 kraw = kreg[s], vraw = vreg[s];
+    const uint32_t off = (ch >> 3) * 8192u + sw128_offset(r, ch & 7);
     float kf[8], vf[8];
-    unpack_bf16x8(kraw, kf);
-    unpack_bf16x8(vraw, vf);
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(a_tile + off), kf);
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(b_tile + off), vf);
     float mx = -INFINITY;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -137,28 +152,52 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
       vmax[e] = fmaxf(vmax[e], fabsf(vf[e]));
       mx = fmaxf(mx, kf[e]);
     }
-    if (!kLinear) continue;
-    // phi = softmax over the 128 channels of this token; the row lives in 16 lanes.
+    if constexpr (kLinear) {
+      // phi = softmax over the 128 channels of this token; the row lives in 16 lanes.
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float ex[8], sum = 0.f;
+      for (int o = 8; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float ex[8], sum = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) { ex[e] = __expf(kf[e] - mx); sum += ex[e]; }
+      for (int e = 0; e < 8; ++e) { ex[e] = __expf(kf[e] - mx); sum += ex[e]; }
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float inv = 1.0f / sum;
-    uint32_t packed[4];
+      for (int o = 8; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const float inv = 1.0f / sum;
+      uint32_t packed[4];
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      __nv_bfloat162 p2 = __floats2bfloat162_rn(valid ? ex[e] * inv : 0.f,
-                                                valid ? ex[e + 1] * inv : 0.f);
-      packed[e / 2] = *reinterpret_cast<uint32_t*>(&p2);
-      psum[e] += __low2float(p2);
-      psum[e + 1] += __high2float(p2);
+      for (int e = 0; e < 8; e += 2) {
+        __nv_bfloat162 p2 = __floats2bfloat162_rn(valid ? ex[e] * inv : 0.f,
+                                                  valid ? ex[e + 1] * inv : 0.f);
+        packed[e / 2] = *reinterpret_cast<uint32_t*>(&p2);
+        psum[e] += __low2float(p2);
+        psum[e + 1] += __high2float(p2);
+      }
+      *reinterpret_cast<uint4*>(a_tile + off) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
-    const uint32_t off = (ch >> 3) * 8192u + sw128_offset(r, ch & 7);
-    *reinterpret_cast<uint4*>(a_tile + off) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    *reinterpret_cast<uint4*>(b_tile + off) = vraw;
+  }
+
+  uint32_t tmem = 0;
+  bool ok = true;
+  if (kLinear) {
+    fence_proxy_async_smem();
+    __syncthreads();                     // phi and V complete; the barrier is initialized
+    if (warp == 0) {
+      tc_fence_after();
+      if (lane == 0) {
+        constexpr uint32_t idesc = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 1, 1, 128, 128);
+        const uint32_t d = tmem_slot;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {   // 4 x K=16 tokens
+          const uint64_t ad = make_sdesc(smem_u32(a_tile) + kk * 2048, 8192, 1024, kLayoutSW128);
+          const uint64_t bd = make_sdesc(smem_u32(b_tile) + kk * 2048, 8192, 1024, kLayoutSW128);
+          mma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar);
+      }
+    }
+    // the operand tiles are free for the reductions once the MMA has read them
+    ok = mbar_wait(&bar, 0, status);
+  } else {
+    __syncthreads();                     // every thread is done with the tiles
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -166,22 +205,11 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
     red_v[g * 128 + 8 * ch + e] = vmax[e];
     red_p[g * 128 + 8 * ch + e] = psum[e];
   }
-  fence_proxy_async_smem();
   __syncthreads();
-
-  const uint32_t tmem = kLinear ? *tmem_slot : 0u;
-  if (kLinear && t == 0) {
+  if (kLinear) {                         // the TMEM address written by warp 0's allocation
     tc_fence_after();
-    constexpr uint32_t idesc = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 1, 1, 128, 128);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {   // 4 x K=16 tokens
-      const uint64_t ad = make_sdesc(smem_u32(a_tile) + kk * 2048, 8192, 1024, kLayoutSW128);
-      const uint64_t bd = make_sdesc(smem_u32(b_tile) + kk * 2048, 8192, 1024, kLayoutSW128);
-      mma_bf16(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
-    }
-    mma_commit(bar);
+    tmem = tmem_slot;
   }
-
   {  // per-channel reductions (thread t = channel t), fixed order over row groups
     const int c = t;
     double ks = 0.0;
@@ -199,11 +227,8 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
   }
   if (!kLinear) return;
 
-  const bool ok = mbar_wait(bar, 0, status);
-  tc_fence_after();
-  // H_j[c][n] (TMEM lane c, column n) -> bf16 tile [n][c] in the freed operand tiles, then
-  // 16-byte stores of the contiguous 32 KB of the row.
-  uint16_t* stage = reinterpret_cast<uint16_t*>(smem);
+  // H_j[c][n] (TMEM lane c, column n) -> hrow[n][c]: each warp stores 32 consecutive channels
+  // (64 contiguous bytes) of one value column per store.
   if (ok) {
     const int c = 32 * warp + lane;
 #pragma unroll 1
@@ -211,19 +236,14 @@ k_stats(TensorArg K, TensorArg V, int N, int nb, int nb_k_pad, double* __restric
       uint32_t r[32];
       tmem_ld32(tmem_addr(tmem, 32 * warp, 32 * cc), r);
       tmem_ld_wait();
+      uint16_t* dst = reinterpret_cast<uint16_t*>(hrow) + (32 * cc) * 128 + c;
 #pragma unroll
       for (int e = 0; e < 32; ++e)
-        stage[(32 * cc + e) * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[e])));
+        dst[e * 128] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[e])));
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (ok) {
-    const uint4* src = reinterpret_cast<const uint4*>(stage);
-    uint4* dst = reinterpret_cast<uint4*>(hrow);
-#pragma unroll 4
-    for (int e = t; e < 128 * 128 / 8; e += kStatsThreads) dst[e] = src[e];
-  }
   if (warp == 0) tmem_dealloc(tmem, 128);
 }
 

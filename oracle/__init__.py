@@ -6,3 +6,4 @@ import this package. The product path never does.
 from .sagesla_oracle import *  # noqa: F401,F403
 from . import norm_oracle  # noqa: F401,E402
 from . import w8a8_oracle  # noqa: F401,E402
+from . import sla_backward_oracle  # noqa: F401,E402

@@ -118,6 +118,11 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The float whose key is k (inverse of order_key on keys of finite floats).
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 constexpr int kTopkThreads = 256;
 
 // Block-wide exclusive prefix sum of one int per thread (256 threads); returns the total.
@@ -247,11 +252,19 @@ k_topk_warp(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __
     const int j = 32 * m + lane;
     key[m] = j < nb ? order_key(__ldg(srow + j)) : 0u;   // 0 is below every real key
   }
-  // Invariants: count(key >= lo) = cnt_lo >= k, count(key > hi) = cnt_above < k.
-  uint32_t lo = 0u, hi = 0xFFFFFFFFu;
-  int cnt_lo = 32 * M, cnt_above = 0;
+  // Invariants: count(key >= lo) = cnt_lo >= k, count(key > hi) = cnt_above < k. The bracket
+  // starts at the row's smallest and largest keys and is split at the midpoint of the two
+  // scores (about half the splits of halving the key range, for score rows of ordinary
+  // spread), or of the keys where the scores' midpoint does not split it.
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+    if (32 * m + lane < nb) { kmin = min(kmin, key[m]); kmax = max(kmax, key[m]); }
+  uint32_t lo = __reduce_min_sync(0xffffffffu, kmin), hi = __reduce_max_sync(0xffffffffu, kmax);
+  int cnt_lo = nb, cnt_above = 0;
   while (lo < hi && cnt_lo - cnt_above > 32) {
-    const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
+    uint32_t mid = order_key(0.5f * key_value(lo) + 0.5f * key_value(hi));
+    if (mid <= lo || mid > hi) mid = lo + ((hi - lo) >> 1) + 1u;
     int c = 0;
 #pragma unroll
     for (int m = 0; m < M; ++m) c += key[m] >= mid ? 1 : 0;

@@ -264,6 +264,40 @@ sagesla_status sagesla_w8a8_gemm(const int8_t* x8, const float* x_scale, int64_t
                                  const uint16_t* bias, void* y, int32_t y_dtype,
                                  int64_t y_stride, int32_t* status, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * SLA backward: gradients of the unquantized sparse-linear attention for fine-tuning.
+ * News.qq.com TurboDiffusion article, section 从训练到部署 (full attention is replaced by SLA
+ * and fine-tuned; SageSLA, SLA plus low-bit quantization, replaces it only at inference).
+ * Forward differentiated: O = O_s + O_l with O_s the exact softmax attention of each query
+ * block over the tokens of its kept key blocks (scale 1/sqrt(128), padded keys excluded) and
+ * O_l the normalized linear attention phi(q) G_i[:, :128] / phi(q) G_i[:, 128] over the key
+ * blocks it does not keep (G_i = sum of H_j = phi(K_j)^T [V_j | 1], phi = softmax over the
+ * 128 channels). The block selection is the forward's (same pooled scores and Top-K ratio)
+ * and is held fixed: the gradients are those of O with the mask constant. */
+
+/* Bytes of device workspace sagesla_sla_backward needs (the forward's layout of
+ * sagesla_get_workspace_layout, followed by the backward's own regions); 0 for invalid
+ * arguments. */
+size_t sagesla_sla_backward_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
+                                           double topk_ratio, int block);
+
+/* dq, dk, dv = gradients of sum(O * d_out) with respect to q, k, v.
+ *   q, k, v, d_out  bf16 views [B, H, N, 128] (the requirements of sagesla_forward)
+ *   dq, dk, dv      bf16 or f32 views of the same shape, one dtype for all three; written
+ *                   in full (f32 results of fp32 accumulation, rounded to nearest even for
+ *                   bf16); they must not overlap the inputs, each other or the workspace
+ *   workspace       device, 256-byte aligned, sagesla_sla_backward_workspace_size bytes; it
+ *                   holds the forward's selection (kept lists, mask) at the forward layout's
+ *                   offsets afterwards
+ * Asynchronous on `stream`; device-side timeouts land in the workspace's status word
+ * (sagesla_stream_status). Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, NO_DEVICE
+ * (nothing launched on any error found before the launches). */
+sagesla_status sagesla_sla_backward(const sagesla_tensor* q, const sagesla_tensor* k,
+                                    const sagesla_tensor* v, const sagesla_tensor* d_out,
+                                    double topk_ratio, int block, sagesla_tensor* dq,
+                                    sagesla_tensor* dk, sagesla_tensor* dv, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device status word of `workspace`
  * (the one used by the last forward on that workspace). Returns SAGESLA_OK, TIMEOUT,
  * DEVICE_CHECK, or CUDA if the stream reported an error. */

@@ -6,4 +6,5 @@ from .binding import (  # noqa: F401
     sagesla_host_workspace_size, sagesla_status_string, sagesla_stream_status,
     sagesla_topk_count, sagesla_workspace_size, SAGESLA_LAYER_NORM, SAGESLA_RMS_NORM,
     sagesla_norm_quant, SAGESLA_NO_NORM, sagesla_w8a8_quantize_weight, sagesla_w8a8_gemm,
+    sagesla_sla_backward, sagesla_sla_backward_workspace_size,
 )

@@ -101,6 +101,11 @@ _SIGNATURES = {
     "sagesla_w8a8_quantize_weight": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                                     ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
                                                     ctypes.c_void_p]),
+    "sagesla_sla_backward_workspace_size": (ctypes.c_size_t, [ctypes.c_int64] * 4 + [
+        ctypes.c_double, ctypes.c_int]),
+    "sagesla_sla_backward": (ctypes.c_int, [ctypes.POINTER(SageslaTensor)] * 4 + [
+        ctypes.c_double, ctypes.c_int] + [ctypes.POINTER(SageslaTensor)] * 3 + [
+        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "sagesla_w8a8_gemm": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                          ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
@@ -251,6 +256,35 @@ def sagesla_forward_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: tor
         ctypes.c_void_p(out_host.data_ptr()), odt, ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel(), ctypes.c_void_p(_stream_ptr(stream))), "sagesla_forward_host")
     return out_host
+
+
+def sagesla_sla_backward_workspace_size(B: int, H: int, N: int, D: int = HEAD_DIM,
+                                        topk_ratio: float = 0.1, block: int = BLOCK) -> int:
+    return int(load_library().sagesla_sla_backward_workspace_size(B, H, N, D, float(topk_ratio),
+                                                                  block))
+
+
+def sagesla_sla_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, d_out: torch.Tensor,
+                         topk_ratio: float = 0.1, block: int = BLOCK, dq=None, dk=None, dv=None,
+                         grad_dtype: torch.dtype = torch.float32,
+                         workspace: torch.Tensor | None = None, stream=None):
+    """Gradients (dq, dk, dv) of sum(O * d_out) for the unquantized SLA forward (the block
+    selection held fixed); q, k, v, d_out bf16 [B, H, N, 128] on the device."""
+    lib = load_library()
+    B, H, N, D = q.shape
+    dq = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=dq.dtype, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=dq.dtype, device=q.device) if dv is None else dv
+    need = sagesla_sla_backward_workspace_size(B, H, N, D, topk_ratio, block)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    views = [_view(x) for x in (q, k, v, d_out, dq, dk, dv)]
+    _check(lib.sagesla_sla_backward(
+        *[ctypes.byref(x) for x in views[:4]], float(topk_ratio), int(block),
+        *[ctypes.byref(x) for x in views[4:]], ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_ptr(stream))),
+        "sagesla_sla_backward")
+    return dq, dk, dv
 
 
 def sagesla_stream_status(stream=None, workspace: torch.Tensor | None = None) -> int:

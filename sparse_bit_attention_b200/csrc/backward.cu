@@ -1,0 +1,1139 @@
+// SLA backward: gradients of the unquantized sparse-linear attention with the block
+// selection of the forward held fixed.
+//
+// Method: news.qq.com TurboDiffusion article, section 从训练到部署 — the full attention layers
+// are replaced by SLA and fine-tuned, and only at inference is SLA swapped for SageSLA (SLA
+// plus low-bit quantization); the sparse and linear branches follow the "Sparse-Linear
+// Attention" method named in the dgmzs.com.cn README translation, section 方法论. With
+// s = q.k/sqrt(128), for a query token t of block i and the tokens u of its kept blocks:
+//     L_t = log sum_u e^{s_tu},  P = e^{s - L},  O_s = P V,  D_t = dO_t . O_s,t,
+//     dS = P (dO V^T - D),  dQ = dS K / sqrt(128),  dK = dS^T Q / sqrt(128),  dV = P^T dO;
+// and for the linear branch (a = phi(q), G_i the sum of the key-block states H_j over the
+// blocks i does not keep, num = a G_i[:, :128], den = a G_i[:, 128], O_l = num / den):
+//     dnum = dO / den,  dden = -(dO . O_l) / den,  da = G_i[:, :128] dnum + G_i[:, 128] dden,
+//     dq += a * da (the softmax Jacobian's projection a . da vanishes: O_l is unchanged when a
+//     is scaled),  dG_i = a^T [dnum | dden],  dH_j = sum of dG_i over the blocks not keeping j,
+//     db = dH_j[:, :128] v + dH_j[:, 128],  dk += b * (db - b . db),  dv += dH_j[:, :128]^T b,
+//     with b = phi(k).
+//
+// B200 mapping. The forward's prologue supplies the kept lists, the complement mask and G_i.
+// Q, K, V and dO are packed into zero-padded [head][row][128] bf16 copies; every 64-row tile is
+// loaded by TMA in the key-interleaved order (row 2i + h of the tile holds token 32h + i) that
+// makes the 16x64b TMEM fragment of an M=64 result hold 32 consecutive tokens per thread, so
+// the P and dS operands written back by the threads are 64 contiguous bytes after one pair
+// exchange. The sparse branch runs on tcgen05 BF16 MMAs (fp32 accumulators in TMEM):
+//   k_bwd_lse     per query block: the sparse forward again (online softmax), giving the
+//                 base-2 log-sum-exp L and D = rowsum(dO * O_s)
+//   k_bwd_dq      per query block over its kept blocks: S, dP, dS, dQ; adds the linear dq
+//   k_bwd_dkv     per key block over the query blocks that keep it: S^T, dP^T, dV, dK; adds
+//                 the linear dk, dv
+// The linear branch runs on the CUDA cores (k_bwd_lin_query, k_bwd_lin_key) around one
+// complement GEMM on the tensor cores (dH = (1 - M)^T dG, the forward's GEMM on the
+// transposed mask).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sagesla {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kScale = 0.08838834764831845f;   // 1 / sqrt(128)
+constexpr uint32_t kTile = 64 * 128 * 2;         // one 64-row bf16 tile (two 8 KB d-chunks)
+constexpr uint32_t kPTile = 64 * 64 * 2;         // a 64 x 64 bf16 operand (one 128-byte atom)
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Token of position p of a key-interleaved 64-row tile.
+__device__ __forceinline__ int tile_token(int p) { return (p >> 1) + 32 * (p & 1); }
+
+// 16x64b TMEM fragment of an M=64 result: warp w, lane t hold row 16w + t/4 + 8(t&1) and the
+// columns kh + 2e (e = 0..31), kh = (t >> 1) & 1.
+__device__ __forceinline__ int frag_row(int warp, int lane) {
+  return 16 * warp + (lane >> 2) + 8 * (lane & 1);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+// This thread's 32 values (columns kh + 2e of a row, i.e. the tile positions of tokens
+// 32kh + e) as bf16 into a 64 x 64 K-major SW128 operand tile in tile-position order: after
+// an exchange with lane ^ 2 (same row, other kh), the thread holds positions 32kh .. 32kh+31
+// and stores them as four 16-byte chunks.
+__device__ __forceinline__ void store_row_operand(uint8_t* tile, int row, int kh,
+                                                  const float (&x)[32]) {
+  uint32_t send[8], mine[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    // kh = 0 keeps e = 0..15 and sends 16..31; kh = 1 keeps 16..31 and sends 0..15
+    send[u] = kh ? pack_bf16x2(x[2 * u], x[2 * u + 1]) : pack_bf16x2(x[16 + 2 * u], x[17 + 2 * u]);
+    mine[u] = kh ? pack_bf16x2(x[16 + 2 * u], x[17 + 2 * u]) : pack_bf16x2(x[2 * u], x[2 * u + 1]);
+  }
+  uint32_t recv[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) recv[u] = __shfl_xor_sync(0xffffffffu, send[u], 2);
+  // position 2e' + h holds token 32h + e'; the thread covers e' = 16kh .. 16kh + 15. The
+  // kh = 0 thread owns tokens e (h = 0), the kh = 1 thread tokens 32 + e (h = 1).
+  uint32_t w[16];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const uint32_t lo_m = mine[u] & 0xFFFFu, hi_m = mine[u] >> 16;
+    const uint32_t lo_r = recv[u] & 0xFFFFu, hi_r = recv[u] >> 16;
+    // words for e' = 16kh + 2u and 16kh + 2u + 1: (h=0 value, h=1 value)
+    w[2 * u] = kh ? (lo_r | (lo_m << 16)) : (lo_m | (lo_r << 16));
+    w[2 * u + 1] = kh ? (hi_r | (hi_m << 16)) : (hi_m | (hi_r << 16));
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<uint4*>(tile + sw128_offset(row, 4 * kh + c)) =
+        make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+}
+
+// ------------------------------------------------------------------ packing and lists
+
+// Q, K, V, dO rows -> zero-padded [head][n_pad][128] bf16 copies (one thread per 16 bytes).
+__global__ void k_bwd_pack(TensorArg q, TensorArg k, TensorArg v, TensorArg d_out, int N,
+                           int n_pad, int64_t total, uint4* __restrict__ qp, uint4* __restrict__ kp,
+                           uint4* __restrict__ vp, uint4* __restrict__ dp) {
+  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (idx >= total) return;
+  const int chunk = static_cast<int>(idx & 15);
+  const int64_t row = idx >> 4;
+  const int64_t bh = row / n_pad;
+  const int n = static_cast<int>(row - bh * n_pad);
+  uint4 z = make_uint4(0, 0, 0, 0);
+  uint4 a = z, b = z, c = z, d = z;
+  if (n < N) {
+    auto ld = [&](const TensorArg& t) {
+      const int64_t bb = bh / t.H, hh = bh % t.H;
+      const uint16_t* base = static_cast<const uint16_t*>(t.data) + bb * t.stride_b +
+                             hh * t.stride_h + static_cast<int64_t>(n) * t.stride_n;
+      return __ldg(reinterpret_cast<const uint4*>(base) + chunk);
+    };
+    a = ld(q); b = ld(k); c = ld(v); d = ld(d_out);
+  }
+  qp[idx] = a; kp[idx] = b; vp[idx] = c; dp[idx] = d;
+}
+
+// For key block j: the query blocks i whose kept list holds j, ascending (one warp per
+// (head, j), reading the kept bitmask column j).
+__global__ void k_bwd_lists(int nb, int mask_words, int64_t BH, const uint32_t* __restrict__ mask,
+                            int32_t* __restrict__ tcount, int32_t* __restrict__ tlist) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  if (w >= BH * nb) return;
+  const int64_t bh = w / nb;
+  const int j = static_cast<int>(w - bh * nb);
+  const uint32_t* mcol = mask + bh * nb * static_cast<int64_t>(mask_words) + (j >> 5);
+  int32_t* out = tlist + (bh * nb + j) * static_cast<int64_t>(nb);
+  int count = 0;
+  for (int i0 = 0; i0 < nb; i0 += 32) {
+    const int i = i0 + lane;
+    const bool kept = i < nb && ((__ldg(mcol + static_cast<int64_t>(i) * mask_words) >> (j & 31)) & 1u);
+    const uint32_t bits = __ballot_sync(0xffffffffu, kept);
+    if (kept) out[count + __popc(bits & ((1u << lane) - 1u))] = i;
+    count += __popc(bits);
+  }
+  if (lane == 0) tcount[bh * nb + j] = count;
+}
+
+// amask [head][nb_m_pad][nb_k_pad] (1 where the key block is not kept) -> its transpose,
+// [head][nb_m_pad][nb_m_pad] with zero rows past nb_k_pad (the row extent of the complement
+// GEMM is a multiple of 128), by 32 x 32 tiles through shared memory.
+__global__ void k_bwd_transpose_mask(int nb_m_pad, int nb_k_pad, const uint16_t* __restrict__ src,
+                                     uint16_t* __restrict__ dst) {
+  __shared__ uint16_t t[32][33];
+  const int64_t bh = blockIdx.z;
+  const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;   // source row i, source column j
+  const uint16_t* s = src + bh * nb_m_pad * static_cast<int64_t>(nb_k_pad);
+  uint16_t* d = dst + bh * nb_m_pad * static_cast<int64_t>(nb_m_pad);
+  for (int r = threadIdx.y; r < 32; r += blockDim.y)
+    t[r][threadIdx.x] = j0 + threadIdx.x < nb_k_pad
+                            ? s[static_cast<int64_t>(i0 + r) * nb_k_pad + j0 + threadIdx.x]
+                            : static_cast<uint16_t>(0);
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y)
+    d[static_cast<int64_t>(j0 + r) * nb_m_pad + i0 + threadIdx.x] = t[threadIdx.x][r];
+}
+
+// ------------------------------------------------------------------ sparse branch (tcgen05)
+
+// Instruction descriptors: M=64 BF16 MMAs with fp32 accumulation.
+constexpr uint32_t kIdescKK64 = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 64, 64);   // S-like
+constexpr uint32_t kIdescKM128 = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 1, 64, 128); // P.V-like
+
+// K-major operand of 64 rows x 128 (bf16, two 8 KB chunks of 64 columns): K-step kk of 16.
+__device__ __forceinline__ uint64_t desc_k128(uint32_t base, int kk) {
+  return make_sdesc(base + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+}
+// K-major 64 x 64 operand (P, dS; one 128-byte atom per row): K-step kk of 16.
+__device__ __forceinline__ uint64_t desc_k64(uint32_t base, int kk) {
+  return make_sdesc(base + kk * 32, 16, 1024, kLayoutSW128);
+}
+// MN-major operand: 64 rows of K x 128 columns of N (two 8 KB chunks of 64 N): K-step kk.
+__device__ __forceinline__ uint64_t desc_mn128(uint32_t base, int kk) {
+  return make_sdesc(base + kk * 2048, 8192, 1024, kLayoutSW128);
+}
+
+// A 64 x 128 tile of rows [row, row + 64) of a packed buffer, key-interleaved (two 8 KB
+// loads, one per 64-column chunk) through the four-dimensional map of that buffer.
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                          int block_row) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(0), "r"(0),
+      "r"(block_row)
+      : "memory");
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst + 8192)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(64), "r"(0), "r"(0),
+      "r"(block_row)
+      : "memory");
+}
+
+struct BwdParams {
+  const int32_t* kept;     // [BH][nb][k]
+  const int32_t* tcount;   // [BH][nb]
+  const int32_t* tlist;    // [BH][nb][nb]
+  const uint16_t* qn;      // packed bf16 rows [BH][n_pad][128]
+  const uint16_t* dn;      // packed dO
+  float* lse;              // [BH][n_pad], base-2 log-sum-exp of the scaled scores
+  float* dd;               // [BH][n_pad], D = rowsum(dO * O_s)
+  const float* lin_q;      // [BH][n_pad][128] linear-branch dq (null: none)
+  const float* lin_k;
+  const float* lin_v;
+  void* dq; void* dk; void* dv;
+  int64_t dq_sb, dq_sh, dq_sn, dk_sb, dk_sh, dk_sn, dv_sb, dv_sh, dv_sn;
+  int32_t g_dtype;         // SAGESLA_F32 or SAGESLA_BF16 for dq, dk, dv
+  int* status;
+  int N, nb, n_pad, k, n_last, H;
+};
+
+constexpr int kBwdThreads = 128;
+
+// Online-softmax pass of one query block over its kept key blocks (bf16 MMAs): writes the
+// base-2 log-sum-exp L of the scaled scores and D = rowsum(dO * O_s) of its 64 rows.
+// TMEM: S [0, 64) and O [64, 192).
+__global__ void __launch_bounds__(kBwdThreads, 2)
+k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+          const __grid_constant__ CUtensorMap tm_v, BwdParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* q_t = smem;                   // Q tile
+  uint8_t* k_t = smem + kTile;           // 2 K stages
+  uint8_t* v_t = smem + 3 * kTile;       // 2 V stages
+  uint8_t* p_t = smem + 5 * kTile;       // P tile
+  __shared__ uint64_t q_full, k_full[2], v_full[2], s_done, pv_done;
+  __shared__ uint32_t tmem_slot;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int U = prm.k;
+  const int32_t* klist = prm.kept + (bh * prm.nb + i) * static_cast<int64_t>(prm.k);
+  const int blk0 = static_cast<int>(bh * (prm.n_pad / 64));   // first 64-row block of the head
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 256);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < 2; ++s) { mbar_init(&k_full[s], 1); mbar_init(&v_full[s], 1); }
+    mbar_init(&s_done, 1);
+    mbar_init(&pv_done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
+    mbar_arrive_expect_tx(&q_full, kTile);
+    load_tile(q_t, &tm_q, &q_full, blk0 + i);
+    const int j0 = __ldg(klist);
+    mbar_arrive_expect_tx(&k_full[0], kTile);
+    load_tile(k_t, &tm_k, &k_full[0], blk0 + j0);
+    mbar_arrive_expect_tx(&v_full[0], kTile);
+    load_tile(v_t, &tm_v, &v_full[0], blk0 + j0);
+  }
+  const int row = frag_row(warp, lane);
+  const int kh = (lane >> 1) & 1;
+  const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
+  const float c2 = kScale * kLog2e;
+  float m_run = -INFINITY, l_part = 0.f;
+  bool ok = true;
+  int j_next = __ldg(klist);
+  for (int n = 0; n < U && ok; ++n) {
+    const int j = j_next;
+    if (n + 1 < U) j_next = __ldg(klist + n + 1);
+    const int st = n & 1;
+    if (threadIdx.x == 0) {
+      ok = (n > 0 || mbar_wait(&q_full, 0, prm.status)) &&
+           mbar_wait(&k_full[st], (n >> 1) & 1, prm.status);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t qa = smem_u32(q_t), kb = smem_u32(k_t + st * kTile);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem, desc_k128(qa, kk), desc_k128(kb, kk), kIdescKK64, kk > 0 ? 1u : 0u);
+        mma_commit(&s_done);
+      }
+    }
+    if (!mbar_wait(&s_done, n & 1, prm.status)) { ok = false; break; }
+    tc_fence_after();
+    // K of the next kept block into the other stage (its previous K was read by S(n-1))
+    if (threadIdx.x == 0 && n + 1 < U) {
+      mbar_arrive_expect_tx(&k_full[st ^ 1], kTile);
+      load_tile(k_t + (st ^ 1) * kTile, &tm_k, &k_full[st ^ 1], blk0 + j_next);
+    }
+    uint32_t sr[32];
+    tmem_ld16x64(tmem + lane_s, sr);
+    tmem_ld_wait();
+    const int valid = (j == prm.nb - 1) ? prm.n_last - 32 * kh : 32;   // real keys of this thread
+    float x[32], mx = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      x[e] = e < valid ? __uint_as_float(sr[e]) * c2 : -INFINITY;
+      mx = fmaxf(mx, x[e]);
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = exp2f(m_run - m_new);
+    float rs = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) { x[e] = exp2f(x[e] - m_new); rs += x[e]; }
+    l_part = alpha * l_part + rs;
+    m_run = m_new;
+    // P.V(n-1) done: frees the P tile and the V stage of block n+1, and O is stable
+    if (n > 0 && !mbar_wait(&pv_done, (n - 1) & 1, prm.status)) { ok = false; break; }
+    tc_fence_after();
+    if (threadIdx.x == 0 && n + 1 < U) {
+      mbar_arrive_expect_tx(&v_full[st ^ 1], kTile);
+      load_tile(v_t + (st ^ 1) * kTile, &tm_v, &v_full[st ^ 1], blk0 + j_next);
+    }
+    if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t o[32];
+        tmem_ld16x64(tmem + lane_s + 64 + 64 * cc, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        tmem_st16x64(tmem + lane_s + 64 + 64 * cc, o);
+      }
+      tmem_st_wait();
+    }
+    store_row_operand(p_t, row, kh, x);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      if (mbar_wait(&v_full[st], (n >> 1) & 1, prm.status)) {
+        const uint32_t pa = smem_u32(p_t), vb = smem_u32(v_t + st * kTile);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + 64, desc_k64(pa, kk), desc_mn128(vb, kk), kIdescKM128,
+                   (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&pv_done);
+      }
+    }
+  }
+  if (ok) ok = mbar_wait(&pv_done, (U - 1) & 1, prm.status);
+  tc_fence_after();
+  // O_s = O / l; D = dO . O_s over the row (this thread: columns kh + 2e and 64 + kh + 2e)
+  const float l_row = l_part + __shfl_xor_sync(0xffffffffu, l_part, 2);
+  const int tok = tile_token(row);
+  const int64_t grow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + tok;
+  float dsum = 0.f;
+  if (ok) {
+    const uint4* drow = reinterpret_cast<const uint4*>(prm.dn + grow * 128);
+#pragma unroll 1
+    for (int cc = 0; cc < 2; ++cc) {
+      uint32_t o[32];
+      tmem_ld16x64(tmem + lane_s + 64 + 64 * cc, o);
+      tmem_ld_wait();
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint4 w = __ldg(drow + 8 * cc + u);    // columns 64cc + 8u .. +7
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {   // element pair (2e, 2e + 1), e = 4u + z
+          const float dv = bf16_bits_to_f32(kh ? (ww[z] >> 16) : (ww[z] & 0xFFFFu));
+          dsum = fmaf(dv, __uint_as_float(o[4 * u + z]), dsum);
+        }
+      }
+    }
+  }
+  dsum += __shfl_xor_sync(0xffffffffu, dsum, 2);
+  if (ok && kh == 0) {
+    prm.lse[grow] = m_run + log2f(l_row);
+    prm.dd[grow] = dsum / l_row;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// Stores this thread's 32 values of chunk cb of a gradient row (columns 64cb + kh + 2e, in
+// g[e]) to the output row: an exchange with lane ^ 2 gives each thread the 32 contiguous
+// columns 64cb + 32kh .. +31, written 16 (f32) or 8 (bf16) bytes at a time.
+__device__ __forceinline__ void store_grad_chunk(const float (&g)[32], int cb, int kh, void* base,
+                                                 int32_t dtype) {
+  const int col0 = 64 * cb + 32 * kh;
+#pragma unroll
+  for (int e = 0; e < 16; e += 2) {
+    float w4[4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      // kh = 0 keeps columns 2(e+u), 2(e+u)+1 of the chunk's first half; kh = 1 the second
+      const float mine0 = g[e + u], mine1 = g[16 + e + u];
+      const float recv = __shfl_xor_sync(0xffffffffu, kh ? mine0 : mine1, 2);
+      w4[2 * u] = kh ? recv : mine0;
+      w4[2 * u + 1] = kh ? mine1 : recv;
+    }
+    if (base == nullptr) continue;
+    if (dtype == SAGESLA_F32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(base) + col0 + 2 * e) =
+          make_float4(w4[0], w4[1], w4[2], w4[3]);
+    } else {
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(base) + col0 + 2 * e) =
+          make_uint2(pack_bf16x2(w4[0], w4[1]), pack_bf16x2(w4[2], w4[3]));
+    }
+  }
+}
+
+__device__ __forceinline__ void* grad_row(void* base, int32_t dtype, int64_t sb, int64_t sh,
+                                          int64_t sn, int64_t bh, int H, int tok) {
+  const int64_t b = bh / H, h = bh % H;
+  const int64_t off = b * sb + h * sh + static_cast<int64_t>(tok) * sn;
+  return static_cast<char*>(base) + off * (dtype == SAGESLA_F32 ? 4 : 2);
+}
+
+// dQ of one query block over its kept key blocks: S = Q K^T and dP = dO V^T (one M=64 N=64
+// group each; S in TMEM lanes 0-15 and dP in lanes 16-31 of each quadrant, columns [0, 64)),
+// dS = P (dP - D) with P = 2^(S c - L), dQ += dS K (columns [64, 192)). The linear-branch dq
+// is added before the store.
+__global__ void __launch_bounds__(kBwdThreads, 2)
+k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+         BwdParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* q_t = smem;                   // Q tile
+  uint8_t* o_t = smem + kTile;           // dO tile
+  uint8_t* k_t = smem + 2 * kTile;       // 2 K stages
+  uint8_t* v_t = smem + 4 * kTile;       // 2 V stages
+  uint8_t* s_t = smem + 6 * kTile;       // dS tile
+  __shared__ uint64_t q_full, kv_full[2], s_done, dq_done;
+  __shared__ uint32_t tmem_slot;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int U = prm.k;
+  const int32_t* klist = prm.kept + (bh * prm.nb + i) * static_cast<int64_t>(prm.k);
+  const int blk0 = static_cast<int>(bh * (prm.n_pad / 64));
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 256);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&kv_full[s], 1);
+    mbar_init(&s_done, 1);
+    mbar_init(&dq_done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_do);
+    mbar_arrive_expect_tx(&q_full, 2 * kTile);
+    load_tile(q_t, &tm_q, &q_full, blk0 + i);
+    load_tile(o_t, &tm_do, &q_full, blk0 + i);
+    const int j0 = __ldg(klist);
+    mbar_arrive_expect_tx(&kv_full[0], 2 * kTile);
+    load_tile(k_t, &tm_k, &kv_full[0], blk0 + j0);
+    load_tile(v_t, &tm_v, &kv_full[0], blk0 + j0);
+  }
+  const int row = frag_row(warp, lane);
+  const int kh = (lane >> 1) & 1;
+  const int tok = tile_token(row);
+  const int64_t grow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + tok;
+  const float l2 = prm.lse[grow], dterm = prm.dd[grow];
+  const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
+  const uint32_t lane_p = static_cast<uint32_t>(32 * warp + 16) << 16;
+  const float c2 = kScale * kLog2e;
+  bool ok = true;
+  int j_next = __ldg(klist);
+  for (int n = 0; n < U && ok; ++n) {
+    const int st = n & 1;
+    if (n + 1 < U) j_next = __ldg(klist + n + 1);
+    if (threadIdx.x == 0) {
+      ok = (n > 0 || mbar_wait(&q_full, 0, prm.status)) &&
+           mbar_wait(&kv_full[st], (n >> 1) & 1, prm.status);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t qa = smem_u32(q_t), oa = smem_u32(o_t);
+        const uint32_t kb = smem_u32(k_t + st * kTile), vb = smem_u32(v_t + st * kTile);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem, desc_k128(qa, kk), desc_k128(kb, kk), kIdescKK64, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + (16u << 16), desc_k128(oa, kk), desc_k128(vb, kk), kIdescKK64,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(&s_done);
+      }
+    }
+    if (!mbar_wait(&s_done, n & 1, prm.status)) { ok = false; break; }
+    tc_fence_after();
+    uint32_t sr[32], pr[32];
+    tmem_ld16x64(tmem + lane_s, sr);
+    tmem_ld16x64(tmem + lane_p, pr);
+    tmem_ld_wait();
+    float ds[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
+      ds[e] = p * (__uint_as_float(pr[e]) - dterm);
+    }
+    // dQ(n-1) has read the dS tile and the K / V stage of block n+1
+    if (n > 0 && !mbar_wait(&dq_done, (n - 1) & 1, prm.status)) { ok = false; break; }
+    tc_fence_after();
+    if (threadIdx.x == 0 && n + 1 < U) {
+      mbar_arrive_expect_tx(&kv_full[st ^ 1], 2 * kTile);
+      load_tile(k_t + (st ^ 1) * kTile, &tm_k, &kv_full[st ^ 1], blk0 + j_next);
+      load_tile(v_t + (st ^ 1) * kTile, &tm_v, &kv_full[st ^ 1], blk0 + j_next);
+    }
+    store_row_operand(s_t, row, kh, ds);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      const uint32_t sa = smem_u32(s_t), kb = smem_u32(k_t + st * kTile);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 64, desc_k64(sa, kk), desc_mn128(kb, kk), kIdescKM128,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&dq_done);
+    }
+  }
+  if (ok) ok = mbar_wait(&dq_done, (U - 1) & 1, prm.status);
+  tc_fence_after();
+  if (ok) {
+    const float* lin = prm.lin_q ? prm.lin_q + grow * 128 : nullptr;
+    const int t = 64 * i + tok;
+    void* dst = t < prm.N ? grad_row(prm.dq, prm.g_dtype, prm.dq_sb, prm.dq_sh, prm.dq_sn, bh,
+                                     prm.H, t)
+                          : nullptr;
+#pragma unroll 1
+    for (int cb = 0; cb < 2; ++cb) {
+      uint32_t o[32];
+      tmem_ld16x64(tmem + lane_s + 64 + 64 * cb, o);
+      tmem_ld_wait();
+      float g[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        g[e] = __uint_as_float(o[e]) * kScale + (lin ? lin[64 * cb + kh + 2 * e] : 0.f);
+      store_grad_chunk(g, cb, kh, dst, prm.g_dtype);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// dK, dV of one key block over the query blocks that keep it: S^T = K Q^T and dP^T = V dO^T
+// (lanes 0-15 / 16-31, columns [0, 64)), P^T = 2^(S^T c - L), dS^T = P^T (dP^T - D),
+// dV += P^T dO (lanes 0-15) and dK += dS^T Q (lanes 16-31), columns [64, 192). The
+// linear-branch dk, dv are added before the stores.
+__global__ void __launch_bounds__(kBwdThreads, 2)
+k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+          BwdParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* k_t = smem;                   // K tile
+  uint8_t* v_t = smem + kTile;           // V tile
+  uint8_t* q_t = smem + 2 * kTile;       // Q tile of the current query block
+  uint8_t* o_t = smem + 3 * kTile;       // dO tile
+  uint8_t* p_t = smem + 4 * kTile;       // P^T tile
+  uint8_t* s_t = smem + 4 * kTile + kPTile;   // dS^T tile
+  __shared__ uint64_t kv_full, qo_full, s_done, acc_done;
+  __shared__ uint32_t tmem_slot;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int T = prm.tcount[bh * prm.nb + j];
+  const int32_t* ilist = prm.tlist + (bh * prm.nb + j) * static_cast<int64_t>(prm.nb);
+  const int blk0 = static_cast<int>(bh * (prm.n_pad / 64));
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 256);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    mbar_init(&kv_full, 1);
+    mbar_init(&qo_full, 1);
+    mbar_init(&s_done, 1);
+    mbar_init(&acc_done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_do);
+    mbar_arrive_expect_tx(&kv_full, 2 * kTile);
+    load_tile(k_t, &tm_k, &kv_full, blk0 + j);
+    load_tile(v_t, &tm_v, &kv_full, blk0 + j);
+    if (T > 0) {
+      const int i0 = __ldg(ilist);
+      mbar_arrive_expect_tx(&qo_full, 2 * kTile);
+      load_tile(q_t, &tm_q, &qo_full, blk0 + i0);
+      load_tile(o_t, &tm_do, &qo_full, blk0 + i0);
+    }
+  }
+  const int row = frag_row(warp, lane);
+  const int kh = (lane >> 1) & 1;
+  const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
+  const uint32_t lane_p = static_cast<uint32_t>(32 * warp + 16) << 16;
+  const float c2 = kScale * kLog2e;
+  bool ok = true;
+  for (int t = 0; t < T && ok; ++t) {
+    const int i = __ldg(ilist + t);
+    if (threadIdx.x == 0) {
+      ok = (t > 0 || mbar_wait(&kv_full, 0, prm.status)) &&
+           mbar_wait(&qo_full, t & 1, prm.status);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t ka = smem_u32(k_t), va = smem_u32(v_t);
+        const uint32_t qb = smem_u32(q_t), ob = smem_u32(o_t);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem, desc_k128(ka, kk), desc_k128(qb, kk), kIdescKK64, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + (16u << 16), desc_k128(va, kk), desc_k128(ob, kk), kIdescKK64,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(&s_done);
+      }
+    }
+    // L and D of the query tokens 32kh + e of block i (this thread's columns)
+    const int64_t qrow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + 32 * kh;
+    float lq[32], dq_[32];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(prm.lse + qrow) + u);
+      const float4 b = __ldg(reinterpret_cast<const float4*>(prm.dd + qrow) + u);
+      lq[4 * u] = a.x; lq[4 * u + 1] = a.y; lq[4 * u + 2] = a.z; lq[4 * u + 3] = a.w;
+      dq_[4 * u] = b.x; dq_[4 * u + 1] = b.y; dq_[4 * u + 2] = b.z; dq_[4 * u + 3] = b.w;
+    }
+    if (!mbar_wait(&s_done, t & 1, prm.status)) { ok = false; break; }
+    tc_fence_after();
+    uint32_t sr[32], pr[32];
+    tmem_ld16x64(tmem + lane_s, sr);
+    tmem_ld16x64(tmem + lane_p, pr);
+    tmem_ld_wait();
+    float pt[32], ds[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      pt[e] = exp2f(__uint_as_float(sr[e]) * c2 - lq[e]);
+      ds[e] = pt[e] * (__uint_as_float(pr[e]) - dq_[e]);
+    }
+    // the previous dV / dK MMAs have read the P^T and dS^T tiles and the Q / dO tiles
+    if (t > 0 && !mbar_wait(&acc_done, (t - 1) & 1, prm.status)) { ok = false; break; }
+    store_row_operand(p_t, row, kh, pt);
+    store_row_operand(s_t, row, kh, ds);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      const uint32_t pa = smem_u32(p_t), sa = smem_u32(s_t);
+      const uint32_t qb = smem_u32(q_t), ob = smem_u32(o_t);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 64, desc_k64(pa, kk), desc_mn128(ob, kk), kIdescKM128,
+                 (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + (16u << 16) + 64, desc_k64(sa, kk), desc_mn128(qb, kk), kIdescKM128,
+                 (t > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&acc_done);
+      // next query block's Q and dO once these MMAs have read the tiles
+      if (t + 1 < T && mbar_wait(&acc_done, t & 1, prm.status)) {
+        const int i1 = __ldg(ilist + t + 1);
+        mbar_arrive_expect_tx(&qo_full, 2 * kTile);
+        load_tile(q_t, &tm_q, &qo_full, blk0 + i1);
+        load_tile(o_t, &tm_do, &qo_full, blk0 + i1);
+      }
+    }
+  }
+  if (ok && T > 0) ok = mbar_wait(&acc_done, (T - 1) & 1, prm.status);
+  tc_fence_after();
+  if (ok) {
+    const int tok = tile_token(row);
+    const int t_key = 64 * j + tok;
+    const int64_t grow = bh * prm.n_pad + t_key;
+    const bool real = t_key < prm.N;
+    void* dst_k = real ? grad_row(prm.dk, prm.g_dtype, prm.dk_sb, prm.dk_sh, prm.dk_sn, bh, prm.H,
+                                  t_key)
+                       : nullptr;
+    void* dst_v = real ? grad_row(prm.dv, prm.g_dtype, prm.dv_sb, prm.dv_sh, prm.dv_sn, bh, prm.H,
+                                  t_key)
+                       : nullptr;
+#pragma unroll 1
+    for (int cb = 0; cb < 2; ++cb) {
+      uint32_t ov[32], okk[32];
+      if (T > 0) {
+        tmem_ld16x64(tmem + lane_s + 64 + 64 * cb, ov);
+        tmem_ld16x64(tmem + lane_p + 64 + 64 * cb, okk);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) { ov[e] = 0u; okk[e] = 0u; }
+      }
+      float gk[32], gv[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int c = 64 * cb + kh + 2 * e;
+        gv[e] = __uint_as_float(ov[e]) + (prm.lin_v ? prm.lin_v[grow * 128 + c] : 0.f);
+        gk[e] = __uint_as_float(okk[e]) * kScale + (prm.lin_k ? prm.lin_k[grow * 128 + c] : 0.f);
+      }
+      store_grad_chunk(gk, cb, kh, dst_k, prm.g_dtype);
+      store_grad_chunk(gv, cb, kh, dst_v, prm.g_dtype);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ------------------------------------------------------------------ linear branch (CUDA cores)
+
+constexpr int kLinThreads = 256;            // 64 tokens x 4 parts of 32 channels
+constexpr int kStateLd = 136;               // padded row of a [129][128] state in shared memory
+constexpr int kLinSmem = (129 * kStateLd) * 2 + 2 * 64 * 129 * 4 + 16;
+
+// phi over the 128 channels of a packed bf16 row, this thread's 32 channels [32 part, +32)
+// (the row's four parts are lanes 4t .. 4t+3 of one warp).
+__device__ __forceinline__ void phi_part(const uint16_t* row, int part, float (&a)[32]) {
+  const uint4* r4 = reinterpret_cast<const uint4*>(row) + 4 * part;
+  float mx = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint4 w = __ldg(r4 + u);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int z = 0; z < 4; ++z) {
+      a[8 * u + 2 * z] = bf16_bits_to_f32(ww[z] & 0xFFFFu);
+      a[8 * u + 2 * z + 1] = bf16_bits_to_f32(ww[z] >> 16);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 32; ++e) mx = fmaxf(mx, a[e]);
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) { a[e] = __expf(a[e] - mx); sum += a[e]; }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  const float inv = 1.f / sum;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) a[e] *= inv;
+}
+
+// A [129][128] bf16 state row block (global, [n][c]) into shared memory with padded rows.
+__device__ __forceinline__ void load_state(uint16_t* dst, const uint16_t* src) {
+  for (int e = threadIdx.x; e < 129 * 16; e += kLinThreads) {
+    const int n = e >> 4, c8 = e & 15;
+    *reinterpret_cast<uint4*>(dst + n * kStateLd + 8 * c8) =
+        __ldg(reinterpret_cast<const uint4*>(src + n * 128) + c8);
+  }
+}
+
+// 8 consecutive bf16 of a shared-memory state row as floats.
+__device__ __forceinline__ void state8(const uint16_t* p, float (&f)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int z = 0; z < 4; ++z) {
+    f[2 * z] = bf16_bits_to_f32(ww[z] & 0xFFFFu);
+    f[2 * z + 1] = bf16_bits_to_f32(ww[z] >> 16);
+  }
+}
+
+// Query side of the linear branch for one query block: a = phi(q), num = a G[:, :128],
+// den = a G[:, 128], dnum = dO / den, dden = -(dO . num / den) / den, dq_l = a * (G[:, :128]
+// dnum + G[:, 128] dden), and dG = a^T [dnum | dden] as bf16 [129][128] ([n][c]).
+__global__ void __launch_bounds__(kLinThreads, 2)
+k_bwd_lin_query(const uint16_t* __restrict__ qn, const uint16_t* __restrict__ dn,
+                const uint16_t* __restrict__ gsum, int nb, int nb_m_pad, int n_pad,
+                float* __restrict__ lin_q, uint16_t* __restrict__ dgsum) {
+  extern __shared__ uint8_t smem_raw[];
+  uint16_t* g_s = reinterpret_cast<uint16_t*>(smem_raw);                 // [129][kStateLd]
+  float* a_s = reinterpret_cast<float*>(smem_raw + 129 * kStateLd * 2);  // [64][129]
+  float* n_s = a_s + 64 * 129;                                           // [64][129]: dnum | dden
+  const int i = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int tid = threadIdx.x;
+  uint16_t* dg = dgsum + (bh * nb_m_pad + i) * static_cast<int64_t>(kHFlat);
+  if (i >= nb) {                       // padding rows of the transposed complement GEMM operand
+    for (int e = tid; e < kHFlat; e += kLinThreads) dg[e] = 0;
+    return;
+  }
+  load_state(g_s, gsum + (bh * nb_m_pad + i) * static_cast<int64_t>(kHFlat));
+  const int t = tid >> 2, part = tid & 3;
+  const int64_t grow = bh * n_pad + 64 * static_cast<int64_t>(i) + t;
+  float a[32];
+  phi_part(qn + grow * 128, part, a);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) a_s[t * 129 + 32 * part + e] = a[e];
+  __syncthreads();
+  // num for this thread's columns n = 32 part + e; den partial over its channels
+  float num[32];
+#pragma unroll
+  for (int g8 = 0; g8 < 4; ++g8) {       // eight columns at a time
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 1
+    for (int c8 = 0; c8 < 16; ++c8) {
+      float av[8];
+#pragma unroll
+      for (int z = 0; z < 8; ++z) av[z] = a_s[t * 129 + 8 * c8 + z];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float gv[8];
+        state8(g_s + (32 * part + 8 * g8 + e) * kStateLd + 8 * c8, gv);
+#pragma unroll
+        for (int z = 0; z < 8; ++z) acc[e] = fmaf(av[z], gv[z], acc[e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) num[8 * g8 + e] = acc[e];
+  }
+  float den = 0.f;
+  {
+    float gv[8];
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      state8(g_s + 128 * kStateLd + 32 * part + 8 * c8, gv);
+#pragma unroll
+      for (int z = 0; z < 8; ++z) den = fmaf(a[8 * c8 + z], gv[z], den);
+    }
+  }
+  den += __shfl_xor_sync(0xffffffffu, den, 1);
+  den += __shfl_xor_sync(0xffffffffu, den, 2);
+  // dnum, dden
+  const uint4* d4 = reinterpret_cast<const uint4*>(dn + grow * 128) + 4 * part;
+  const float inv_den = 1.f / den;
+  float dden = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint4 w = __ldg(d4 + u);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int z = 0; z < 4; ++z) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int e = 8 * u + 2 * z + hh;
+        const float dov = bf16_bits_to_f32(hh ? (ww[z] >> 16) : (ww[z] & 0xFFFFu));
+        dden = fmaf(dov, num[e] * inv_den, dden);
+        n_s[t * 129 + 32 * part + e] = dov * inv_den;
+      }
+    }
+  }
+  dden += __shfl_xor_sync(0xffffffffu, dden, 1);
+  dden += __shfl_xor_sync(0xffffffffu, dden, 2);
+  dden = -dden * inv_den;
+  if (part == 0) n_s[t * 129 + 128] = dden;
+  __syncthreads();
+  // da for this thread's channels c = 32 part + e: sum over n of G[n][c] dnum[n] + G[128][c] dden
+  float da[32];
+  {
+    float gv[8];
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      state8(g_s + 128 * kStateLd + 32 * part + 8 * c8, gv);
+#pragma unroll
+      for (int z = 0; z < 8; ++z) da[8 * c8 + z] = gv[z] * dden;
+    }
+  }
+  for (int n = 0; n < 128; ++n) {
+    const float dnv = n_s[t * 129 + n];
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      float gv[8];
+      state8(g_s + n * kStateLd + 32 * part + 8 * c8, gv);
+#pragma unroll
+      for (int z = 0; z < 8; ++z) da[8 * c8 + z] = fmaf(gv[z], dnv, da[8 * c8 + z]);
+    }
+  }
+  float4* lq = reinterpret_cast<float4*>(lin_q + grow * 128 + 32 * part);
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    lq[u] = make_float4(a[4 * u] * da[4 * u], a[4 * u + 1] * da[4 * u + 1],
+                        a[4 * u + 2] * da[4 * u + 2], a[4 * u + 3] * da[4 * u + 3]);
+  // dG[n][c] = sum over the block's tokens of a[t][c] (dnum | dden)[t][n]; thread: channel c,
+  // rows n = nh, nh + 2, ...
+  const int c = tid & 127, nh = tid >> 7;
+  float acol[64];
+#pragma unroll
+  for (int tt = 0; tt < 64; ++tt) acol[tt] = a_s[tt * 129 + c];
+  for (int n = nh; n < 129; n += 2) {
+    float sacc = 0.f;
+#pragma unroll
+    for (int tt = 0; tt < 64; ++tt) sacc = fmaf(acol[tt], n_s[tt * 129 + n], sacc);
+    dg[n * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(sacc));
+  }
+}
+
+// Key side of the linear branch for one key block: b = phi(k), db = dH[:, :128] v + dH[:, 128],
+// dk_l = b * (db - b . db), dv_l = dH[:, :128]^T b (dH as bf16 [129][128], [n][c]).
+__global__ void __launch_bounds__(kLinThreads, 2)
+k_bwd_lin_key(const uint16_t* __restrict__ kn, const uint16_t* __restrict__ vn,
+              const uint16_t* __restrict__ dhsum, int nb_m_pad, int n_pad,
+              float* __restrict__ lin_k, float* __restrict__ lin_v) {
+  extern __shared__ uint8_t smem_raw[];
+  uint16_t* h_s = reinterpret_cast<uint16_t*>(smem_raw);                 // [129][kStateLd]
+  float* b_s = reinterpret_cast<float*>(smem_raw + 129 * kStateLd * 2);  // [64][129]
+  float* v_s = b_s + 64 * 129;                                           // [64][129]
+  const int j = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int tid = threadIdx.x;
+  load_state(h_s, dhsum + (bh * nb_m_pad + j) * static_cast<int64_t>(kHFlat));
+  const int t = tid >> 2, part = tid & 3;
+  const int64_t grow = bh * n_pad + 64 * static_cast<int64_t>(j) + t;
+  float b[32];
+  phi_part(kn + grow * 128, part, b);
+  const uint4* v4 = reinterpret_cast<const uint4*>(vn + grow * 128) + 4 * part;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint4 w = __ldg(v4 + u);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int z = 0; z < 4; ++z) {
+      v_s[t * 129 + 32 * part + 8 * u + 2 * z] = bf16_bits_to_f32(ww[z] & 0xFFFFu);
+      v_s[t * 129 + 32 * part + 8 * u + 2 * z + 1] = bf16_bits_to_f32(ww[z] >> 16);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 32; ++e) b_s[t * 129 + 32 * part + e] = b[e];
+  __syncthreads();
+  // db for this thread's channels c = 32 part + e
+  float db[32];
+  {
+    float hv[8];
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      state8(h_s + 128 * kStateLd + 32 * part + 8 * c8, hv);
+#pragma unroll
+      for (int z = 0; z < 8; ++z) db[8 * c8 + z] = hv[z];
+    }
+  }
+  for (int n = 0; n < 128; ++n) {
+    const float vv = v_s[t * 129 + n];
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      float hv[8];
+      state8(h_s + n * kStateLd + 32 * part + 8 * c8, hv);
+#pragma unroll
+      for (int z = 0; z < 8; ++z) db[8 * c8 + z] = fmaf(hv[z], vv, db[8 * c8 + z]);
+    }
+  }
+  float proj = 0.f;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) proj = fmaf(b[e], db[e], proj);
+  proj += __shfl_xor_sync(0xffffffffu, proj, 1);
+  proj += __shfl_xor_sync(0xffffffffu, proj, 2);
+  float4* lk = reinterpret_cast<float4*>(lin_k + grow * 128 + 32 * part);
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    lk[u] = make_float4(b[4 * u] * (db[4 * u] - proj), b[4 * u + 1] * (db[4 * u + 1] - proj),
+                        b[4 * u + 2] * (db[4 * u + 2] - proj), b[4 * u + 3] * (db[4 * u + 3] - proj));
+  // dv for this thread's columns n = 32 part + e: sum over c of b[c] dH[n][c]
+  float4* lv = reinterpret_cast<float4*>(lin_v + grow * 128 + 32 * part);
+#pragma unroll
+  for (int g8 = 0; g8 < 4; ++g8) {       // eight columns at a time
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 1
+    for (int c8 = 0; c8 < 16; ++c8) {
+      float bv[8];
+#pragma unroll
+      for (int z = 0; z < 8; ++z) bv[z] = b_s[t * 129 + 8 * c8 + z];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float hv[8];
+        state8(h_s + (32 * part + 8 * g8 + e) * kStateLd + 8 * c8, hv);
+#pragma unroll
+        for (int z = 0; z < 8; ++z) acc[e] = fmaf(bv[z], hv[z], acc[e]);
+      }
+    }
+    lv[2 * g8] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    lv[2 * g8 + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+}  // namespace
+
+bool make_backward_layout(const ForwardPlan& p, BackwardLayout* bl) {
+  size_t off = p.lay.total_bytes;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = (off + bytes + 255) & ~static_cast<size_t>(255);
+    return at;
+  };
+  const size_t rows = static_cast<size_t>(p.BH * p.n_pad);
+  bl->qn = take(rows * 256);
+  bl->kn = take(rows * 256);
+  bl->vn = take(rows * 256);
+  bl->dn = take(rows * 256);
+  bl->lse = take(rows * 4);
+  bl->dd = take(rows * 4);
+  bl->tcount = take(static_cast<size_t>(p.BH * p.nb) * 4);
+  bl->tlist = take(static_cast<size_t>(p.BH * p.nb * p.nb) * 4);
+  if (!p.linear_empty) {
+    bl->lin_q = take(rows * 512);
+    bl->lin_k = take(rows * 512);
+    bl->lin_v = take(rows * 512);
+    bl->amask_t = take(static_cast<size_t>(p.BH * p.nb_m_pad * p.nb_m_pad) * 2);
+    bl->dg = take(static_cast<size_t>(p.BH * p.nb_m_pad) * kHFlat * 2);
+    bl->dh = take(static_cast<size_t>(p.BH * p.nb_m_pad) * kHFlat * 2);
+  } else {
+    bl->lin_q = bl->lin_k = bl->lin_v = bl->amask_t = bl->dg = bl->dh = 0;
+  }
+  bl->total = off;
+  return true;
+}
+
+namespace {
+
+// Four-dimensional map of a packed [rows][128] bf16 buffer whose box is one key-interleaved
+// 64 x 64 tile: dims (column, half, row in half, 64-row block), strides 32 rows, 1 row and 64
+// rows, box (64, 2, 32, 1); the box lands in shared memory as rows 2i + h <- token 32h + i.
+bool encode_interleaved(CUtensorMap* map, const void* base, int64_t rows) {
+  const uint64_t dims[4] = {128, 2, 32, static_cast<uint64_t>(rows / 64)};
+  const uint64_t strides[3] = {32 * 256, 256, 64 * 256};
+  const uint32_t box[4] = {64, 2, 32, 1};
+  return encode_tmap_nd(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, TensorArg q,
+                                TensorArg k, TensorArg v, TensorArg d_out, const GradOut& g,
+                                char* ws, cudaStream_t stream) {
+  const auto& L = p.lay;
+  const int64_t rows = p.BH * p.n_pad;
+  cudaError_t e;
+  // packed copies, transposed kept lists
+  {
+    const int64_t total = rows * 16;
+    k_bwd_pack<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
+        q, k, v, d_out, static_cast<int>(p.N), static_cast<int>(p.n_pad), total,
+        reinterpret_cast<uint4*>(ws + bl.qn), reinterpret_cast<uint4*>(ws + bl.kn),
+        reinterpret_cast<uint4*>(ws + bl.vn), reinterpret_cast<uint4*>(ws + bl.dn));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int64_t warps = p.BH * p.nb;
+    k_bwd_lists<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, stream>>>(
+        static_cast<int>(p.nb), static_cast<int>(p.mask_words), p.BH,
+        reinterpret_cast<const uint32_t*>(ws + L.mask), reinterpret_cast<int32_t*>(ws + bl.tcount),
+        reinterpret_cast<int32_t*>(ws + bl.tlist));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  CUtensorMap tq, tk, tv, td;
+  if (!encode_interleaved(&tq, ws + bl.qn, rows) || !encode_interleaved(&tk, ws + bl.kn, rows) ||
+      !encode_interleaved(&tv, ws + bl.vn, rows) || !encode_interleaved(&td, ws + bl.dn, rows))
+    return cudaErrorInvalidValue;
+  BwdParams prm;
+  prm.kept = reinterpret_cast<const int32_t*>(ws + L.kept);
+  prm.tcount = reinterpret_cast<const int32_t*>(ws + bl.tcount);
+  prm.tlist = reinterpret_cast<const int32_t*>(ws + bl.tlist);
+  prm.qn = reinterpret_cast<const uint16_t*>(ws + bl.qn);
+  prm.dn = reinterpret_cast<const uint16_t*>(ws + bl.dn);
+  prm.lse = reinterpret_cast<float*>(ws + bl.lse);
+  prm.dd = reinterpret_cast<float*>(ws + bl.dd);
+  prm.lin_q = p.linear_empty ? nullptr : reinterpret_cast<const float*>(ws + bl.lin_q);
+  prm.lin_k = p.linear_empty ? nullptr : reinterpret_cast<const float*>(ws + bl.lin_k);
+  prm.lin_v = p.linear_empty ? nullptr : reinterpret_cast<const float*>(ws + bl.lin_v);
+  prm.dq = g.dq; prm.dk = g.dk; prm.dv = g.dv;
+  prm.dq_sb = g.dq_s[0]; prm.dq_sh = g.dq_s[1]; prm.dq_sn = g.dq_s[2];
+  prm.dk_sb = g.dk_s[0]; prm.dk_sh = g.dk_s[1]; prm.dk_sn = g.dk_s[2];
+  prm.dv_sb = g.dv_s[0]; prm.dv_sh = g.dv_s[1]; prm.dv_sn = g.dv_s[2];
+  prm.g_dtype = g.dtype;
+  prm.status = reinterpret_cast<int*>(ws + L.status);
+  prm.N = static_cast<int>(p.N);
+  prm.nb = static_cast<int>(p.nb);
+  prm.n_pad = static_cast<int>(p.n_pad);
+  prm.k = static_cast<int>(p.k);
+  prm.n_last = p.n_last;
+  prm.H = static_cast<int>(p.H);
+  const dim3 grid(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.BH));
+  const int smem_lse = 1024 + 5 * kTile + kPTile;
+  const int smem_dq = 1024 + 6 * kTile + kPTile;
+  const int smem_dkv = 1024 + 4 * kTile + 2 * kPTile;
+  static bool configured = false;
+  if (!configured) {
+    if ((e = cudaFuncSetAttribute(k_bwd_lse, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_lse)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(k_bwd_dq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(k_bwd_dkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(k_bwd_lin_query, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(k_bwd_lin_key, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem)) != cudaSuccess)
+      return e;
+    configured = true;
+  }
+  k_bwd_lse<<<grid, kBwdThreads, smem_lse, stream>>>(tq, tk, tv, prm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (!p.linear_empty) {
+    const dim3 gq(static_cast<unsigned>(p.nb_m_pad), static_cast<unsigned>(p.BH));
+    k_bwd_lin_query<<<gq, kLinThreads, kLinSmem, stream>>>(
+        prm.qn, prm.dn, reinterpret_cast<const uint16_t*>(ws + L.gsum), static_cast<int>(p.nb),
+        static_cast<int>(p.nb_m_pad), static_cast<int>(p.n_pad),
+        reinterpret_cast<float*>(ws + bl.lin_q), reinterpret_cast<uint16_t*>(ws + bl.dg));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const dim3 gt(static_cast<unsigned>(p.nb_m_pad / 32), static_cast<unsigned>(p.nb_m_pad / 32),
+                  static_cast<unsigned>(p.BH));
+    k_bwd_transpose_mask<<<gt, dim3(32, 8), 0, stream>>>(
+        static_cast<int>(p.nb_m_pad), static_cast<int>(p.nb_k_pad),
+        reinterpret_cast<const uint16_t*>(ws + L.amask), reinterpret_cast<uint16_t*>(ws + bl.amask_t));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // dH = (1 - M)^T dG: the complement GEMM with the transposed mask, rows and depth nb_m_pad
+    if ((e = launch_mask_gemm(ws + bl.amask_t, ws + bl.dg, ws + bl.dh, p.BH, p.nb_m_pad,
+                              p.nb_m_pad, prm.status, stream)) != cudaSuccess)
+      return e;
+    const dim3 gk(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.BH));
+    k_bwd_lin_key<<<gk, kLinThreads, kLinSmem, stream>>>(
+        reinterpret_cast<const uint16_t*>(ws + bl.kn), reinterpret_cast<const uint16_t*>(ws + bl.vn),
+        reinterpret_cast<const uint16_t*>(ws + bl.dh), static_cast<int>(p.nb_m_pad),
+        static_cast<int>(p.n_pad), reinterpret_cast<float*>(ws + bl.lin_k),
+        reinterpret_cast<float*>(ws + bl.lin_v));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  k_bwd_dq<<<grid, kBwdThreads, smem_dq, stream>>>(tq, tk, tv, td, prm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  k_bwd_dkv<<<grid, kBwdThreads, smem_dkv, stream>>>(tq, tk, tv, td, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace sagesla

@@ -40,6 +40,36 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint64_t inner,
                     uint64_t row_bytes, const void* base, uint32_t box_inner, uint32_t box_outer,
                     CUtensorMapSwizzle swizzle);
 
+// Same for a tiled map of any rank (dims[0] contiguous; strides in bytes of dims 1..rank-1).
+bool encode_tmap_nd(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const void* base,
+                    const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                    CUtensorMapSwizzle swizzle);
+
+// Workspace of the SLA backward: the forward's layout followed by these regions.
+struct BackwardLayout {
+  size_t qn, kn, vn, dn;            // packed bf16 Q, K, V, dO [BH][n_pad][128]
+  size_t lse, dd;                   // [BH][n_pad] f32
+  size_t tcount, tlist;             // query blocks keeping each key block: [BH][nb], [BH][nb][nb]
+  size_t lin_q, lin_k, lin_v;       // linear-branch gradients [BH][n_pad][128] f32
+  size_t amask_t;                   // transposed complement mask [BH][nb_m_pad][nb_m_pad] bf16
+  size_t dg, dh;                    // [BH][nb_m_pad][129 * 128] bf16
+  size_t total;
+};
+bool make_backward_layout(const ForwardPlan& p, BackwardLayout* bl);
+
+// Gradient outputs of the backward (one dtype for all three; strides in elements).
+struct GradOut {
+  void* dq; void* dk; void* dv;
+  int64_t dq_s[3], dk_s[3], dv_s[3];
+  int32_t dtype;
+};
+cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, TensorArg q,
+                                TensorArg k, TensorArg v, TensorArg d_out, const GradOut& g,
+                                char* ws, cudaStream_t stream);
+// C[BH][M][16512] = A[BH][M][K] . B[BH][K][16512] (bf16, M a multiple of 128, K of 64).
+cudaError_t launch_mask_gemm(const void* a, const void* b, void* c, int64_t BH, int64_t M,
+                             int64_t K, int* status, cudaStream_t stream);
+
 // Kernel launchers (defined next to their kernels); each returns the launch error.
 cudaError_t launch_stats(const ForwardPlan& p, TensorArg k, TensorArg v, char* ws,
                          cudaStream_t stream);

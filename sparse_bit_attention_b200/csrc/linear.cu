@@ -164,31 +164,34 @@ k_complement_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 
 }  // namespace
 
+cudaError_t launch_mask_gemm(const void* a, const void* b, void* c, int64_t BH, int64_t M,
+                             int64_t K, int* status, cudaStream_t stream) {
+  CUtensorMap ta, tb, tg;
+  if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, BH * M, K * 2, a, kTileK, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHFlat, BH * K,
+                      static_cast<uint64_t>(kHFlat) * 2, b, 64, kTileK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHFlat, BH * M,
+                      static_cast<uint64_t>(kHFlat) * 2, c, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(k_complement_gemm,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid((kHFlat + kTileN - 1) / kTileN, static_cast<unsigned>((M + kTileM - 1) / kTileM),
+            static_cast<unsigned>(BH));
+  k_complement_gemm<<<grid, kGemmThreads, kGemmSmem, stream>>>(
+      ta, tb, tg, static_cast<int>(M), static_cast<int>(K), status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_complement_gemm(const ForwardPlan& p, char* ws, cudaStream_t stream) {
   const auto& L = p.lay;
-  CUtensorMap ta, tb;
-  if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.nb_k_pad, p.BH * p.nb_m_pad,
-                      p.nb_k_pad * 2, ws + L.amask, kTileK, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  if (!encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHFlat, p.BH * p.nb_k_pad,
-                      static_cast<uint64_t>(kHFlat) * 2, ws + L.hflat, 64, kTileK,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  CUtensorMap tg;
-  if (!encode_tmap_2d(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHFlat, p.BH * p.nb_m_pad,
-                      static_cast<uint64_t>(kHFlat) * 2, ws + L.gsum, 64, 32,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_complement_gemm,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-  if (e != cudaSuccess) return e;
-  dim3 grid((kHFlat + kTileN - 1) / kTileN, static_cast<unsigned>((p.nb_m_pad + kTileM - 1) / kTileM),
-            static_cast<unsigned>(p.BH));
-  k_complement_gemm<<<grid, kGemmThreads, kGemmSmem, stream>>>(
-      ta, tb, tg, static_cast<int>(p.nb_m_pad), static_cast<int>(p.nb_k_pad),
-      reinterpret_cast<int*>(ws + L.status));
-  return cudaGetLastError();
+  return launch_mask_gemm(ws + L.amask, ws + L.hflat, ws + L.gsum, p.BH, p.nb_m_pad, p.nb_k_pad,
+                          reinterpret_cast<int*>(ws + L.status), stream);
 }
 
 }  // namespace sagesla

@@ -98,9 +98,9 @@ bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* 
   return true;
 }
 
-bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint64_t inner, uint64_t outer,
-                    uint64_t row_bytes, const void* base, uint32_t box_inner, uint32_t box_outer,
-                    CUtensorMapSwizzle swizzle) {
+namespace {
+// cuTensorMapEncodeTiled through the runtime's driver entry point, resolved once.
+bool have_encode() {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -109,7 +109,14 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint64_t inner,
         q == cudaDriverEntryPointSuccess)
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
-  if (!g_encode) return false;
+  return g_encode != nullptr;
+}
+}  // namespace
+
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, const void* base, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle) {
+  if (!have_encode()) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
@@ -119,6 +126,21 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint64_t inner,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_nd(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const void* base,
+                    const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                    CUtensorMapSwizzle swizzle) {
+  if (!have_encode() || rank < 1 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es[5];
+  for (uint32_t r = 0; r < rank; ++r) { d[r] = dims[r]; b[r] = box[r]; es[r] = 1; }
+  for (uint32_t r = 0; r + 1 < rank; ++r) st[r] = strides[r];
+  const CUresult res = g_encode(map, dtype, rank, const_cast<void*>(base), d, st, b, es,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
 }
 
 namespace {
@@ -301,6 +323,84 @@ sagesla_status sagesla_forward(const sagesla_tensor* q, const sagesla_tensor* k,
                                void* stream) {
   return sagesla_forward_ex(q, k, v, topk_ratio, block, out, workspace, workspace_bytes, stream,
                             nullptr);
+}
+
+size_t sagesla_sla_backward_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D,
+                                           double topk_ratio, int block) {
+  if (D != kHeadDim || block != kBlock) return 0;
+  ForwardPlan p;
+  if (!make_plan(B, H, N, topk_ratio, &p)) return 0;
+  BackwardLayout bl;
+  if (!make_backward_layout(p, &bl)) return 0;
+  return bl.total;
+}
+
+sagesla_status sagesla_sla_backward(const sagesla_tensor* q, const sagesla_tensor* k,
+                                    const sagesla_tensor* v, const sagesla_tensor* d_out,
+                                    double topk_ratio, int block, sagesla_tensor* dq,
+                                    sagesla_tensor* dk, sagesla_tensor* dv, void* workspace,
+                                    size_t workspace_bytes, void* stream_ptr) {
+  sagesla_status st;
+  if ((st = check_view(q, nullptr, false)) != SAGESLA_OK) return st;
+  for (const sagesla_tensor* t : {k, v, d_out})
+    if ((st = check_view(t, q, false)) != SAGESLA_OK) return st;
+  for (const sagesla_tensor* t : {dq, dk, dv})
+    if ((st = check_view(t, q, true)) != SAGESLA_OK) return st;
+  if (dk->dtype != dq->dtype || dv->dtype != dq->dtype) return SAGESLA_ERR_UNSUPPORTED;
+  if (block != kBlock) return SAGESLA_ERR_UNSUPPORTED;
+  if (!valid_ratio(topk_ratio)) return SAGESLA_ERR_INVALID_ARG;
+  ForwardPlan p;
+  if (!make_plan(q->B, q->H, q->N, topk_ratio, &p)) return SAGESLA_ERR_INVALID_ARG;
+  BackwardLayout bl;
+  if (!make_backward_layout(p, &bl)) return SAGESLA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
+      workspace_bytes < bl.total)
+    return SAGESLA_ERR_WORKSPACE;
+  // outputs must not overlap the inputs, each other or the workspace
+  const uintptr_t w0 = reinterpret_cast<uintptr_t>(workspace);
+  const sagesla_tensor* outs[3] = {dq, dk, dv};
+  for (int a = 0; a < 3; ++a) {
+    uintptr_t o0, o1, x0, x1;
+    extent(outs[a], &o0, &o1);
+    if (overlaps(o0, o1, w0, w0 + bl.total)) return SAGESLA_ERR_INVALID_ARG;
+    for (const sagesla_tensor* t : {q, k, v, d_out}) {
+      extent(t, &x0, &x1);
+      if (overlaps(o0, o1, x0, x1)) return SAGESLA_ERR_INVALID_ARG;
+    }
+    for (int b = a + 1; b < 3; ++b) {
+      extent(outs[b], &x0, &x1);
+      if (overlaps(o0, o1, x0, x1)) return SAGESLA_ERR_INVALID_ARG;
+    }
+  }
+  if ((st = check_device()) != SAGESLA_OK) return st;
+
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  char* ws = static_cast<char*>(workspace);
+  const TensorArg qa = to_arg(q), ka = to_arg(k), va = to_arg(v), da = to_arg(d_out);
+  SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.lay.status, 0, sizeof(int32_t), stream));
+  // the forward's selection and complement sums (same kernels, so the same block mask)
+  SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
+  SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
+  SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
+  if (!p.linear_empty) {
+    SAGESLA_LAUNCH(launch_scores(p, ws, stream));
+    SAGESLA_LAUNCH(launch_topk(p, ws, stream));
+    SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
+  } else {
+    SAGESLA_LAUNCH(launch_fill_all_kept(p, ws, stream));
+  }
+  GradOut g;
+  g.dq = dq->data; g.dk = dk->data; g.dv = dv->data;
+  const sagesla_tensor* gs[3] = {dq, dk, dv};
+  int64_t* dst[3] = {g.dq_s, g.dk_s, g.dv_s};
+  for (int a = 0; a < 3; ++a) {
+    dst[a][0] = gs[a]->stride_b;
+    dst[a][1] = gs[a]->stride_h;
+    dst[a][2] = gs[a]->stride_n;
+  }
+  g.dtype = dq->dtype;
+  SAGESLA_LAUNCH(launch_sla_backward(p, bl, qa, ka, va, da, g, ws, stream));
+  return SAGESLA_OK;
 }
 
 }  // extern "C"

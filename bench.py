@@ -59,7 +59,7 @@ def parse_args():
                     help="Top-K ratio (default: 0.1; 1.0 is the dense SageAttention mode)")
     ap.add_argument("--sweep", action="store_true",
                     help="Top-K ratio sweep and dense BF16 comparison, one JSON line per point")
-    ap.add_argument("--kernel-case", choices=["norm", "w8a8"], default=None,
+    ap.add_argument("--kernel-case", choices=["norm", "w8a8", "bwd"], default=None,
                     help="run a small case of one next-row kernel a few times (for ncu captures)")
     args = ap.parse_args()
     globals()["WORKLOAD"] = args.workload
@@ -493,6 +493,72 @@ def _time_w8a8(sba, torch, steps, warmup, M=75600, K=5120, N=5120):
     return M, K, N, ms_w8, ms_bf16
 
 
+def backward_tensor_flops(B, H, nb, k):
+    """Tensor-core FLOPs of the SLA backward's sparse branch: per kept (query block, key block)
+    pair nine 64x64x128 products (S and P.V again for the log-sum-exp; S, dP and dQ; S^T, dP^T,
+    dV and dK), 2 FLOPs per multiply-add; plus the two complement GEMMs (G and dH), each
+    2 nb_pad^2 16512 per head."""
+    nb_pad = -(-nb // 128) * 128
+    return B * H * nb * k * 9 * 2 * (64 * 64 * 128) + B * H * 2 * 2 * nb_pad * nb_pad * 16512
+
+
+def _time_backward(sba, torch, q, k, v, ratio, steps, warmup):
+    """SLA backward (bf16 gradients) on resident inputs and a seeded dO, and torch's dense
+    bf16 attention backward of the same shape for context."""
+    g = torch.Generator().manual_seed(21)
+    d_out = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(q.device)
+    B, H, N, D = q.shape
+    ws = sba.alloc_workspace(sba.sagesla_sla_backward_workspace_size(B, H, N, D, ratio), q.device)
+    grads = [torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) for _ in range(3)]
+    run = lambda: sba.sagesla_sla_backward(q, k, v, d_out, ratio, dq=grads[0], dk=grads[1],
+                                           dv=grads[2], workspace=ws)
+    for _ in range(warmup):
+        run()
+    st = sba.sagesla_stream_status(None, ws)
+    if st != 0:
+        raise RuntimeError(f"device status: {sba.sagesla_status_string(st)}")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del ws, grads
+    torch.cuda.empty_cache()
+    # dense baseline: forward + backward of torch SDPA minus its forward
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    ms_dense, backend = None, None
+    for be in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION):
+        try:
+            with sdpa_kernel([be]):
+                qq, kk, vv = (x.detach().requires_grad_(True) for x in (q, k, v))
+                out = F.scaled_dot_product_attention(qq, kk, vv)
+                out.backward(d_out)
+                torch.cuda.synchronize()
+                e0.record()
+                for _ in range(max(1, steps // 2)):
+                    out = F.scaled_dot_product_attention(qq, kk, vv)
+                    out.backward(d_out)
+                e1.record()
+                torch.cuda.synchronize()
+                fwd_bwd = e0.elapsed_time(e1) / max(1, steps // 2)
+                e0.record()
+                for _ in range(max(1, steps // 2)):
+                    F.scaled_dot_product_attention(qq, kk, vv)
+                e1.record()
+                torch.cuda.synchronize()
+                ms_dense = fwd_bwd - e0.elapsed_time(e1) / max(1, steps // 2)
+                backend = be.name
+                del qq, kk, vv, out
+            break
+        except RuntimeError:
+            continue
+    torch.cuda.empty_cache()
+    return ms, ms_dense, backend
+
+
 def run_sweep(args):
     import torch
     import sparse_bit_attention_b200 as sba
@@ -518,6 +584,19 @@ def run_sweep(args):
                 "dense_equiv_tops": dense_ops / (ms / 1e3) / 1e12,
                 "stage_ms": stage}), flush=True)
         if name == "wan21_14b_720p":
+            lay = sba.sagesla_get_workspace_layout(B, H, N, D, 0.1)
+            ms_b, ms_dense, be = _time_backward(sba, torch, q, k, v, 0.1, max(3, steps // 2),
+                                                args.warmup)
+            peaks, src = measured_peaks()
+            fl = backward_tensor_flops(B, H, lay["nb"], lay["k"])
+            print(json.dumps({
+                "sweep": "sla_backward", "workload": name, "topk_ratio": 0.1,
+                "grad_dtype": "bfloat16", "ms_per_backward": ms_b,
+                "tokens_per_s": B * N / (ms_b / 1e3), "tensor_tflop": fl / 1e12,
+                "tensor_tflops": fl / (ms_b / 1e3) / 1e12,
+                "frac_of_bf16_sustained": fl / (ms_b / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                "peak_source": src, "dense_baseline": f"torch SDPA backward ({be}), bf16",
+                "dense_backward_ms": ms_dense}), flush=True)
             backend, ms = _time_sdpa(torch, q, k, v, max(2, steps // 2), 1)
             print(json.dumps({
                 "sweep": name, "baseline": "torch scaled_dot_product_attention, bf16 dense",
@@ -564,6 +643,17 @@ def run_kernel_case(args):
         for _ in range(3):
             sba.sagesla_norm_quant(x, sba.SAGESLA_LAYER_NORM, 1e-6, None, None, scale, shift,
                                    rows_per_sample=M, want_codes=True)
+    elif args.kernel_case == "bwd":
+        # SLA backward on the Wan2.1-1.3B-480P attention shape (B1 H12 N32760, ratio 0.1)
+        from sparse_bit_attention_b200 import inputs
+        q, k, v = (x.cuda() for x in inputs.make_qkv("wan21_1p3b_480p"))
+        d_out = torch.randn(q.shape, generator=g).to(torch.bfloat16).cuda()
+        B, H, N, D = q.shape
+        ws = sba.alloc_workspace(sba.sagesla_sla_backward_workspace_size(B, H, N, D, 0.1))
+        for _ in range(2):
+            sba.sagesla_sla_backward(q, k, v, d_out, 0.1, grad_dtype=torch.bfloat16, workspace=ws)
+        if sba.sagesla_stream_status(None, ws) != 0:
+            raise RuntimeError("device status after the backward")
     else:
         M, K, N = 16384, 5120, 5120
         x = (torch.randn(M, K, generator=g) * 1.5).to(torch.bfloat16).cuda()

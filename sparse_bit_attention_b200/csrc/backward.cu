@@ -725,273 +725,357 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
-// ------------------------------------------------------------------ linear branch (CUDA cores)
+// ------------------------------------------------------------------ linear branch (tcgen05)
 
-constexpr int kLinThreads = 256;            // 64 tokens x 4 parts of 32 channels
-constexpr int kStateLd = 136;               // padded row of a [129][128] state in shared memory
-constexpr int kLinSmem = (129 * kStateLd) * 2 + 2 * 64 * 129 * 4 + 16;
+// A [129][128] state block (G_i or dH_j, bf16 [n][c]) lives in shared memory as rows n < 128
+// only, two 16 KB chunks of 64 channels (128-byte swizzled), loaded by TMA; row 128 is read
+// from global memory. As a B operand it is K-major with K = c (N = n) or MN-major with K = n
+// (N = c).
+__device__ __forceinline__ uint64_t desc_state_kmajor(uint32_t base, int kk) {   // K = c
+  return make_sdesc(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+}
+__device__ __forceinline__ uint64_t desc_state_mnmajor(uint32_t base, int kk) {  // K = n
+  return make_sdesc(base + kk * 2048, 16384, 1024, kLayoutSW128);
+}
+constexpr uint32_t kStateTile = 2 * 16384;
+constexpr uint32_t kIdescMM128 = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 1, 1, 128, 128);
+constexpr uint32_t kIdescKK128 = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 64, 128);
 
-// phi over the 128 channels of a packed bf16 row, this thread's 32 channels [32 part, +32)
-// (the row's four parts are lanes 4t .. 4t+3 of one warp).
-__device__ __forceinline__ void phi_part(const uint16_t* row, int part, float (&a)[32]) {
-  const uint4* r4 = reinterpret_cast<const uint4*>(row) + 4 * part;
-  float mx = -INFINITY;
+// This thread's half of phi over a packed bf16 row (channels 64 kh .. 64 kh + 63; the row's
+// other half is lane ^ 2) into the K-major A tile (chunk kh of row r) and the f32 copy a32.
+__device__ __forceinline__ void phi_half_row(const uint16_t* row, int r, int kh, uint8_t* tile,
+                                             float* a32) {
+  const uint4* r4 = reinterpret_cast<const uint4*>(row) + 8 * kh;
+  float x[64];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < 8; ++u) {
     const uint4 w = __ldg(r4 + u);
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int z = 0; z < 4; ++z) {
-      a[8 * u + 2 * z] = bf16_bits_to_f32(ww[z] & 0xFFFFu);
-      a[8 * u + 2 * z + 1] = bf16_bits_to_f32(ww[z] >> 16);
+      x[8 * u + 2 * z] = bf16_bits_to_f32(ww[z] & 0xFFFFu);
+      x[8 * u + 2 * z + 1] = bf16_bits_to_f32(ww[z] >> 16);
     }
   }
+  float mx = -INFINITY;
 #pragma unroll
-  for (int e = 0; e < 32; ++e) mx = fmaxf(mx, a[e]);
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  for (int e = 0; e < 64; ++e) mx = fmaxf(mx, x[e]);
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   float sum = 0.f;
 #pragma unroll
-  for (int e = 0; e < 32; ++e) { a[e] = __expf(a[e] - mx); sum += a[e]; }
-  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  for (int e = 0; e < 64; ++e) { x[e] = __expf(x[e] - mx); sum += x[e]; }
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
   const float inv = 1.f / sum;
 #pragma unroll
-  for (int e = 0; e < 32; ++e) a[e] *= inv;
-}
-
-// A [129][128] bf16 state row block (global, [n][c]) into shared memory with padded rows.
-__device__ __forceinline__ void load_state(uint16_t* dst, const uint16_t* src) {
-  for (int e = threadIdx.x; e < 129 * 16; e += kLinThreads) {
-    const int n = e >> 4, c8 = e & 15;
-    *reinterpret_cast<uint4*>(dst + n * kStateLd + 8 * c8) =
-        __ldg(reinterpret_cast<const uint4*>(src + n * 128) + c8);
-  }
-}
-
-// 8 consecutive bf16 of a shared-memory state row as floats.
-__device__ __forceinline__ void state8(const uint16_t* p, float (&f)[8]) {
-  const uint4 w = *reinterpret_cast<const uint4*>(p);
-  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+  for (int u = 0; u < 8; ++u) {
+    uint32_t w[4];
 #pragma unroll
-  for (int z = 0; z < 4; ++z) {
-    f[2 * z] = bf16_bits_to_f32(ww[z] & 0xFFFFu);
-    f[2 * z + 1] = bf16_bits_to_f32(ww[z] >> 16);
+    for (int z = 0; z < 4; ++z) {
+      const float lo = x[8 * u + 2 * z] * inv, hi = x[8 * u + 2 * z + 1] * inv;
+      a32[r * 132 + 64 * kh + 8 * u + 2 * z] = lo;
+      a32[r * 132 + 64 * kh + 8 * u + 2 * z + 1] = hi;
+      w[z] = pack_bf16x2(lo, hi);
+    }
+    *reinterpret_cast<uint4*>(tile + kh * 8192 + sw128_offset(r, u)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
-// Query side of the linear branch for one query block: a = phi(q), num = a G[:, :128],
-// den = a G[:, 128], dnum = dO / den, dden = -(dO . num / den) / den, dq_l = a * (G[:, :128]
-// dnum + G[:, 128] dden), and dG = a^T [dnum | dden] as bf16 [129][128] ([n][c]).
+// This thread's 64 values of row r of a 64 x 128 K-major bf16 operand (columns 64cb + kh + 2e
+// in x[cb][e]) written after an exchange with lane ^ 2, 32 contiguous columns per chunk.
+__device__ __forceinline__ void store_row128(uint8_t* tile, int r, int kh, const float (&x)[2][32]) {
+#pragma unroll
+  for (int cb = 0; cb < 2; ++cb) {
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      float w4[4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float mine0 = x[cb][e + u], mine1 = x[cb][16 + e + u];
+        const float recv = __shfl_xor_sync(0xffffffffu, kh ? mine0 : mine1, 2);
+        w4[2 * u] = kh ? recv : mine0;
+        w4[2 * u + 1] = kh ? mine1 : recv;
+      }
+      w[e] = pack_bf16x2(w4[0], w4[1]);
+      w[e + 1] = pack_bf16x2(w4[2], w4[3]);
+    }
+    // columns 64cb + 32kh .. +31 = 16-byte chunks 4kh .. 4kh + 3 of chunk cb's row
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<uint4*>(tile + cb * 8192 + sw128_offset(r, 4 * kh + c)) =
+          make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+  }
+}
+
+constexpr int kLinThreads = 128;
+constexpr int kLinSmem = 1024 + 2 * kTile + kStateTile + 64 * 132 * 4 + 129 * 4 + 64 * 4;
+
+// Query side of the linear branch for one query block (M=64 rows = tokens in order):
+//   num = phi(Q) G[:, :128]          (tcgen05, TMEM lanes 0-15, columns [0, 128))
+//   den = phi(q) . G[:, 128], dnum = dO / den, dden = -(dO . num) / den^2
+//   da = dnum G[:, :128]^T           (lanes 16-31, columns [0, 128)) + dden G[:, 128]
+//   dq_l = phi(q) * da;   dG = phi(Q)^T [dnum | dden]   (M=128 over channels, columns [128, 256))
 __global__ void __launch_bounds__(kLinThreads, 2)
-k_bwd_lin_query(const uint16_t* __restrict__ qn, const uint16_t* __restrict__ dn,
-                const uint16_t* __restrict__ gsum, int nb, int nb_m_pad, int n_pad,
-                float* __restrict__ lin_q, uint16_t* __restrict__ dgsum) {
+k_bwd_lin_query(const __grid_constant__ CUtensorMap tm_g, const uint16_t* __restrict__ qn,
+                const uint16_t* __restrict__ dn, const uint16_t* __restrict__ gsum, int nb,
+                int nb_m_pad, int n_pad, float* __restrict__ lin_q, uint16_t* __restrict__ dgsum,
+                int* status) {
   extern __shared__ uint8_t smem_raw[];
-  uint16_t* g_s = reinterpret_cast<uint16_t*>(smem_raw);                 // [129][kStateLd]
-  float* a_s = reinterpret_cast<float*>(smem_raw + 129 * kStateLd * 2);  // [64][129]
-  float* n_s = a_s + 64 * 129;                                           // [64][129]: dnum | dden
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* a_t = smem;                               // phi(Q) bf16 [t][c]
+  uint8_t* n_t = smem + kTile;                       // dnum bf16 [t][n]
+  uint8_t* g_t = smem + 2 * kTile;                   // G rows n < 128
+  float* a32 = reinterpret_cast<float*>(smem + 2 * kTile + kStateTile);   // [64][132]
+  float* g128 = a32 + 64 * 132;                      // G[128][c]
+  float* dden_s = g128 + 129;                        // [64]
+  __shared__ uint64_t g_full, mma1, mma2;
+  __shared__ uint32_t tmem_slot;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x;
   const int64_t bh = blockIdx.y;
-  const int tid = threadIdx.x;
-  uint16_t* dg = dgsum + (bh * nb_m_pad + i) * static_cast<int64_t>(kHFlat);
-  if (i >= nb) {                       // padding rows of the transposed complement GEMM operand
-    for (int e = tid; e < kHFlat; e += kLinThreads) dg[e] = 0;
+  const int64_t grow0 = (bh * nb_m_pad + i) * 129;   // first state row of block i
+  uint16_t* dg = dgsum + grow0 * 128;
+  if (i >= nb) {   // padding rows of the transposed complement GEMM operand
+    for (int e = threadIdx.x; e < kHFlat; e += kLinThreads) dg[e] = 0;
     return;
   }
-  load_state(g_s, gsum + (bh * nb_m_pad + i) * static_cast<int64_t>(kHFlat));
-  const int t = tid >> 2, part = tid & 3;
-  const int64_t grow = bh * n_pad + 64 * static_cast<int64_t>(i) + t;
-  float a[32];
-  phi_part(qn + grow * 128, part, a);
-#pragma unroll
-  for (int e = 0; e < 32; ++e) a_s[t * 129 + 32 * part + e] = a[e];
-  __syncthreads();
-  // num for this thread's columns n = 32 part + e; den partial over its channels
-  float num[32];
-#pragma unroll
-  for (int g8 = 0; g8 < 4; ++g8) {       // eight columns at a time
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 1
-    for (int c8 = 0; c8 < 16; ++c8) {
-      float av[8];
-#pragma unroll
-      for (int z = 0; z < 8; ++z) av[z] = a_s[t * 129 + 8 * c8 + z];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float gv[8];
-        state8(g_s + (32 * part + 8 * g8 + e) * kStateLd + 8 * c8, gv);
-#pragma unroll
-        for (int z = 0; z < 8; ++z) acc[e] = fmaf(av[z], gv[z], acc[e]);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) num[8 * g8 + e] = acc[e];
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 256);
+    tmem_relinquish();
   }
+  if (threadIdx.x == 32) {
+    mbar_init(&g_full, 1); mbar_init(&mma1, 1); mbar_init(&mma2, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&g_full, kStateTile);
+    tma_load_2d(g_t, &tm_g, &g_full, 0, static_cast<int>(grow0));
+    tma_load_2d(g_t + 16384, &tm_g, &g_full, 64, static_cast<int>(grow0));
+  }
+  g128[threadIdx.x] = bf16_bits_to_f32(gsum[(grow0 + 128) * 128 + threadIdx.x]);
+  const int r = frag_row(warp, lane);
+  const int kh = (lane >> 1) & 1;
+  const int64_t trow = bh * n_pad + 64 * static_cast<int64_t>(i) + r;
+  phi_half_row(qn + trow * 128, r, kh, a_t, a32);
+  __syncthreads();                                   // g128 and a32 complete
   float den = 0.f;
-  {
-    float gv[8];
+#pragma unroll 8
+  for (int c = 64 * kh; c < 64 * kh + 64; ++c) den = fmaf(a32[r * 132 + c], g128[c], den);
+  den += __shfl_xor_sync(0xffffffffu, den, 2);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    ok = mbar_wait(&g_full, 0, status);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t aa = smem_u32(a_t), gb = smem_u32(g_t);
 #pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8) {
-      state8(g_s + 128 * kStateLd + 32 * part + 8 * c8, gv);
-#pragma unroll
-      for (int z = 0; z < 8; ++z) den = fmaf(a[8 * c8 + z], gv[z], den);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem, desc_k128(aa, kk), desc_state_kmajor(gb, kk), kIdescKK128, kk > 0 ? 1u : 0u);
+      mma_commit(&mma1);
     }
   }
-  den += __shfl_xor_sync(0xffffffffu, den, 1);
-  den += __shfl_xor_sync(0xffffffffu, den, 2);
-  // dnum, dden
-  const uint4* d4 = reinterpret_cast<const uint4*>(dn + grow * 128) + 4 * part;
-  const float inv_den = 1.f / den;
-  float dden = 0.f;
+  ok = mbar_wait(&mma1, 0, status);
+  tc_fence_after();
+  const uint32_t lane_a = static_cast<uint32_t>(32 * warp) << 16;
+  const uint32_t lane_b = static_cast<uint32_t>(32 * warp + 16) << 16;
+  float dnum[2][32];
+  float dpart = 0.f;
+  {
+    const uint4* d4 = reinterpret_cast<const uint4*>(dn + trow * 128);
+    const float inv_den = 1.f / den;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const uint4 w = __ldg(d4 + u);
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    for (int cb = 0; cb < 2; ++cb) {
+      uint32_t o[32];
+      tmem_ld16x64(tmem + lane_a + 64 * cb, o);
+      tmem_ld_wait();
 #pragma unroll
-    for (int z = 0; z < 4; ++z) {
+      for (int u = 0; u < 8; ++u) {
+        const uint4 w = __ldg(d4 + 8 * cb + u);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int e = 8 * u + 2 * z + hh;
-        const float dov = bf16_bits_to_f32(hh ? (ww[z] >> 16) : (ww[z] & 0xFFFFu));
-        dden = fmaf(dov, num[e] * inv_den, dden);
-        n_s[t * 129 + 32 * part + e] = dov * inv_den;
+        for (int z = 0; z < 4; ++z) {
+          const int e = 4 * u + z;
+          const float dov = bf16_bits_to_f32(kh ? (ww[z] >> 16) : (ww[z] & 0xFFFFu));
+          dpart = fmaf(dov, __uint_as_float(o[e]), dpart);
+          dnum[cb][e] = dov * inv_den;
+        }
       }
     }
   }
-  dden += __shfl_xor_sync(0xffffffffu, dden, 1);
-  dden += __shfl_xor_sync(0xffffffffu, dden, 2);
-  dden = -dden * inv_den;
-  if (part == 0) n_s[t * 129 + 128] = dden;
+  dpart += __shfl_xor_sync(0xffffffffu, dpart, 2);
+  const float dden = -dpart / (den * den);
+  if (kh == 0) dden_s[r] = dden;
+  store_row128(n_t, r, kh, dnum);
+  fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
-  // da for this thread's channels c = 32 part + e: sum over n of G[n][c] dnum[n] + G[128][c] dden
-  float da[32];
-  {
-    float gv[8];
+  if (threadIdx.x == 0 && ok) {
+    tc_fence_after();
+    const uint32_t nb_ = smem_u32(n_t), gb = smem_u32(g_t), aa = smem_u32(a_t);
 #pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8) {
-      state8(g_s + 128 * kStateLd + 32 * part + 8 * c8, gv);
+    for (int kk = 0; kk < 8; ++kk)   // da = dnum G^T: K = n (128)
+      mma_bf16(tmem + (16u << 16), desc_k128(nb_, kk), desc_state_mnmajor(gb, kk), kIdescKM128,
+               kk > 0 ? 1u : 0u);
 #pragma unroll
-      for (int z = 0; z < 8; ++z) da[8 * c8 + z] = gv[z] * dden;
+    for (int kk = 0; kk < 4; ++kk)   // dG = phi(Q)^T dnum: M = c, N = n, K = t (64)
+      mma_bf16(tmem + 128, desc_mn128(aa, kk), desc_mn128(nb_, kk), kIdescMM128,
+               kk > 0 ? 1u : 0u);
+    mma_commit(&mma2);
+  }
+  ok = ok && mbar_wait(&mma2, 0, status);
+  tc_fence_after();
+  if (ok) {
+    // dq_l = phi(q) * (da + dden G[:, 128])
+#pragma unroll 1
+    for (int cb = 0; cb < 2; ++cb) {
+      uint32_t o[32];
+      tmem_ld16x64(tmem + lane_b + 64 * cb, o);
+      tmem_ld_wait();
+      float g[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int c = 64 * cb + kh + 2 * e;
+        g[e] = a32[r * 132 + c] * (__uint_as_float(o[e]) + dden * g128[c]);
+      }
+      store_grad_chunk(g, cb, kh, lin_q + trow * 128, SAGESLA_F32);
     }
-  }
-  for (int n = 0; n < 128; ++n) {
-    const float dnv = n_s[t * 129 + n];
+    // dG rows n < 128: TMEM lane c = 32 warp + lane, columns 128 + n; row 128 = sum_t a dden
+    const int c = 32 * warp + lane;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t o[32];
+      tmem_ld32(tmem_addr(tmem, 32 * warp, 128 + 32 * cc), o);
+      tmem_ld_wait();
 #pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8) {
-      float gv[8];
-      state8(g_s + n * kStateLd + 32 * part + 8 * c8, gv);
-#pragma unroll
-      for (int z = 0; z < 8; ++z) da[8 * c8 + z] = fmaf(gv[z], dnv, da[8 * c8 + z]);
+      for (int e = 0; e < 32; ++e)
+        dg[(32 * cc + e) * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(o[e])));
     }
+    float s128 = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < 64; ++t) s128 = fmaf(a32[t * 132 + c], dden_s[t], s128);
+    dg[128 * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(s128));
   }
-  float4* lq = reinterpret_cast<float4*>(lin_q + grow * 128 + 32 * part);
-#pragma unroll
-  for (int u = 0; u < 8; ++u)
-    lq[u] = make_float4(a[4 * u] * da[4 * u], a[4 * u + 1] * da[4 * u + 1],
-                        a[4 * u + 2] * da[4 * u + 2], a[4 * u + 3] * da[4 * u + 3]);
-  // dG[n][c] = sum over the block's tokens of a[t][c] (dnum | dden)[t][n]; thread: channel c,
-  // rows n = nh, nh + 2, ...
-  const int c = tid & 127, nh = tid >> 7;
-  float acol[64];
-#pragma unroll
-  for (int tt = 0; tt < 64; ++tt) acol[tt] = a_s[tt * 129 + c];
-  for (int n = nh; n < 129; n += 2) {
-    float sacc = 0.f;
-#pragma unroll
-    for (int tt = 0; tt < 64; ++tt) sacc = fmaf(acol[tt], n_s[tt * 129 + n], sacc);
-    dg[n * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(sacc));
-  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
-// Key side of the linear branch for one key block: b = phi(k), db = dH[:, :128] v + dH[:, 128],
-// dk_l = b * (db - b . db), dv_l = dH[:, :128]^T b (dH as bf16 [129][128], [n][c]).
+// Key side of the linear branch for one key block (rows = tokens in order), b = phi(k):
+//   db = V dH[:, :128]^T (lanes 0-15) + dH[:, 128];  dv_l = b dH[:, :128] (lanes 16-31);
+//   dk_l = b * (db - b . db).
 __global__ void __launch_bounds__(kLinThreads, 2)
-k_bwd_lin_key(const uint16_t* __restrict__ kn, const uint16_t* __restrict__ vn,
-              const uint16_t* __restrict__ dhsum, int nb_m_pad, int n_pad,
-              float* __restrict__ lin_k, float* __restrict__ lin_v) {
+k_bwd_lin_key(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_vn,
+              const uint16_t* __restrict__ kn, const uint16_t* __restrict__ dhsum, int nb_m_pad,
+              int n_pad, float* __restrict__ lin_k, float* __restrict__ lin_v, int* status) {
   extern __shared__ uint8_t smem_raw[];
-  uint16_t* h_s = reinterpret_cast<uint16_t*>(smem_raw);                 // [129][kStateLd]
-  float* b_s = reinterpret_cast<float*>(smem_raw + 129 * kStateLd * 2);  // [64][129]
-  float* v_s = b_s + 64 * 129;                                           // [64][129]
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* b_t = smem;                               // phi(K) bf16 [t][c]
+  uint8_t* v_t = smem + kTile;                       // V bf16 [t][n]
+  uint8_t* h_t = smem + 2 * kTile;                   // dH rows n < 128
+  float* b32 = reinterpret_cast<float*>(smem + 2 * kTile + kStateTile);   // [64][132]
+  float* h128 = b32 + 64 * 132;                      // dH[128][c]
+  __shared__ uint64_t ld_full, mma1;
+  __shared__ uint32_t tmem_slot;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x;
   const int64_t bh = blockIdx.y;
-  const int tid = threadIdx.x;
-  load_state(h_s, dhsum + (bh * nb_m_pad + j) * static_cast<int64_t>(kHFlat));
-  const int t = tid >> 2, part = tid & 3;
-  const int64_t grow = bh * n_pad + 64 * static_cast<int64_t>(j) + t;
-  float b[32];
-  phi_part(kn + grow * 128, part, b);
-  const uint4* v4 = reinterpret_cast<const uint4*>(vn + grow * 128) + 4 * part;
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const uint4 w = __ldg(v4 + u);
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int z = 0; z < 4; ++z) {
-      v_s[t * 129 + 32 * part + 8 * u + 2 * z] = bf16_bits_to_f32(ww[z] & 0xFFFFu);
-      v_s[t * 129 + 32 * part + 8 * u + 2 * z + 1] = bf16_bits_to_f32(ww[z] >> 16);
-    }
+  const int64_t hrow0 = (bh * nb_m_pad + j) * 129;
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 128);
+    tmem_relinquish();
   }
-#pragma unroll
-  for (int e = 0; e < 32; ++e) b_s[t * 129 + 32 * part + e] = b[e];
+  if (threadIdx.x == 32) {
+    mbar_init(&ld_full, 1); mbar_init(&mma1, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
   __syncthreads();
-  // db for this thread's channels c = 32 part + e
-  float db[32];
-  {
-    float hv[8];
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const int64_t trow0 = bh * n_pad + 64 * static_cast<int64_t>(j);
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&ld_full, kStateTile + kTile);
+    tma_load_2d(h_t, &tm_h, &ld_full, 0, static_cast<int>(hrow0));
+    tma_load_2d(h_t + 16384, &tm_h, &ld_full, 64, static_cast<int>(hrow0));
+    tma_load_2d(v_t, &tm_vn, &ld_full, 0, static_cast<int>(trow0));
+    tma_load_2d(v_t + 8192, &tm_vn, &ld_full, 64, static_cast<int>(trow0));
+  }
+  h128[threadIdx.x] = bf16_bits_to_f32(dhsum[(hrow0 + 128) * 128 + threadIdx.x]);
+  const int r = frag_row(warp, lane);
+  const int kh = (lane >> 1) & 1;
+  const int64_t trow = trow0 + r;
+  phi_half_row(kn + trow * 128, r, kh, b_t, b32);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    ok = mbar_wait(&ld_full, 0, status);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t va = smem_u32(v_t), ba = smem_u32(b_t), hb = smem_u32(h_t);
 #pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8) {
-      state8(h_s + 128 * kStateLd + 32 * part + 8 * c8, hv);
+      for (int kk = 0; kk < 8; ++kk)   // db = V dH^T: K = n
+        mma_bf16(tmem, desc_k128(va, kk), desc_state_mnmajor(hb, kk), kIdescKM128, kk > 0 ? 1u : 0u);
 #pragma unroll
-      for (int z = 0; z < 8; ++z) db[8 * c8 + z] = hv[z];
+      for (int kk = 0; kk < 8; ++kk)   // dv = b dH: K = c
+        mma_bf16(tmem + (16u << 16), desc_k128(ba, kk), desc_state_kmajor(hb, kk), kIdescKK128,
+                 kk > 0 ? 1u : 0u);
+      mma_commit(&mma1);
     }
   }
-  for (int n = 0; n < 128; ++n) {
-    const float vv = v_s[t * 129 + n];
+  ok = mbar_wait(&mma1, 0, status);
+  tc_fence_after();
+  if (ok) {
+    const uint32_t lane_a = static_cast<uint32_t>(32 * warp) << 16;
+    const uint32_t lane_b = static_cast<uint32_t>(32 * warp + 16) << 16;
+    float db[2][32];
+    float proj = 0.f;
 #pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8) {
-      float hv[8];
-      state8(h_s + n * kStateLd + 32 * part + 8 * c8, hv);
+    for (int cb = 0; cb < 2; ++cb) {
+      uint32_t o[32];
+      tmem_ld16x64(tmem + lane_a + 64 * cb, o);
+      tmem_ld_wait();
 #pragma unroll
-      for (int z = 0; z < 8; ++z) db[8 * c8 + z] = fmaf(hv[z], vv, db[8 * c8 + z]);
-    }
-  }
-  float proj = 0.f;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) proj = fmaf(b[e], db[e], proj);
-  proj += __shfl_xor_sync(0xffffffffu, proj, 1);
-  proj += __shfl_xor_sync(0xffffffffu, proj, 2);
-  float4* lk = reinterpret_cast<float4*>(lin_k + grow * 128 + 32 * part);
-#pragma unroll
-  for (int u = 0; u < 8; ++u)
-    lk[u] = make_float4(b[4 * u] * (db[4 * u] - proj), b[4 * u + 1] * (db[4 * u + 1] - proj),
-                        b[4 * u + 2] * (db[4 * u + 2] - proj), b[4 * u + 3] * (db[4 * u + 3] - proj));
-  // dv for this thread's columns n = 32 part + e: sum over c of b[c] dH[n][c]
-  float4* lv = reinterpret_cast<float4*>(lin_v + grow * 128 + 32 * part);
-#pragma unroll
-  for (int g8 = 0; g8 < 4; ++g8) {       // eight columns at a time
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 1
-    for (int c8 = 0; c8 < 16; ++c8) {
-      float bv[8];
-#pragma unroll
-      for (int z = 0; z < 8; ++z) bv[z] = b_s[t * 129 + 8 * c8 + z];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float hv[8];
-        state8(h_s + (32 * part + 8 * g8 + e) * kStateLd + 8 * c8, hv);
-#pragma unroll
-        for (int z = 0; z < 8; ++z) acc[e] = fmaf(bv[z], hv[z], acc[e]);
+      for (int e = 0; e < 32; ++e) {
+        const int c = 64 * cb + kh + 2 * e;
+        db[cb][e] = __uint_as_float(o[e]) + h128[c];
+        proj = fmaf(b32[r * 132 + c], db[cb][e], proj);
       }
     }
-    lv[2 * g8] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    lv[2 * g8 + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    proj += __shfl_xor_sync(0xffffffffu, proj, 2);
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) {
+      float g[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int c = 64 * cb + kh + 2 * e;
+        g[e] = b32[r * 132 + c] * (db[cb][e] - proj);
+      }
+      store_grad_chunk(g, cb, kh, lin_k + trow * 128, SAGESLA_F32);
+    }
+#pragma unroll 1
+    for (int cb = 0; cb < 2; ++cb) {
+      uint32_t o[32];
+      tmem_ld16x64(tmem + lane_b + 64 * cb, o);
+      tmem_ld_wait();
+      float g[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) g[e] = __uint_as_float(o[e]);
+      store_grad_chunk(g, cb, kh, lin_v + trow * 128, SAGESLA_F32);
+    }
   }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 }  // namespace
@@ -1106,11 +1190,22 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
   k_bwd_lse<<<grid, kBwdThreads, smem_lse, stream>>>(tq, tk, tv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (!p.linear_empty) {
+    CUtensorMap tg, th, tvn;
+    if (!encode_tmap_2d(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128,
+                        static_cast<uint64_t>(p.BH * p.nb_m_pad * 129), 256, ws + L.gsum, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d(&th, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128,
+                        static_cast<uint64_t>(p.BH * p.nb_m_pad * 129), 256, ws + bl.dh, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d(&tvn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128, static_cast<uint64_t>(rows),
+                        256, ws + bl.vn, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
     const dim3 gq(static_cast<unsigned>(p.nb_m_pad), static_cast<unsigned>(p.BH));
     k_bwd_lin_query<<<gq, kLinThreads, kLinSmem, stream>>>(
-        prm.qn, prm.dn, reinterpret_cast<const uint16_t*>(ws + L.gsum), static_cast<int>(p.nb),
+        tg, prm.qn, prm.dn, reinterpret_cast<const uint16_t*>(ws + L.gsum), static_cast<int>(p.nb),
         static_cast<int>(p.nb_m_pad), static_cast<int>(p.n_pad),
-        reinterpret_cast<float*>(ws + bl.lin_q), reinterpret_cast<uint16_t*>(ws + bl.dg));
+        reinterpret_cast<float*>(ws + bl.lin_q), reinterpret_cast<uint16_t*>(ws + bl.dg),
+        prm.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 gt(static_cast<unsigned>(p.nb_m_pad / 32), static_cast<unsigned>(p.nb_m_pad / 32),
                   static_cast<unsigned>(p.BH));
@@ -1124,10 +1219,10 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
       return e;
     const dim3 gk(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.BH));
     k_bwd_lin_key<<<gk, kLinThreads, kLinSmem, stream>>>(
-        reinterpret_cast<const uint16_t*>(ws + bl.kn), reinterpret_cast<const uint16_t*>(ws + bl.vn),
+        th, tvn, reinterpret_cast<const uint16_t*>(ws + bl.kn),
         reinterpret_cast<const uint16_t*>(ws + bl.dh), static_cast<int>(p.nb_m_pad),
         static_cast<int>(p.n_pad), reinterpret_cast<float*>(ws + bl.lin_k),
-        reinterpret_cast<float*>(ws + bl.lin_v));
+        reinterpret_cast<float*>(ws + bl.lin_v), prm.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   k_bwd_dq<<<grid, kBwdThreads, smem_dq, stream>>>(tq, tk, tv, td, prm);

@@ -221,7 +221,9 @@ constexpr int kBwdThreads = 128;
 
 // Online-softmax pass of one query block over its kept key blocks (bf16 MMAs): writes the
 // base-2 log-sum-exp L of the scaled scores and D = rowsum(dO * O_s) of its 64 rows.
-// TMEM: S [0, 64) and O [64, 192).
+// TMEM: two S buffers [0, 64) and [64, 128), O [128, 256). S of block n + 1 is issued (by
+// thread 0) as soon as S of block n is in registers, so that it runs under the softmax of
+// block n; P.V is issued by warp 1.
 __global__ void __launch_bounds__(kBwdThreads, 2)
 k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_v, BwdParams prm) {
@@ -231,7 +233,7 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   uint8_t* k_t = smem + kTile;           // 2 K stages
   uint8_t* v_t = smem + 3 * kTile;       // 2 V stages
   uint8_t* p_t = smem + 5 * kTile;       // P tile
-  __shared__ uint64_t q_full, k_full[2], v_full[2], s_done, pv_done;
+  __shared__ uint64_t q_full, k_full[2], v_full[2], s_done[2], pv_done;
   __shared__ uint32_t tmem_slot;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -246,8 +248,9 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   }
   if (threadIdx.x == 32) {
     mbar_init(&q_full, 1);
-    for (int s = 0; s < 2; ++s) { mbar_init(&k_full[s], 1); mbar_init(&v_full[s], 1); }
-    mbar_init(&s_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1); mbar_init(&v_full[s], 1); mbar_init(&s_done[s], 1);
+    }
     mbar_init(&pv_done, 1);
     fence_mbar_init();
   }
@@ -255,6 +258,8 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  const uint32_t qa = smem_u32(q_t);
+  bool ok = true;
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
     mbar_arrive_expect_tx(&q_full, kTile);
@@ -264,40 +269,48 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     load_tile(k_t, &tm_k, &k_full[0], blk0 + j0);
     mbar_arrive_expect_tx(&v_full[0], kTile);
     load_tile(v_t, &tm_v, &v_full[0], blk0 + j0);
+    if (U > 1) {
+      mbar_arrive_expect_tx(&k_full[1], kTile);
+      load_tile(k_t + kTile, &tm_k, &k_full[1], blk0 + __ldg(klist + 1));
+    }
+    ok = mbar_wait(&q_full, 0, prm.status) && mbar_wait(&k_full[0], 0, prm.status);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem, desc_k128(qa, kk), desc_k128(smem_u32(k_t), kk), kIdescKK64, kk > 0 ? 1u : 0u);
+      mma_commit(&s_done[0]);
+    }
   }
   const int row = frag_row(warp, lane);
   const int kh = (lane >> 1) & 1;
   const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
   const float c2 = kScale * kLog2e;
   float m_run = -INFINITY, l_part = 0.f;
-  bool ok = true;
-  int j_next = __ldg(klist);
   for (int n = 0; n < U && ok; ++n) {
-    const int j = j_next;
-    if (n + 1 < U) j_next = __ldg(klist + n + 1);
+    const int j = __ldg(klist + n);
     const int st = n & 1;
-    if (threadIdx.x == 0) {
-      ok = (n > 0 || mbar_wait(&q_full, 0, prm.status)) &&
-           mbar_wait(&k_full[st], (n >> 1) & 1, prm.status);
-      if (ok) {
-        tc_fence_after();
-        const uint32_t qa = smem_u32(q_t), kb = smem_u32(k_t + st * kTile);
+    if (!mbar_wait(&s_done[st], (n >> 1) & 1, prm.status)) { ok = false; break; }
+    tc_fence_after();
+    uint32_t sr[32];
+    tmem_ld16x64(tmem + lane_s + 64 * st, sr);
+    tmem_ld_wait();
+    if (threadIdx.x == 0 && n + 1 < U) {
+      // S(n+1) into the other buffer (read by every thread before the last barrier), and K of
+      // block n+2 into the stage S(n) has finished reading
+      if (mbar_wait(&k_full[st ^ 1], ((n + 1) >> 1) & 1, prm.status)) {
+        const uint32_t kb = smem_u32(k_t + (st ^ 1) * kTile);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem, desc_k128(qa, kk), desc_k128(kb, kk), kIdescKK64, kk > 0 ? 1u : 0u);
-        mma_commit(&s_done);
+          mma_bf16(tmem + 64 * (st ^ 1), desc_k128(qa, kk), desc_k128(kb, kk), kIdescKK64,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(&s_done[st ^ 1]);
+      }
+      if (n + 2 < U) {
+        mbar_arrive_expect_tx(&k_full[st], kTile);
+        load_tile(k_t + st * kTile, &tm_k, &k_full[st], blk0 + __ldg(klist + n + 2));
       }
     }
-    if (!mbar_wait(&s_done, n & 1, prm.status)) { ok = false; break; }
-    tc_fence_after();
-    // K of the next kept block into the other stage (its previous K was read by S(n-1))
-    if (threadIdx.x == 0 && n + 1 < U) {
-      mbar_arrive_expect_tx(&k_full[st ^ 1], kTile);
-      load_tile(k_t + (st ^ 1) * kTile, &tm_k, &k_full[st ^ 1], blk0 + j_next);
-    }
-    uint32_t sr[32];
-    tmem_ld16x64(tmem + lane_s, sr);
-    tmem_ld_wait();
     const int valid = (j == prm.nb - 1) ? prm.n_last - 32 * kh : 32;   // real keys of this thread
     float x[32], mx = -INFINITY;
 #pragma unroll
@@ -318,17 +331,17 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     tc_fence_after();
     if (threadIdx.x == 0 && n + 1 < U) {
       mbar_arrive_expect_tx(&v_full[st ^ 1], kTile);
-      load_tile(v_t + (st ^ 1) * kTile, &tm_v, &v_full[st ^ 1], blk0 + j_next);
+      load_tile(v_t + (st ^ 1) * kTile, &tm_v, &v_full[st ^ 1], blk0 + __ldg(klist + n + 1));
     }
     if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
-        tmem_ld16x64(tmem + lane_s + 64 + 64 * cc, o);
+        tmem_ld16x64(tmem + lane_s + 128 + 64 * cc, o);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-        tmem_st16x64(tmem + lane_s + 64 + 64 * cc, o);
+        tmem_st16x64(tmem + lane_s + 128 + 64 * cc, o);
       }
       tmem_st_wait();
     }
@@ -336,13 +349,13 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 32) {
       tc_fence_after();
       if (mbar_wait(&v_full[st], (n >> 1) & 1, prm.status)) {
         const uint32_t pa = smem_u32(p_t), vb = smem_u32(v_t + st * kTile);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 64, desc_k64(pa, kk), desc_mn128(vb, kk), kIdescKM128,
+          mma_bf16(tmem + 128, desc_k64(pa, kk), desc_mn128(vb, kk), kIdescKM128,
                    (n > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&pv_done);
       }
@@ -360,7 +373,7 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 #pragma unroll 1
     for (int cc = 0; cc < 2; ++cc) {
       uint32_t o[32];
-      tmem_ld16x64(tmem + lane_s + 64 + 64 * cc, o);
+      tmem_ld16x64(tmem + lane_s + 128 + 64 * cc, o);
       tmem_ld_wait();
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -450,7 +463,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   if (threadIdx.x == 32) {
     mbar_init(&q_full, 1);
     for (int s = 0; s < 2; ++s) mbar_init(&kv_full[s], 1);
-    mbar_init(&s_done, 1);
+    mbar_init(&s_done, 2);               // S from warp 0, dP from warp 1
     mbar_init(&dq_done, 1);
     fence_mbar_init();
   }
@@ -481,20 +494,18 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   for (int n = 0; n < U && ok; ++n) {
     const int st = n & 1;
     if (n + 1 < U) j_next = __ldg(klist + n + 1);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 || threadIdx.x == 32) {   // S (warp 0) and dP (warp 1) in parallel
       ok = (n > 0 || mbar_wait(&q_full, 0, prm.status)) &&
            mbar_wait(&kv_full[st], (n >> 1) & 1, prm.status);
       if (ok) {
         tc_fence_after();
-        const uint32_t qa = smem_u32(q_t), oa = smem_u32(o_t);
-        const uint32_t kb = smem_u32(k_t + st * kTile), vb = smem_u32(v_t + st * kTile);
+        const bool is_s = threadIdx.x == 0;
+        const uint32_t a = smem_u32(is_s ? q_t : o_t);
+        const uint32_t b = smem_u32((is_s ? k_t : v_t) + st * kTile);
+        const uint32_t d = is_s ? tmem : tmem + (16u << 16);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem, desc_k128(qa, kk), desc_k128(kb, kk), kIdescKK64, kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + (16u << 16), desc_k128(oa, kk), desc_k128(vb, kk), kIdescKK64,
-                   kk > 0 ? 1u : 0u);
+          mma_bf16(d, desc_k128(a, kk), desc_k128(b, kk), kIdescKK64, kk > 0 ? 1u : 0u);
         mma_commit(&s_done);
       }
     }
@@ -522,7 +533,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 64) {
       tc_fence_after();
       const uint32_t sa = smem_u32(s_t), kb = smem_u32(k_t + st * kTile);
 #pragma unroll
@@ -589,8 +600,8 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   if (threadIdx.x == 32) {
     mbar_init(&kv_full, 1);
     mbar_init(&qo_full, 1);
-    mbar_init(&s_done, 1);
-    mbar_init(&acc_done, 1);
+    mbar_init(&s_done, 2);               // S^T from warp 0, dP^T from warp 1
+    mbar_init(&acc_done, 2);             // dV from warp 2, dK from warp 3
     fence_mbar_init();
   }
   tc_fence_before();
@@ -617,20 +628,17 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   bool ok = true;
   for (int t = 0; t < T && ok; ++t) {
     const int i = __ldg(ilist + t);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 || threadIdx.x == 32) {   // S^T (warp 0) and dP^T (warp 1)
       ok = (t > 0 || mbar_wait(&kv_full, 0, prm.status)) &&
            mbar_wait(&qo_full, t & 1, prm.status);
       if (ok) {
         tc_fence_after();
-        const uint32_t ka = smem_u32(k_t), va = smem_u32(v_t);
-        const uint32_t qb = smem_u32(q_t), ob = smem_u32(o_t);
+        const bool is_s = threadIdx.x == 0;
+        const uint32_t a = smem_u32(is_s ? k_t : v_t), b = smem_u32(is_s ? q_t : o_t);
+        const uint32_t d = is_s ? tmem : tmem + (16u << 16);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem, desc_k128(ka, kk), desc_k128(qb, kk), kIdescKK64, kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + (16u << 16), desc_k128(va, kk), desc_k128(ob, kk), kIdescKK64,
-                   kk > 0 ? 1u : 0u);
+          mma_bf16(d, desc_k128(a, kk), desc_k128(b, kk), kIdescKK64, kk > 0 ? 1u : 0u);
         mma_commit(&s_done);
       }
     }
@@ -663,26 +671,22 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 64 || threadIdx.x == 96) {  // dV (warp 2) and dK (warp 3)
       tc_fence_after();
-      const uint32_t pa = smem_u32(p_t), sa = smem_u32(s_t);
-      const uint32_t qb = smem_u32(q_t), ob = smem_u32(o_t);
+      const bool is_v = threadIdx.x == 64;
+      const uint32_t a = smem_u32(is_v ? p_t : s_t), b = smem_u32(is_v ? o_t : q_t);
+      const uint32_t d = is_v ? tmem + 64 : tmem + (16u << 16) + 64;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 64, desc_k64(pa, kk), desc_mn128(ob, kk), kIdescKM128,
-                 (t > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + (16u << 16) + 64, desc_k64(sa, kk), desc_mn128(qb, kk), kIdescKM128,
-                 (t > 0 || kk > 0) ? 1u : 0u);
+        mma_bf16(d, desc_k64(a, kk), desc_mn128(b, kk), kIdescKM128, (t > 0 || kk > 0) ? 1u : 0u);
       mma_commit(&acc_done);
+    }
+    if (threadIdx.x == 0 && t + 1 < T && mbar_wait(&acc_done, t & 1, prm.status)) {
       // next query block's Q and dO once these MMAs have read the tiles
-      if (t + 1 < T && mbar_wait(&acc_done, t & 1, prm.status)) {
-        const int i1 = __ldg(ilist + t + 1);
-        mbar_arrive_expect_tx(&qo_full, 2 * kTile);
-        load_tile(q_t, &tm_q, &qo_full, blk0 + i1);
-        load_tile(o_t, &tm_do, &qo_full, blk0 + i1);
-      }
+      const int i1 = __ldg(ilist + t + 1);
+      mbar_arrive_expect_tx(&qo_full, 2 * kTile);
+      load_tile(q_t, &tm_q, &qo_full, blk0 + i1);
+      load_tile(o_t, &tm_do, &qo_full, blk0 + i1);
     }
   }
   if (ok && T > 0) ok = mbar_wait(&acc_done, (T - 1) & 1, prm.status);

@@ -17,8 +17,10 @@ bounded sample of the same workload per step, extrapolated to the whole forward.
 
 --sweep (one GPU) prints one JSON line per point instead: the forward on the 14B-720P random
 workload and on the smoothed-field locality workload over Top-K ratios 0.05-0.2 and the dense
-mode (ratio 1: every block kept, selection and linear branch skipped), and a dense BF16
-attention of the same shape through torch's scaled_dot_product_attention for comparison.
+mode (ratio 1: every block kept, selection and linear branch skipped), a dense BF16
+attention of the same shape through torch's scaled_dot_product_attention for comparison, the
+SLA backward (ratio 0.1, bf16 gradients) against torch's dense attention backward, and the
+fused-norm and W8A8 kernels on the same token rows.
 """
 from __future__ import annotations
 

@@ -287,15 +287,22 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
   const float c2 = kScale * kLog2e;
   float m_run = -INFINITY, l_part = 0.f;
+  ok = __syncthreads_and(ok);   // thread 0's waits above decide for every thread
   for (int n = 0; n < U && ok; ++n) {
     const int j = __ldg(klist + n);
     const int st = n & 1;
-    if (!mbar_wait(&s_done[st], (n >> 1) & 1, prm.status)) { ok = false; break; }
+    // a failed wait only clears ok: every thread leaves the loop together after its barrier
+    ok = mbar_wait(&s_done[st], (n >> 1) & 1, prm.status);
     tc_fence_after();
     uint32_t sr[32];
-    tmem_ld16x64(tmem + lane_s + 64 * st, sr);
-    tmem_ld_wait();
-    if (threadIdx.x == 0 && n + 1 < U) {
+    if (ok) {
+      tmem_ld16x64(tmem + lane_s + 64 * st, sr);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sr[e] = 0u;
+    }
+    if (ok && threadIdx.x == 0 && n + 1 < U) {
       // S(n+1) into the other buffer (read by every thread before the last barrier), and K of
       // block n+2 into the stage S(n) has finished reading
       if (mbar_wait(&k_full[st ^ 1], ((n + 1) >> 1) & 1, prm.status)) {
@@ -327,13 +334,13 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     l_part = alpha * l_part + rs;
     m_run = m_new;
     // P.V(n-1) done: frees the P tile and the V stage of block n+1, and O is stable
-    if (n > 0 && !mbar_wait(&pv_done, (n - 1) & 1, prm.status)) { ok = false; break; }
+    ok = ok && (n == 0 || mbar_wait(&pv_done, (n - 1) & 1, prm.status));
     tc_fence_after();
-    if (threadIdx.x == 0 && n + 1 < U) {
+    if (ok && threadIdx.x == 0 && n + 1 < U) {
       mbar_arrive_expect_tx(&v_full[st ^ 1], kTile);
       load_tile(v_t + (st ^ 1) * kTile, &tm_v, &v_full[st ^ 1], blk0 + __ldg(klist + n + 1));
     }
-    if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+    if (n > 0 && __any_sync(0xffffffffu, ok && alpha != 1.f)) {
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
@@ -348,7 +355,8 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     store_row_operand(p_t, row, kh, x);
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
     if (threadIdx.x == 32) {
       tc_fence_after();
       if (mbar_wait(&v_full[st], (n >> 1) & 1, prm.status)) {
@@ -491,10 +499,10 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   const float c2 = kScale * kLog2e;
   bool ok = true;
   int j_next = __ldg(klist);
-  for (int n = 0; n < U && ok; ++n) {
+  for (int n = 0; n < U; ++n) {
     const int st = n & 1;
     if (n + 1 < U) j_next = __ldg(klist + n + 1);
-    if (threadIdx.x == 0 || threadIdx.x == 32) {   // S (warp 0) and dP (warp 1) in parallel
+    if (ok && (threadIdx.x == 0 || threadIdx.x == 32)) {   // S (warp 0) and dP (warp 1)
       ok = (n > 0 || mbar_wait(&q_full, 0, prm.status)) &&
            mbar_wait(&kv_full[st], (n >> 1) & 1, prm.status);
       if (ok) {
@@ -509,22 +517,28 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         mma_commit(&s_done);
       }
     }
-    if (!mbar_wait(&s_done, n & 1, prm.status)) { ok = false; break; }
+    // a failed wait only clears ok: every thread leaves the loop together after its barrier
+    ok = ok && mbar_wait(&s_done, n & 1, prm.status);
     tc_fence_after();
-    uint32_t sr[32], pr[32];
-    tmem_ld16x64(tmem + lane_s, sr);
-    tmem_ld16x64(tmem + lane_p, pr);
-    tmem_ld_wait();
     float ds[32];
+    if (ok) {
+      uint32_t sr[32], pr[32];
+      tmem_ld16x64(tmem + lane_s, sr);
+      tmem_ld16x64(tmem + lane_p, pr);
+      tmem_ld_wait();
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
-      ds[e] = p * (__uint_as_float(pr[e]) - dterm);
+      for (int e = 0; e < 32; ++e) {
+        const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
+        ds[e] = p * (__uint_as_float(pr[e]) - dterm);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ds[e] = 0.f;
     }
     // dQ(n-1) has read the dS tile and the K / V stage of block n+1
-    if (n > 0 && !mbar_wait(&dq_done, (n - 1) & 1, prm.status)) { ok = false; break; }
+    ok = ok && (n == 0 || mbar_wait(&dq_done, (n - 1) & 1, prm.status));
     tc_fence_after();
-    if (threadIdx.x == 0 && n + 1 < U) {
+    if (ok && threadIdx.x == 0 && n + 1 < U) {
       mbar_arrive_expect_tx(&kv_full[st ^ 1], 2 * kTile);
       load_tile(k_t + (st ^ 1) * kTile, &tm_k, &kv_full[st ^ 1], blk0 + j_next);
       load_tile(v_t + (st ^ 1) * kTile, &tm_v, &kv_full[st ^ 1], blk0 + j_next);
@@ -532,7 +546,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     store_row_operand(s_t, row, kh, ds);
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
     if (threadIdx.x == 64) {
       tc_fence_after();
       const uint32_t sa = smem_u32(s_t), kb = smem_u32(k_t + st * kTile);
@@ -571,7 +586,9 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
 // dK, dV of one key block over the query blocks that keep it: S^T = K Q^T and dP^T = V dO^T
 // (lanes 0-15 / 16-31, columns [0, 64)), P^T = 2^(S^T c - L), dS^T = P^T (dP^T - D),
 // dV += P^T dO (lanes 0-15) and dK += dS^T Q (lanes 16-31), columns [64, 192). The
-// linear-branch dk, dv are added before the stores.
+// linear-branch dk, dv are added before the stores. A failed (timed-out) wait only clears a
+// thread's ok flag; the flags are ANDed at the loop's barrier, so every thread leaves the loop
+// at the same iteration.
 __global__ void __launch_bounds__(kBwdThreads, 2)
 k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -626,9 +643,9 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   const uint32_t lane_p = static_cast<uint32_t>(32 * warp + 16) << 16;
   const float c2 = kScale * kLog2e;
   bool ok = true;
-  for (int t = 0; t < T && ok; ++t) {
+  for (int t = 0; t < T; ++t) {
     const int i = __ldg(ilist + t);
-    if (threadIdx.x == 0 || threadIdx.x == 32) {   // S^T (warp 0) and dP^T (warp 1)
+    if (ok && (threadIdx.x == 0 || threadIdx.x == 32)) {   // S^T (warp 0) and dP^T (warp 1)
       ok = (t > 0 || mbar_wait(&kv_full, 0, prm.status)) &&
            mbar_wait(&qo_full, t & 1, prm.status);
       if (ok) {
@@ -652,25 +669,32 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       lq[4 * u] = a.x; lq[4 * u + 1] = a.y; lq[4 * u + 2] = a.z; lq[4 * u + 3] = a.w;
       dq_[4 * u] = b.x; dq_[4 * u + 1] = b.y; dq_[4 * u + 2] = b.z; dq_[4 * u + 3] = b.w;
     }
-    if (!mbar_wait(&s_done, t & 1, prm.status)) { ok = false; break; }
+    // a failed wait only clears ok: every thread leaves the loop together after its barrier
+    ok = ok && mbar_wait(&s_done, t & 1, prm.status);
     tc_fence_after();
-    uint32_t sr[32], pr[32];
-    tmem_ld16x64(tmem + lane_s, sr);
-    tmem_ld16x64(tmem + lane_p, pr);
-    tmem_ld_wait();
     float pt[32], ds[32];
+    if (ok) {
+      uint32_t sr[32], pr[32];
+      tmem_ld16x64(tmem + lane_s, sr);
+      tmem_ld16x64(tmem + lane_p, pr);
+      tmem_ld_wait();
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      pt[e] = exp2f(__uint_as_float(sr[e]) * c2 - lq[e]);
-      ds[e] = pt[e] * (__uint_as_float(pr[e]) - dq_[e]);
+      for (int e = 0; e < 32; ++e) {
+        pt[e] = exp2f(__uint_as_float(sr[e]) * c2 - lq[e]);
+        ds[e] = pt[e] * (__uint_as_float(pr[e]) - dq_[e]);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) { pt[e] = 0.f; ds[e] = 0.f; }
     }
     // the previous dV / dK MMAs have read the P^T and dS^T tiles and the Q / dO tiles
-    if (t > 0 && !mbar_wait(&acc_done, (t - 1) & 1, prm.status)) { ok = false; break; }
+    ok = ok && (t == 0 || mbar_wait(&acc_done, (t - 1) & 1, prm.status));
     store_row_operand(p_t, row, kh, pt);
     store_row_operand(s_t, row, kh, ds);
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
     if (threadIdx.x == 64 || threadIdx.x == 96) {  // dV (warp 2) and dK (warp 3)
       tc_fence_after();
       const bool is_v = threadIdx.x == 64;

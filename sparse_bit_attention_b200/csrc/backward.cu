@@ -25,7 +25,8 @@
 //   k_bwd_lse     per query block: the sparse forward again (online softmax), giving the
 //                 base-2 log-sum-exp L and D = rowsum(dO * O_s)
 //   k_bwd_dq      per query block over its kept blocks: S, dP, dS, dQ; adds the linear dq
-//   k_bwd_dkv     per key block over the query blocks that keep it: S^T, dP^T, dV, dK; adds
+//   k_bwd_dkv     per key block over the query blocks that keep it (compressed per-head lists
+//                 built from the kept bitmask): S^T, dP^T, dV, dK; adds
 //                 the linear dk, dv
 // The linear branch runs on the CUDA cores (k_bwd_lin_query, k_bwd_lin_key) around one
 // complement GEMM on the tensor cores (dH = (1 - M)^T dG, the forward's GEMM on the
@@ -121,17 +122,77 @@ __global__ void k_bwd_pack(TensorArg q, TensorArg k, TensorArg v, TensorArg d_ou
   qp[idx] = a; kp[idx] = b; vp[idx] = c; dp[idx] = d;
 }
 
-// For key block j: the query blocks i whose kept list holds j, ascending (one warp per
-// (head, j), reading the kept bitmask column j).
-__global__ void k_bwd_lists(int nb, int mask_words, int64_t BH, const uint32_t* __restrict__ mask,
-                            int32_t* __restrict__ tcount, int32_t* __restrict__ tlist) {
+// Query blocks that keep each key block, as one compressed list per head: tcount[head][j]
+// query blocks keep key block j; their indices, ascending, are tlist[head][toff[head][j] ..],
+// nb * k entries per head in all. Three passes: counts (one warp per (head, j) reading the kept
+// bitmask column j), an exclusive scan per head, and the fill.
+__global__ void k_bwd_list_count(int nb, int mask_words, int64_t BH, const uint32_t* __restrict__ mask,
+                                 int32_t* __restrict__ tcount) {
   const int lane = threadIdx.x & 31;
   const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
   if (w >= BH * nb) return;
   const int64_t bh = w / nb;
   const int j = static_cast<int>(w - bh * nb);
   const uint32_t* mcol = mask + bh * nb * static_cast<int64_t>(mask_words) + (j >> 5);
-  int32_t* out = tlist + (bh * nb + j) * static_cast<int64_t>(nb);
+  int count = 0;
+  for (int i0 = 0; i0 < nb; i0 += 32) {
+    const int i = i0 + lane;
+    const bool kept = i < nb && ((__ldg(mcol + static_cast<int64_t>(i) * mask_words) >> (j & 31)) & 1u);
+    count += __popc(__ballot_sync(0xffffffffu, kept));
+  }
+  if (lane == 0) tcount[bh * nb + j] = count;
+}
+
+// toff[head][j] = sum of tcount[head][0 .. j-1] (one 1024-thread CTA per head).
+__global__ void __launch_bounds__(1024) k_bwd_list_scan(int nb, const int32_t* __restrict__ tcount,
+                                                        int32_t* __restrict__ toff) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int64_t bh = blockIdx.x;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int32_t* cnt = tcount + bh * nb;
+  int32_t* off = toff + bh * (nb + 1);
+  if (t == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < nb; base += 1024) {
+    const int v = base + t < nb ? cnt[base + t] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int s = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      warp_sums[lane] = s;                       // inclusive scan of the warp totals
+    }
+    __syncthreads();
+    const int excl = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+    if (base + t < nb) off[base + t] = excl;
+    __syncthreads();
+    if (t == 0) carry += warp_sums[31];
+    __syncthreads();
+  }
+  if (t == 0) off[nb] = carry;
+}
+
+__global__ void k_bwd_list_fill(int nb, int k, int mask_words, int64_t BH,
+                                const uint32_t* __restrict__ mask, const int32_t* __restrict__ toff,
+                                int32_t* __restrict__ tlist) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  if (w >= BH * nb) return;
+  const int64_t bh = w / nb;
+  const int j = static_cast<int>(w - bh * nb);
+  const uint32_t* mcol = mask + bh * nb * static_cast<int64_t>(mask_words) + (j >> 5);
+  int32_t* out = tlist + bh * nb * static_cast<int64_t>(k) + toff[bh * (nb + 1) + j];
   int count = 0;
   for (int i0 = 0; i0 < nb; i0 += 32) {
     const int i = i0 + lane;
@@ -140,7 +201,6 @@ __global__ void k_bwd_lists(int nb, int mask_words, int64_t BH, const uint32_t* 
     if (kept) out[count + __popc(bits & ((1u << lane) - 1u))] = i;
     count += __popc(bits);
   }
-  if (lane == 0) tcount[bh * nb + j] = count;
 }
 
 // amask [head][nb_m_pad][nb_k_pad] (1 where the key block is not kept) -> its transpose,
@@ -202,7 +262,8 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
 struct BwdParams {
   const int32_t* kept;     // [BH][nb][k]
   const int32_t* tcount;   // [BH][nb]
-  const int32_t* tlist;    // [BH][nb][nb]
+  const int32_t* toff;     // [BH][nb + 1]
+  const int32_t* tlist;    // [BH][nb * k], compressed per head
   const uint16_t* qn;      // packed bf16 rows [BH][n_pad][128]
   const uint16_t* dn;      // packed dO
   float* lse;              // [BH][n_pad], base-2 log-sum-exp of the scaled scores
@@ -235,6 +296,7 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   uint8_t* p_t = smem + 5 * kTile;       // P tile
   __shared__ uint64_t q_full, k_full[2], v_full[2], s_done[2], pv_done;
   __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;   // set by any thread whose wait timed out
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x;
@@ -252,6 +314,7 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       mbar_init(&k_full[s], 1); mbar_init(&v_full[s], 1); mbar_init(&s_done[s], 1);
     }
     mbar_init(&pv_done, 1);
+    abort_flag = 0;
     fence_mbar_init();
   }
   tc_fence_before();
@@ -287,7 +350,9 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
   const float c2 = kScale * kLog2e;
   float m_run = -INFINITY, l_part = 0.f;
-  ok = __syncthreads_and(ok);   // thread 0's waits above decide for every thread
+  if (!ok) abort_flag = 1;       // thread 0's waits above decide for every thread
+  __syncthreads();
+  ok = !abort_flag;
   for (int n = 0; n < U && ok; ++n) {
     const int j = __ldg(klist + n);
     const int st = n & 1;
@@ -295,13 +360,8 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     ok = mbar_wait(&s_done[st], (n >> 1) & 1, prm.status);
     tc_fence_after();
     uint32_t sr[32];
-    if (ok) {
-      tmem_ld16x64(tmem + lane_s + 64 * st, sr);
-      tmem_ld_wait();
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) sr[e] = 0u;
-    }
+    tmem_ld16x64(tmem + lane_s + 64 * st, sr);
+    tmem_ld_wait();
     if (ok && threadIdx.x == 0 && n + 1 < U) {
       // S(n+1) into the other buffer (read by every thread before the last barrier), and K of
       // block n+2 into the stage S(n) has finished reading
@@ -340,7 +400,7 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       mbar_arrive_expect_tx(&v_full[st ^ 1], kTile);
       load_tile(v_t + (st ^ 1) * kTile, &tm_v, &v_full[st ^ 1], blk0 + __ldg(klist + n + 1));
     }
-    if (n > 0 && __any_sync(0xffffffffu, ok && alpha != 1.f)) {
+    if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
@@ -355,8 +415,9 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     store_row_operand(p_t, row, kh, x);
     fence_proxy_async_smem();
     tc_fence_before();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
+    if (!ok) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) { ok = false; break; }
     if (threadIdx.x == 32) {
       tc_fence_after();
       if (mbar_wait(&v_full[st], (n >> 1) & 1, prm.status)) {
@@ -457,6 +518,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   uint8_t* s_t = smem + 6 * kTile;       // dS tile
   __shared__ uint64_t q_full, kv_full[2], s_done, dq_done;
   __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;   // set by any thread whose wait timed out
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x;
@@ -473,6 +535,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     for (int s = 0; s < 2; ++s) mbar_init(&kv_full[s], 1);
     mbar_init(&s_done, 2);               // S from warp 0, dP from warp 1
     mbar_init(&dq_done, 1);
+    abort_flag = 0;
     fence_mbar_init();
   }
   tc_fence_before();
@@ -520,20 +583,15 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     // a failed wait only clears ok: every thread leaves the loop together after its barrier
     ok = ok && mbar_wait(&s_done, n & 1, prm.status);
     tc_fence_after();
+    uint32_t sr[32], pr[32];
+    tmem_ld16x64(tmem + lane_s, sr);
+    tmem_ld16x64(tmem + lane_p, pr);
+    tmem_ld_wait();
     float ds[32];
-    if (ok) {
-      uint32_t sr[32], pr[32];
-      tmem_ld16x64(tmem + lane_s, sr);
-      tmem_ld16x64(tmem + lane_p, pr);
-      tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
-        ds[e] = p * (__uint_as_float(pr[e]) - dterm);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) ds[e] = 0.f;
+    for (int e = 0; e < 32; ++e) {
+      const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
+      ds[e] = p * (__uint_as_float(pr[e]) - dterm);
     }
     // dQ(n-1) has read the dS tile and the K / V stage of block n+1
     ok = ok && (n == 0 || mbar_wait(&dq_done, (n - 1) & 1, prm.status));
@@ -546,8 +604,9 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     store_row_operand(s_t, row, kh, ds);
     fence_proxy_async_smem();
     tc_fence_before();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
+    if (!ok) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) { ok = false; break; }
     if (threadIdx.x == 64) {
       tc_fence_after();
       const uint32_t sa = smem_u32(s_t), kb = smem_u32(k_t + st * kTile);
@@ -603,12 +662,14 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   uint8_t* s_t = smem + 4 * kTile + kPTile;   // dS^T tile
   __shared__ uint64_t kv_full, qo_full, s_done, acc_done;
   __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;   // set by any thread whose wait timed out
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int T = prm.tcount[bh * prm.nb + j];
-  const int32_t* ilist = prm.tlist + (bh * prm.nb + j) * static_cast<int64_t>(prm.nb);
+  const int32_t* ilist = prm.tlist + bh * prm.nb * static_cast<int64_t>(prm.k) +
+                         prm.toff[bh * (prm.nb + 1) + j];
   const int blk0 = static_cast<int>(bh * (prm.n_pad / 64));
   if (warp == 0) {
     tmem_alloc(&tmem_slot, 256);
@@ -619,6 +680,7 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     mbar_init(&qo_full, 1);
     mbar_init(&s_done, 2);               // S^T from warp 0, dP^T from warp 1
     mbar_init(&acc_done, 2);             // dV from warp 2, dK from warp 3
+    abort_flag = 0;
     fence_mbar_init();
   }
   tc_fence_before();
@@ -672,20 +734,15 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     // a failed wait only clears ok: every thread leaves the loop together after its barrier
     ok = ok && mbar_wait(&s_done, t & 1, prm.status);
     tc_fence_after();
+    uint32_t sr[32], pr[32];
+    tmem_ld16x64(tmem + lane_s, sr);
+    tmem_ld16x64(tmem + lane_p, pr);
+    tmem_ld_wait();
     float pt[32], ds[32];
-    if (ok) {
-      uint32_t sr[32], pr[32];
-      tmem_ld16x64(tmem + lane_s, sr);
-      tmem_ld16x64(tmem + lane_p, pr);
-      tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        pt[e] = exp2f(__uint_as_float(sr[e]) * c2 - lq[e]);
-        ds[e] = pt[e] * (__uint_as_float(pr[e]) - dq_[e]);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) { pt[e] = 0.f; ds[e] = 0.f; }
+    for (int e = 0; e < 32; ++e) {
+      pt[e] = exp2f(__uint_as_float(sr[e]) * c2 - lq[e]);
+      ds[e] = pt[e] * (__uint_as_float(pr[e]) - dq_[e]);
     }
     // the previous dV / dK MMAs have read the P^T and dS^T tiles and the Q / dO tiles
     ok = ok && (t == 0 || mbar_wait(&acc_done, (t - 1) & 1, prm.status));
@@ -693,8 +750,9 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     store_row_operand(s_t, row, kh, ds);
     fence_proxy_async_smem();
     tc_fence_before();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
+    if (!ok) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) { ok = false; break; }
     if (threadIdx.x == 64 || threadIdx.x == 96) {  // dV (warp 2) and dK (warp 3)
       tc_fence_after();
       const bool is_v = threadIdx.x == 64;
@@ -1123,7 +1181,8 @@ bool make_backward_layout(const ForwardPlan& p, BackwardLayout* bl) {
   bl->lse = take(rows * 4);
   bl->dd = take(rows * 4);
   bl->tcount = take(static_cast<size_t>(p.BH * p.nb) * 4);
-  bl->tlist = take(static_cast<size_t>(p.BH * p.nb * p.nb) * 4);
+  bl->toff = take(static_cast<size_t>(p.BH * (p.nb + 1)) * 4);
+  bl->tlist = take(static_cast<size_t>(p.BH * p.nb * p.k) * 4);
   if (!p.linear_empty) {
     bl->lin_q = take(rows * 512);
     bl->lin_k = take(rows * 512);
@@ -1168,10 +1227,19 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
         reinterpret_cast<uint4*>(ws + bl.vn), reinterpret_cast<uint4*>(ws + bl.dn));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t warps = p.BH * p.nb;
-    k_bwd_lists<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, stream>>>(
-        static_cast<int>(p.nb), static_cast<int>(p.mask_words), p.BH,
-        reinterpret_cast<const uint32_t*>(ws + L.mask), reinterpret_cast<int32_t*>(ws + bl.tcount),
-        reinterpret_cast<int32_t*>(ws + bl.tlist));
+    const unsigned lgrid = static_cast<unsigned>((warps * 32 + 255) / 256);
+    const uint32_t* mask = reinterpret_cast<const uint32_t*>(ws + L.mask);
+    k_bwd_list_count<<<lgrid, 256, 0, stream>>>(static_cast<int>(p.nb), static_cast<int>(p.mask_words),
+                                                p.BH, mask, reinterpret_cast<int32_t*>(ws + bl.tcount));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_bwd_list_scan<<<static_cast<unsigned>(p.BH), 1024, 0, stream>>>(
+        static_cast<int>(p.nb), reinterpret_cast<const int32_t*>(ws + bl.tcount),
+        reinterpret_cast<int32_t*>(ws + bl.toff));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_bwd_list_fill<<<lgrid, 256, 0, stream>>>(static_cast<int>(p.nb), static_cast<int>(p.k),
+                                               static_cast<int>(p.mask_words), p.BH, mask,
+                                               reinterpret_cast<const int32_t*>(ws + bl.toff),
+                                               reinterpret_cast<int32_t*>(ws + bl.tlist));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   CUtensorMap tq, tk, tv, td;
@@ -1181,6 +1249,7 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
   BwdParams prm;
   prm.kept = reinterpret_cast<const int32_t*>(ws + L.kept);
   prm.tcount = reinterpret_cast<const int32_t*>(ws + bl.tcount);
+  prm.toff = reinterpret_cast<const int32_t*>(ws + bl.toff);
   prm.tlist = reinterpret_cast<const int32_t*>(ws + bl.tlist);
   prm.qn = reinterpret_cast<const uint16_t*>(ws + bl.qn);
   prm.dn = reinterpret_cast<const uint16_t*>(ws + bl.dn);

@@ -49,7 +49,8 @@ bool encode_tmap_nd(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, 
 struct BackwardLayout {
   size_t qn, kn, vn, dn;            // packed bf16 Q, K, V, dO [BH][n_pad][128]
   size_t lse, dd;                   // [BH][n_pad] f32
-  size_t tcount, tlist;             // query blocks keeping each key block: [BH][nb], [BH][nb][nb]
+  size_t tcount, toff, tlist;       // query blocks keeping each key block: counts [BH][nb],
+                                    // offsets [BH][nb + 1], indices [BH][nb * k]
   size_t lin_q, lin_k, lin_v;       // linear-branch gradients [BH][n_pad][128] f32
   size_t amask_t;                   // transposed complement mask [BH][nb_m_pad][nb_m_pad] bf16
   size_t dg, dh;                    // [BH][nb_m_pad][129 * 128] bf16

@@ -515,46 +515,51 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int tok = 64 * qblock + r;             // token index within the head
     const int64_t b_ = bh / prm.q.H, h_ = bh % prm.q.H;
     float den = 0.f;
+    // the branch below exchanges values with lane ^ 2: take it warp-uniformly even when a
+    // timed-out wait (read per lane from ctl->abort) left the lanes disagreeing
+    ok = __all_sync(0xffffffffu, ok) != 0;
     if (prm.linear && ok) {
-      // phi(q) of this row: the thread writes channels 64kh .. 64kh+63 (chunk kh) of the A
-      // operand (bf16, K-major, 128-byte swizzle) and sums its part of the normalizer.
+      // phi(q) of this row: the thread takes channels 64kh .. 64kh+63 (chunk kh of the A
+      // operand: bf16, K-major, 128-byte swizzle), the other half is lane ^ 2; the pair reduces
+      // the max and the normalizer, and each thread sums its part of the denominator.
       const uint16_t* qrow = static_cast<const uint16_t*>(prm.q.data) + b_ * prm.q.stride_b +
                              h_ * prm.q.stride_h + static_cast<int64_t>(min(tok, prm.N - 1)) * prm.q.stride_n;
-      const uint4* q4 = reinterpret_cast<const uint4*>(qrow);
+      const uint4* q4 = reinterpret_cast<const uint4*>(qrow) + 8 * kh;
       float mx = -INFINITY;
 #pragma unroll 4
-      for (int u = 0; u < 16; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const uint4 rr = __ldg(q4 + u);
         const uint32_t w[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
         for (int z = 0; z < 4; ++z)
           mx = fmaxf(mx, fmaxf(__uint_as_float(w[z] << 16), __uint_as_float(w[z] & 0xFFFF0000u)));
       }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       float sum = 0.f;
 #pragma unroll 4
-      for (int u = 0; u < 16; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const uint4 rr = __ldg(q4 + u);
         const uint32_t w[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
         for (int z = 0; z < 4; ++z)
           sum += __expf(__uint_as_float(w[z] << 16) - mx) + __expf(__uint_as_float(w[z] & 0xFFFF0000u) - mx);
       }
-      const float inv = 1.f / sum;
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      const float inv = tok < prm.N ? 1.f / sum : 0.f;
       const uint4* g128 = reinterpret_cast<const uint4*>(
-          prm.gsum + ((bh * prm.nb_m_pad + qblock) * 129 + 128) * 128);
+          prm.gsum + ((bh * prm.nb_m_pad + qblock) * 129 + 128) * 128) + 8 * kh;
       float dsum = 0.f;
 #pragma unroll 2
       for (int uu = 0; uu < 8; ++uu) {
-        const int u = 8 * kh + uu;
-        const uint4 rr = __ldg(q4 + u);
-        const uint4 gg = __ldg(g128 + u);
+        const uint4 rr = __ldg(q4 + uu);
+        const uint4 gg = __ldg(g128 + uu);
         const uint32_t w[4] = {rr.x, rr.y, rr.z, rr.w};
         const uint32_t gw[4] = {gg.x, gg.y, gg.z, gg.w};
         uint32_t packed[4];
 #pragma unroll
         for (int z = 0; z < 4; ++z) {
-          const float a0 = tok < prm.N ? __expf(__uint_as_float(w[z] << 16) - mx) * inv : 0.f;
-          const float a1 = tok < prm.N ? __expf(__uint_as_float(w[z] & 0xFFFF0000u) - mx) * inv : 0.f;
+          const float a0 = __expf(__uint_as_float(w[z] << 16) - mx) * inv;
+          const float a1 = __expf(__uint_as_float(w[z] & 0xFFFF0000u) - mx) * inv;
           __nv_bfloat162 p2 = __floats2bfloat162_rn(a0, a1);
           packed[z] = *reinterpret_cast<uint32_t*>(&p2);
           dsum = fmaf(__low2float(p2), __uint_as_float(gw[z] << 16), dsum);

@@ -5,9 +5,10 @@
 // ratio 0.1) and skipping the rest. Here a pair is (query block i, key block j) of 64 tokens
 // and its score is the dot product of the pooled block means.
 //
-//  k_scores  fp32 FMA tiles (128 x 128, 8 x 8 per thread, packed f32x2) of qbar . kbar^T -> raw dot products
-//            [head][nb][nb], each a sum over the 128 channels in ascending order. FFMA, not a
-//            low-precision tensor-core product, keeps the ranking accurate to ~1e-7 relative.
+//  k_scores  qbar . kbar^T -> raw dot products [head][nb][nb] on the tensor cores (tcgen05
+//            kind::tf32, 128 x 128 tiles) as three TF32 products of exact hi / lo splits
+//            (3xTF32): about 2^-20 relative per product, where one TF32 product (2^-11) could
+//            reorder blocks well outside the selection's tie margin.
 //  k_topk_warp  one warp per (query block, head) for rows of up to 2048 key blocks: bisection
 //            for the k-th largest order-preserving 32-bit key with the row in registers, then
 //            an ordered compaction that takes every larger score and the lowest-index equal
@@ -23,92 +24,150 @@ namespace sagesla {
 
 namespace {
 
-constexpr int kScoreTile = 128;            // 128 x 128 scores per CTA, 8 x 8 per thread
-constexpr int kScoreChunk = 32;            // channels staged in shared memory at a time
+constexpr int kScoreTile = 128;                          // 128 x 128 scores per CTA (M = N = 128)
+constexpr int kScoreChunk = 32;                          // channels per stage: one 128-byte fp32 row
+constexpr int kScorePart = kScoreTile * kScoreChunk * 4; // 16 KB: one operand part of a stage
+constexpr int kScoreSmem = 4 * kScorePart + 1024;        // A hi / lo, B hi / lo, alignment slack
+constexpr uint32_t kFmtTF32 = 2;
 
-__device__ __forceinline__ unsigned long long pk2(float a, float b) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void up2(unsigned long long v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
-                                                   unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Thread (ty, tx) of 16 x 16 computes the 8 x 8 scores of rows i0 + 8ty + a (a < 8) and
-// columns j0 + 4tx + 64h + u (h < 2, u < 4) with packed f32x2 FMAs. Per channel it reads its
-// rows and columns as 128-bit shared loads (6 shared-memory wavefronts per warp for 32 packed
-// FMAs, so the FMA pipe sets the pace) and it stores 16-byte column groups, a warp covering
-// 256 contiguous bytes of a row (rows are ld floats apart, ld a multiple of 4). Each score is
-// one FMA chain over the channels in ascending order.
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void mma_tf32(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// x = hi + lo exactly, hi with the low 13 mantissa bits cleared (a TF32 value), so that the
+// tensor core reads hi without loss and lo (|lo| < 2^-10 |x|) to 2^-11 of itself.
+__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
+  hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+  lo = x - hi;
+}
+
+// One CTA computes the 128 x 128 raw dot products qbar[i] . kbar[j] of rows i0.. and columns
+// j0.. of one head on the tensor cores in three TF32 products (3xTF32): with a = a_hi + a_lo
+// and b = b_hi + b_lo split exactly, a.b = a_lo.b_hi + a_hi.b_lo + a_hi.b_hi up to the
+// dropped a_lo.b_lo and the TF32 reading of the lo parts, about 2^-20 of |a||b| per product:
+// far inside the 1e-4 relative margin within which the Top-K selection counts as a tie.
+// Channels are staged 32 at a time (a 128-byte row per block, 128-byte swizzle, K-major),
+// each stage split into hi and lo parts by the 128 threads; thread 0 issues the 12 MMAs of a
+// stage (4 K-steps of 8 channels x 3 products) into one fp32 TMEM accumulator of 128 columns.
+// The global loads of stage c+1 are in flight while the MMAs of stage c run. Rows or columns
+// past nb read as zero; columns up to ld (the padded row length) are written.
+__global__ void __launch_bounds__(128)
 k_scores(int nb, int ld, const float* __restrict__ qbar, const float* __restrict__ kbar,
-         float* __restrict__ scores) {
-  __shared__ __align__(16) float qs[kScoreChunk][kScoreTile];
-  __shared__ __align__(16) float ks[kScoreChunk][kScoreTile];
+         float* __restrict__ scores, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t mma_bar;
+  __shared__ uint32_t tmem_slot;
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* a_hi = smem;
+  uint8_t* a_lo = smem + kScorePart;
+  uint8_t* b_hi = smem + 2 * kScorePart;
+  uint8_t* b_lo = smem + 3 * kScorePart;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int64_t bh = blockIdx.z;
   const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
-  const int t = threadIdx.x;
-  const int ty = t >> 4, tx = t & 15;
-  unsigned long long acc[8][4];   // [row a][column pair: 2h + u/2]
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0ull;
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, kScoreTile);
+    tmem_relinquish();
+  }
+  if (t == 0) {
+    mbar_init(&mma_bar, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
   const float* qh = qbar + bh * nb * static_cast<int64_t>(kHeadDim);
   const float* kh = kbar + bh * nb * static_cast<int64_t>(kHeadDim);
+  constexpr uint32_t idesc = make_idesc(kFmtF32, kFmtTF32, kFmtTF32, 0, 0, kScoreTile, kScoreTile);
+  bool ok = true;
 #pragma unroll 1
-  for (int c0 = 0; c0 < kHeadDim; c0 += kScoreChunk) {
-    __syncthreads();
-    // 128 rows x 8 float4 chunks per operand; consecutive threads take consecutive rows
+  for (int c = 0; c < kHeadDim / kScoreChunk; ++c) {
+    // 128 rows x 8 chunks of 16 bytes per operand; a warp reads 4 whole 128-byte rows
+    float4 qv[8], kv[8];
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int e = t + 256 * it;
-      const int r = e & 127, cq = e >> 7;
-      float4 qv = make_float4(0.f, 0.f, 0.f, 0.f), kv = qv;
-      if (i0 + r < nb) qv = __ldg(reinterpret_cast<const float4*>(qh + (i0 + r) * kHeadDim + c0) + cq);
-      if (j0 + r < nb) kv = __ldg(reinterpret_cast<const float4*>(kh + (j0 + r) * kHeadDim + c0) + cq);
-      qs[4 * cq + 0][r] = qv.x; qs[4 * cq + 1][r] = qv.y; qs[4 * cq + 2][r] = qv.z; qs[4 * cq + 3][r] = qv.w;
-      ks[4 * cq + 0][r] = kv.x; ks[4 * cq + 1][r] = kv.y; ks[4 * cq + 2][r] = kv.z; ks[4 * cq + 3][r] = kv.w;
+    for (int it = 0; it < 8; ++it) {
+      const int e = t + 128 * it, r = e >> 3, ch = e & 7;
+      qv[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+      kv[it] = qv[it];
+      if (i0 + r < nb)
+        qv[it] = __ldg(reinterpret_cast<const float4*>(qh + (i0 + r) * kHeadDim + c * kScoreChunk) + ch);
+      if (j0 + r < nb)
+        kv[it] = __ldg(reinterpret_cast<const float4*>(kh + (j0 + r) * kHeadDim + c * kScoreChunk) + ch);
     }
-    __syncthreads();
-#pragma unroll 2
-    for (int c = 0; c < kScoreChunk; ++c) {
-      const float4 q0 = *reinterpret_cast<const float4*>(&qs[c][8 * ty]);
-      const float4 q1 = *reinterpret_cast<const float4*>(&qs[c][8 * ty + 4]);
-      const ulonglong2 k0 = *reinterpret_cast<const ulonglong2*>(&ks[c][4 * tx]);
-      const ulonglong2 k1 = *reinterpret_cast<const ulonglong2*>(&ks[c][4 * tx + 64]);
-      const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      const unsigned long long kb[4] = {k0.x, k0.y, k1.x, k1.y};
+    // the MMAs of the previous stage read the buffers about to be overwritten
+    if (c > 0) ok = mbar_wait(&mma_bar, (c - 1) & 1, status);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const unsigned long long q2 = pk2(qa[a], qa[a]);
+    for (int it = 0; it < 8; ++it) {
+      const int e = t + 128 * it, r = e >> 3, ch = e & 7;
+      const uint32_t off = sw128_offset(r, ch);
+      float4 h, l;
+      split_tf32(qv[it].x, h.x, l.x); split_tf32(qv[it].y, h.y, l.y);
+      split_tf32(qv[it].z, h.z, l.z); split_tf32(qv[it].w, h.w, l.w);
+      *reinterpret_cast<float4*>(a_hi + off) = h;
+      *reinterpret_cast<float4*>(a_lo + off) = l;
+      split_tf32(kv[it].x, h.x, l.x); split_tf32(kv[it].y, h.y, l.y);
+      split_tf32(kv[it].z, h.z, l.z); split_tf32(kv[it].w, h.w, l.w);
+      *reinterpret_cast<float4*>(b_hi + off) = h;
+      *reinterpret_cast<float4*>(b_lo + off) = l;
+    }
+    fence_proxy_async_smem();
+    if (__syncthreads_or(!ok)) {          // a timed-out wait: every thread leaves here
+      ok = false;
+      break;
+    }
+    if (t == 0) {
+      tc_fence_after();
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fma2(q2, kb[b], acc[a][b]);
+      for (int ks = 0; ks < kScoreChunk / 8; ++ks) {
+        // K-step of 8 fp32 = 32 bytes inside the swizzled 128-byte rows; 8-row groups 1 KB apart
+        const uint64_t dah = make_sdesc(smem_u32(a_hi) + 32 * ks, 16, 1024, kLayoutSW128);
+        const uint64_t dal = make_sdesc(smem_u32(a_lo) + 32 * ks, 16, 1024, kLayoutSW128);
+        const uint64_t dbh = make_sdesc(smem_u32(b_hi) + 32 * ks, 16, 1024, kLayoutSW128);
+        const uint64_t dbl = make_sdesc(smem_u32(b_lo) + 32 * ks, 16, 1024, kLayoutSW128);
+        mma_tf32(tmem, dal, dbh, idesc, (c | ks) != 0);      // small terms first
+        mma_tf32(tmem, dah, dbl, idesc, 1);
+        mma_tf32(tmem, dah, dbh, idesc, 1);
+      }
+      mma_commit(&mma_bar);
+    }
+  }
+  if (ok) ok = mbar_wait(&mma_bar, (kHeadDim / kScoreChunk - 1) & 1, status);
+  ok = !__syncthreads_or(!ok);
+  tc_fence_after();
+  if (ok) {
+    // warp w reads TMEM lanes 32w..32w+31 = rows; each thread stores 32 columns per load
+    const int i = i0 + 32 * warp + lane;
+    float* srow = scores + (bh * nb + i) * static_cast<int64_t>(ld);
+#pragma unroll 1
+    for (int cb = 0; cb < kScoreTile / 32; ++cb) {
+      uint32_t v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * cb, v);
+      tmem_ld_wait();
+      if (i < nb) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int j = j0 + 32 * cb + 4 * q;
+          if (j < ld)
+            *reinterpret_cast<float4*>(srow + j) =
+                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        }
       }
     }
   }
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int i = i0 + 8 * ty + a;
-    if (i >= nb) continue;
-    float* srow = scores + (bh * nb + i) * static_cast<int64_t>(ld);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int j = j0 + 4 * tx + 64 * h;
-      if (j >= ld) continue;
-      float4 v;
-      up2(acc[a][2 * h], v.x, v.y);
-      up2(acc[a][2 * h + 1], v.z, v.w);
-      *reinterpret_cast<float4*>(srow + j) = v;
-    }
-  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kScoreTile);
 }
 
 // Order-preserving map float -> uint32 (larger float, larger key); -0 is mapped like +0.
@@ -341,12 +400,16 @@ __global__ void k_scale_scores(int64_t n, int nb, int ld, const float* __restric
 
 cudaError_t launch_scores(const ForwardPlan& p, char* ws, cudaStream_t stream) {
   const auto& L = p.lay;
-  const unsigned nt = static_cast<unsigned>((p.nb + kScoreTile - 1) / kScoreTile);
-  dim3 grid(nt, nt, static_cast<unsigned>(p.BH));
-  k_scores<<<grid, 256, 0, stream>>>(static_cast<int>(p.nb), static_cast<int>(p.scores_ld),
-                                     reinterpret_cast<const float*>(ws + L.qbar),
-                                     reinterpret_cast<const float*>(ws + L.kbar),
-                                     reinterpret_cast<float*>(ws + L.scores));
+  const cudaError_t attr =
+      cudaFuncSetAttribute(k_scores, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
+  if (attr != cudaSuccess) return attr;
+  dim3 grid(static_cast<unsigned>((p.scores_ld + kScoreTile - 1) / kScoreTile),
+            static_cast<unsigned>((p.nb + kScoreTile - 1) / kScoreTile), static_cast<unsigned>(p.BH));
+  k_scores<<<grid, 128, kScoreSmem, stream>>>(static_cast<int>(p.nb), static_cast<int>(p.scores_ld),
+                                              reinterpret_cast<const float*>(ws + L.qbar),
+                                              reinterpret_cast<const float*>(ws + L.kbar),
+                                              reinterpret_cast<float*>(ws + L.scores),
+                                              reinterpret_cast<int*>(ws + L.status));
   return cudaGetLastError();
 }
 

@@ -9,13 +9,17 @@
 //            kind::tf32, 128 x 128 tiles) as three TF32 products of exact hi / lo splits
 //            (3xTF32): about 2^-20 relative per product, where one TF32 product (2^-11) could
 //            reorder blocks well outside the selection's tie margin.
-//  k_topk_warp  one warp per (query block, head) for rows of up to 2048 key blocks: bisection
-//            for the k-th largest order-preserving 32-bit key with the row in registers, then
-//            an ordered compaction that takes every larger score and the lowest-index equal
+//  k_topk_warp  one warp per (query block, head) row for rows of up to 2048 key blocks,
+//            persistent over the rows with the next row's scores loaded during the current
+//            selection: bisection for the k-th largest order-preserving 32-bit key with the row
+//            in registers down to at most 32 candidates, a warp bitonic sort of those, then an
+//            ordered compaction that takes every larger score and the lowest-index equal
 //            ones. Writes the kept list (ascending), the bitmask and the bf16 complement mask
 //            row (1 = not kept) of the linear branch.
 //  k_topk    the same selection for longer rows, one CTA per row (radix select by bytes).
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -283,34 +287,30 @@ k_topk(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __restr
   }
 }
 
-// One warp per (query block, head) row for rows of at most 32*M key blocks: the row's keys
-// stay in registers (key j = 32m + lane in key[m]); the k-th largest key T is found by
-// bisection on the 32-bit key space with warp-wide counts of the keys >= the midpoint, over
-// all keys until at most 32 remain between the bounds, then over those alone; the row is
-// then compacted in ascending j, taking every key above T and the lowest-index keys
-// equal to T. Same selection as k_topk, without block-wide synchronization.
-template <int M>
-__global__ void __launch_bounds__(128, M <= 24 ? 8 : (M <= 40 ? 6 : 4))
-k_topk_warp(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __restrict__ scores,
-            int32_t* __restrict__ kept, uint32_t* __restrict__ mask,
-            __nv_bfloat16* __restrict__ amask, int nb_m_pad) {
-  const int lane = threadIdx.x & 31;
-  const int i = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int64_t bh = blockIdx.y;
-  if (i >= nb_m_pad) return;
-  __nv_bfloat16* arow = amask + (bh * nb_m_pad + i) * static_cast<int64_t>(nb_k_pad);
-  const __nv_bfloat16 one = __float2bfloat16_rn(1.f), zero = __float2bfloat16_rn(0.f);
-  if (i >= nb) {   // padding rows of the complement mask
-    for (int j = lane; j < nb_k_pad; j += 32) arow[j] = zero;
-    return;
-  }
-  const float* srow = scores + (bh * nb + i) * static_cast<int64_t>(ld);
-  uint32_t key[M];
+// Bitonic sort of one key per lane into descending order across lanes 0..31 (15
+// compare-exchange stages: in stage (size, step) the lower lane of each pair keeps the larger
+// key inside blocks of `size` lanes that end up descending, the smaller one otherwise).
+__device__ __forceinline__ uint32_t warp_sort_desc(uint32_t v, int lane) {
 #pragma unroll
-  for (int m = 0; m < M; ++m) {
-    const int j = 32 * m + lane;
-    key[m] = j < nb ? order_key(__ldg(srow + j)) : 0u;   // 0 is below every real key
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int step = size >> 1; step > 0; step >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, v, step);
+      const bool desc_block = (lane & size) == 0;
+      const bool lower = (lane & step) == 0;
+      v = (lower == desc_block) ? max(v, o) : min(v, o);
+    }
   }
+  return v;
+}
+
+// Selection of one row whose order-preserving keys sit in registers, key[m] of lane l being
+// block j = 32m + l (0 for j >= nb, below every real key).
+template <int M>
+__device__ __forceinline__ void topk_row(const uint32_t (&key)[M], int lane, uint32_t* cw, int nb,
+                                         int k, int mask_words, int nb_k_pad, int32_t* krow,
+                                         uint32_t* mrow, __nv_bfloat16* arow) {
+  const __nv_bfloat16 one = __float2bfloat16_rn(1.f), zero = __float2bfloat16_rn(0.f);
   // Invariants: count(key >= lo) = cnt_lo >= k, count(key > hi) = cnt_above < k. The bracket
   // starts at the row's smallest and largest keys and is split at the midpoint of the two
   // scores (about half the splits of halving the key range, for score rows of ordinary
@@ -330,11 +330,12 @@ k_topk_warp(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __
     c = __reduce_add_sync(0xffffffffu, c);
     if (c >= k) { lo = mid; cnt_lo = c; } else { hi = mid - 1u; cnt_above = c; }
   }
+  // T = the k-th largest key; n_gt / n_ge = how many keys are above / at least T
+  uint32_t T = lo;
+  int n_gt = cnt_above, n_ge = cnt_lo;
   if (lo < hi) {
-    // At most 32 keys lie in [lo, hi]: gather them one per lane and finish the bisection on
-    // them alone (count(key >= mid) = cnt_above + candidates >= mid).
-    __shared__ uint32_t cand[4][32];
-    uint32_t* cw = cand[threadIdx.x >> 5];
+    // At most 32 keys lie in [lo, hi]: gather them one per lane, sort them, and read T off
+    // as the (k - cnt_above)-th largest of them.
     int n_cand = 0;
 #pragma unroll
     for (int m = 0; m < M; ++m) {
@@ -344,37 +345,106 @@ k_topk_warp(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __
       n_cand += __popc(bits);
     }
     __syncwarp();
-    const bool has = lane < n_cand;
-    const uint32_t ck = has ? cw[lane] : 0u;
-    while (lo < hi) {   // cnt_above stays the count above the gathered range
-      const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
-      const int c = cnt_above + __popc(__ballot_sync(0xffffffffu, has && ck >= mid));
-      if (c >= k) lo = mid; else hi = mid - 1u;
+    const uint32_t sorted = warp_sort_desc(lane < n_cand ? cw[lane] : 0u, lane);
+    __syncwarp();                          // cw is rewritten by the warp's next row
+    T = __shfl_sync(0xffffffffu, sorted, k - cnt_above - 1);
+    n_gt = cnt_above + __popc(__ballot_sync(0xffffffffu, sorted > T));
+    n_ge = cnt_above + __popc(__ballot_sync(0xffffffffu, sorted >= T));
+  }
+  const uint32_t below = (1u << lane) - 1u;
+  int kept_base = 0;
+  if (n_ge == k) {
+    // no tie at T to split: exactly the keys >= T are kept (T > 0, so never a padding slot)
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const int j = 32 * m + lane;
+      const bool sel = key[m] >= T;
+      const uint32_t sel_bits = __ballot_sync(0xffffffffu, sel);
+      if (sel) krow[kept_base + __popc(sel_bits & below)] = j;
+      if (lane == 0 && m < mask_words) mrow[m] = sel_bits;
+      if (j < nb_k_pad) arow[j] = (j < nb && !sel) ? one : zero;
+      kept_base += __popc(sel_bits);
+    }
+  } else {
+    // keys equal to T: the lowest-index ones, up to k - n_gt of them
+    const int take_equal = k - n_gt;
+    int eq_base = 0;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const int j = 32 * m + lane;
+      const bool eq = j < nb && key[m] == T;
+      const uint32_t eq_bits = __ballot_sync(0xffffffffu, eq);
+      const bool sel = j < nb && (key[m] > T || (eq && eq_base + __popc(eq_bits & below) < take_equal));
+      const uint32_t sel_bits = __ballot_sync(0xffffffffu, sel);
+      if (sel) krow[kept_base + __popc(sel_bits & below)] = j;
+      if (lane == 0 && m < mask_words) mrow[m] = sel_bits;
+      if (j < nb_k_pad) arow[j] = (j < nb && !sel) ? one : zero;
+      eq_base += __popc(eq_bits);
+      kept_base += __popc(sel_bits);
     }
   }
-  const uint32_t T = lo;
-  int gt = 0;
-#pragma unroll
-  for (int m = 0; m < M; ++m) gt += key[m] > T ? 1 : 0;
-  const int take_equal = k - __reduce_add_sync(0xffffffffu, gt);
-  int32_t* krow = kept + (bh * nb + i) * static_cast<int64_t>(k);
-  uint32_t* mrow = mask + (bh * nb + i) * static_cast<int64_t>(mask_words);
-  const uint32_t below = (1u << lane) - 1u;
-  int eq_base = 0, kept_base = 0;
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-    const int j = 32 * m + lane;
-    const bool eq = j < nb && key[m] == T;
-    const uint32_t eq_bits = __ballot_sync(0xffffffffu, eq);
-    const bool sel = j < nb && (key[m] > T || (eq && eq_base + __popc(eq_bits & below) < take_equal));
-    const uint32_t sel_bits = __ballot_sync(0xffffffffu, sel);
-    if (sel) krow[kept_base + __popc(sel_bits & below)] = j;
-    if (lane == 0 && m < mask_words) mrow[m] = sel_bits;
-    if (j < nb_k_pad) arow[j] = (j < nb && !sel) ? one : zero;
-    eq_base += __popc(eq_bits);
-    kept_base += __popc(sel_bits);
-  }
   for (int j = 32 * M + lane; j < nb_k_pad; j += 32) arow[j] = zero;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Rows of up to 32*M key blocks, one warp per row, persistent: warp w of the grid takes rows
+// w, w + (warps in the grid), ... of all heads (padding rows i >= nb only clear their
+// complement-mask row). The scores of the warp's next row are copied into its shared-memory
+// row buffer (cp.async) while the current row is selected, so the DRAM latency of a row
+// load overlaps the selection of the previous one.
+template <int M>
+__global__ void __launch_bounds__(128, M <= 8 ? 8 : (M <= 16 ? 6 : (M <= 48 ? 4 : 3)))
+k_topk_warp(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __restrict__ scores,
+            int32_t* __restrict__ kept, uint32_t* __restrict__ mask,
+            __nv_bfloat16* __restrict__ amask, int nb_m_pad, int64_t n_rows) {
+  __shared__ uint32_t cand[4][32];
+  __shared__ __align__(16) float rowbuf[4][32 * M];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t* cw = cand[warp];
+  float* rb = rowbuf[warp];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * 4;
+  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+  // the nb real scores of a row as 16-byte chunks (rows are ld >= 4 * chunks floats apart)
+  const int chunks = (nb + 3) >> 2;
+  auto prefetch_row = [&](int64_t rw) {
+    const int64_t bh = rw / nb_m_pad;
+    const int i = static_cast<int>(rw - bh * nb_m_pad);
+    if (i >= nb) return;
+    const float* srow = scores + (bh * nb + i) * static_cast<int64_t>(ld);
+    for (int c = lane; c < chunks; c += 32) cp_async16(rb + 4 * c, srow + 4 * c);
+    cp_async_commit();
+  };
+  int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  if (row < n_rows) prefetch_row(row);
+  for (; row < n_rows; row += stride) {
+    const int64_t bh = row / nb_m_pad;
+    const int i = static_cast<int>(row - bh * nb_m_pad);
+    __nv_bfloat16* arow = amask + (bh * nb_m_pad + i) * static_cast<int64_t>(nb_k_pad);
+    if (i >= nb) {   // padding rows of the complement mask (nothing was copied for them)
+      for (int j = lane; j < nb_k_pad; j += 32) arow[j] = zero;
+      if (row + stride < n_rows) prefetch_row(row + stride);
+      continue;
+    }
+    cp_async_wait_all();
+    __syncwarp();
+    uint32_t key[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const int j = 32 * m + lane;
+      key[m] = j < nb ? order_key(rb[j]) : 0u;   // 0 is below every real key
+    }
+    __syncwarp();                              // the row buffer is refilled next
+    if (row + stride < n_rows) prefetch_row(row + stride);
+    topk_row<M>(key, lane, cw, nb, k, mask_words, nb_k_pad,
+                kept + (bh * nb + i) * static_cast<int64_t>(k),
+                mask + (bh * nb + i) * static_cast<int64_t>(mask_words), arow);
+  }
+  cp_async_wait_all();
 }
 
 // Every key block kept (k == nb): kept lists 0..nb-1 and full masks. Written only when a
@@ -416,12 +486,21 @@ cudaError_t launch_scores(const ForwardPlan& p, char* ws, cudaStream_t stream) {
 template <int M>
 static cudaError_t launch_topk_warp(const ForwardPlan& p, char* ws, cudaStream_t stream) {
   const auto& L = p.lay;
-  dim3 grid(static_cast<unsigned>((p.nb_m_pad + 3) / 4), static_cast<unsigned>(p.BH));
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+      (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_topk_warp<M>, 128, 0)) !=
+          cudaSuccess)
+    return e;
+  const int64_t n_rows = p.BH * p.nb_m_pad;
+  const int64_t resident = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1);
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>((n_rows + 3) / 4, resident));
   k_topk_warp<M><<<grid, 128, 0, stream>>>(
       static_cast<int>(p.nb), static_cast<int>(p.scores_ld), static_cast<int>(p.k), static_cast<int>(p.mask_words),
       static_cast<int>(p.nb_k_pad), reinterpret_cast<const float*>(ws + L.scores),
       reinterpret_cast<int32_t*>(ws + L.kept), reinterpret_cast<uint32_t*>(ws + L.mask),
-      reinterpret_cast<__nv_bfloat16*>(ws + L.amask), static_cast<int>(p.nb_m_pad));
+      reinterpret_cast<__nv_bfloat16*>(ws + L.amask), static_cast<int>(p.nb_m_pad), n_rows);
   return cudaGetLastError();
 }
 

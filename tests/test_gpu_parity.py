@@ -122,7 +122,25 @@ def test_dense_mode(n, seed):
     assert torch.equal(plain["out"], res["out"])
 
 
-@pytest.mark.parametrize("n", [4096, 2050 * 64])
+@pytest.mark.parametrize("nb,ratio,seed", [
+    (200, 0.1, 41),     # 7 chunks of 32 key blocks per lane row
+    (700, 0.15, 42),    # 22 chunks
+    (1000, 0.05, 43),   # 32 chunks, the bucket's full width
+    (1400, 0.1, 44),    # 44 chunks
+    (1900, 0.1, 45),    # 60 chunks
+])
+def test_selection_for_every_row_length_bucket(nb, ratio, seed):
+    """Rows of each register-resident size of the warp selection: kept lists and masks against
+    the oracle's Top-K, codes bit-exact, sampled query blocks against the oracle output."""
+    n = nb * 64 - 17
+    q, k, v = inputs.make_random(1, 1, n, seed, k_offset_std=1.0)
+    res = gpu_run(q, k, v, ratio)
+    assert res["layout"]["nb"] == nb
+    err, _ = compare_head(q, k, v, ratio, res, 0, 0, rows=_sampled_rows(nb, seed, count=2))
+    assert err <= OUT_TOL, err
+
+
+@pytest.mark.parametrize("n", [4096, 700 * 64, 2050 * 64])
 def test_equal_scores_keep_the_lowest_blocks(n):
     """Constant K makes every score of a row equal: the selection keeps blocks 0..k-1."""
     q, _, v = inputs.make_random(1, 1, n, 31)

@@ -13,8 +13,8 @@
 //                       one weight block: its exact int32 product comes out of 4 M=128 N=256
 //                       K=32 kind::i8 MMAs into one of two TMEM buffers (2 x 256 columns),
 //                       and eight "promotion" warps move it into fp32 register accumulators
-//                       scaled by the block's weight scale (int -> float exactly through the
-//                       1.5 * 2^23 bias, then one packed FMA), while the tensor core already
+//                       scaled by the block's weight scale (one exact int -> float conversion
+//                       per element, |s| < 2^22, then one packed FMA), while the tensor core already
 //                       works on the next K block in the other buffer. The epilogue multiplies
 //                       by the token scale, adds the bias, rounds and leaves through shared
 //                       memory with bulk tensor stores.
@@ -112,11 +112,6 @@ __device__ __forceinline__ unsigned long long fma2g(unsigned long long a, unsign
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-__device__ __forceinline__ unsigned long long add2g(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 
 __device__ __forceinline__ void tma_store_2d_g(const CUtensorMap* map, const void* smem_src,
                                                int x, int y) {
@@ -197,7 +192,6 @@ k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     unsigned long long acc[64];
 #pragma unroll
     for (int i = 0; i < 64; ++i) acc[i] = 0ull;
-    const unsigned long long unbias = pk2g(-12582912.0f, -12582912.0f);
     bool ok = true;
     for (int kb = 0; kb < nkb; ++kb) {
       const int b = kb & 1;
@@ -212,10 +206,8 @@ k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          // exact int -> float: |s| < 2^22, so bits(s + 0x4B400000) = 1.5 * 2^23 + s
-          const unsigned long long f2 = add2g(
-              pk2g(__int_as_float(static_cast<int>(r[e] + 0x4B400000u)),
-                   __int_as_float(static_cast<int>(r[e + 1] + 0x4B400000u))), unbias);
+          const unsigned long long f2 = pk2g(__int2float_rn(static_cast<int>(r[e])),
+                                             __int2float_rn(static_cast<int>(r[e + 1])));
           acc[16 * cc + (e >> 1)] = fma2g(c2, f2, acc[16 * cc + (e >> 1)]);
         }
       }

@@ -22,8 +22,8 @@
 // makes the 16x64b TMEM fragment of an M=64 result hold 32 consecutive tokens per thread, so
 // the P and dS operands written back by the threads are 64 contiguous bytes after one pair
 // exchange. The sparse branch runs on tcgen05 BF16 MMAs (fp32 accumulators in TMEM):
-//   k_bwd_lse     per query block: the sparse forward again (online softmax), giving the
-//                 base-2 log-sum-exp L and D = rowsum(dO * O_s)
+//   k_bwd_lse     per query block: the scores again (online softmax), giving the base-2
+//                 log-sum-exp L and D = rowsum(dO * O_s), taken as rowsum(P * dO V^T)
 //   k_bwd_dq      per query block over its kept blocks: S, dP, dS, dQ; adds the linear dq
 //   k_bwd_dkv     per key block over the query blocks that keep it (compressed per-head lists
 //                 built from the kept bitmask): S^T, dP^T, dV, dK; adds
@@ -281,22 +281,31 @@ struct BwdParams {
 constexpr int kBwdThreads = 128;
 
 // Online-softmax pass of one query block over its kept key blocks (bf16 MMAs): writes the
-// base-2 log-sum-exp L of the scaled scores and D = rowsum(dO * O_s) of its 64 rows.
-// TMEM: two S buffers [0, 64) and [64, 128), O [128, 256). S of block n + 1 is issued (by
-// thread 0) as soon as S of block n is in registers, so that it runs under the softmax of
-// block n; P.V is issued by warp 1.
-__global__ void __launch_bounds__(kBwdThreads, 2)
-k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-          const __grid_constant__ CUtensorMap tm_v, BwdParams prm) {
+// base-2 log-sum-exp L of the scaled scores and D = rowsum(dO * O_s) of its 64 rows. D is
+// taken as rowsum(P * dP) with dP = dO V^T (the same sum: O_s = P V), accumulated online like
+// the normalizer, both rescaled by the per-row factor when the running maximum moves, so the
+// pass needs neither a P operand tile nor an O accumulator.
+// Warps 0-3 take the softmax (one row pair per lane pair, as everywhere here); warp 4 issues
+// S = Q K^T and warp 5 dP = dO V^T of each block into double buffers (TMEM [0, 128) and
+// [128, 256)), running ahead of the softmax by one block; warp 6 loads the K and V tiles into
+// a two-stage ring, refilling a stage as soon as the MMAs of the block in it have completed.
+// Everything is ordered by mbarriers (no block-wide barrier in the loop); every wait is
+// bounded, and a timed-out wait ends every role's loop through abort_flag.
+constexpr int kLseThreads = 224;
+
+__global__ void __launch_bounds__(kLseThreads, 2)
+k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+          BwdParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* q_t = smem;                   // Q tile
-  uint8_t* k_t = smem + kTile;           // 2 K stages
-  uint8_t* v_t = smem + 3 * kTile;       // 2 V stages
-  uint8_t* p_t = smem + 5 * kTile;       // P tile
-  __shared__ uint64_t q_full, k_full[2], v_full[2], s_done[2], pv_done;
+  uint8_t* do_t = smem + kTile;          // dO tile
+  uint8_t* k_t = smem + 2 * kTile;       // 2 K stages
+  uint8_t* v_t = smem + 4 * kTile;       // 2 V stages
+  __shared__ uint64_t q_full, k_full[2], v_full[2], s_done[2], s_free[2];
   __shared__ uint32_t tmem_slot;
-  __shared__ volatile int abort_flag;   // set by any thread whose wait timed out
+  __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x;
@@ -311,9 +320,10 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   if (threadIdx.x == 32) {
     mbar_init(&q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1); mbar_init(&v_full[s], 1); mbar_init(&s_done[s], 1);
+      mbar_init(&k_full[s], 1); mbar_init(&v_full[s], 1);
+      mbar_init(&s_done[s], 2);          // the S and the dP commit of a block
+      mbar_init(&s_free[s], 4);          // the four softmax warps have read a block
     }
-    mbar_init(&pv_done, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -321,145 +331,105 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  const uint32_t qa = smem_u32(q_t);
   bool ok = true;
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
-    mbar_arrive_expect_tx(&q_full, kTile);
-    load_tile(q_t, &tm_q, &q_full, blk0 + i);
-    const int j0 = __ldg(klist);
-    mbar_arrive_expect_tx(&k_full[0], kTile);
-    load_tile(k_t, &tm_k, &k_full[0], blk0 + j0);
-    mbar_arrive_expect_tx(&v_full[0], kTile);
-    load_tile(v_t, &tm_v, &v_full[0], blk0 + j0);
-    if (U > 1) {
-      mbar_arrive_expect_tx(&k_full[1], kTile);
-      load_tile(k_t + kTile, &tm_k, &k_full[1], blk0 + __ldg(klist + 1));
+  if (warp == 6) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q); prefetch_tmap(&tm_do); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(&q_full, 2 * kTile);
+      load_tile(q_t, &tm_q, &q_full, blk0 + i);
+      load_tile(do_t, &tm_do, &q_full, blk0 + i);
+      for (int m = 0; m < U; ++m) {
+        const int b = m & 1;
+        // stage b held block m - 2: its S and dP MMAs must have completed
+        if (m >= 2 && (abort_flag || !mbar_wait(&s_done[b], ((m - 2) >> 1) & 1, prm.status))) {
+          ok = false;
+          break;
+        }
+        const int jm = blk0 + __ldg(klist + m);
+        mbar_arrive_expect_tx(&k_full[b], kTile);
+        load_tile(k_t + b * kTile, &tm_k, &k_full[b], jm);
+        mbar_arrive_expect_tx(&v_full[b], kTile);
+        load_tile(v_t + b * kTile, &tm_v, &v_full[b], jm);
+      }
+      if (!ok) abort_flag = 1;
     }
-    ok = mbar_wait(&q_full, 0, prm.status) && mbar_wait(&k_full[0], 0, prm.status);
-    if (ok) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem, desc_k128(qa, kk), desc_k128(smem_u32(k_t), kk), kIdescKK64, kk > 0 ? 1u : 0u);
-      mma_commit(&s_done[0]);
-    }
-  }
-  const int row = frag_row(warp, lane);
-  const int kh = (lane >> 1) & 1;
-  const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
-  const float c2 = kScale * kLog2e;
-  float m_run = -INFINITY, l_part = 0.f;
-  if (!ok) abort_flag = 1;       // thread 0's waits above decide for every thread
-  __syncthreads();
-  ok = !abort_flag;
-  for (int n = 0; n < U && ok; ++n) {
-    const int j = __ldg(klist + n);
-    const int st = n & 1;
-    // a failed wait only clears ok: every thread leaves the loop together after its barrier
-    ok = mbar_wait(&s_done[st], (n >> 1) & 1, prm.status);
-    tc_fence_after();
-    uint32_t sr[32];
-    tmem_ld16x64(tmem + lane_s + 64 * st, sr);
-    tmem_ld_wait();
-    if (ok && threadIdx.x == 0 && n + 1 < U) {
-      // S(n+1) into the other buffer (read by every thread before the last barrier), and K of
-      // block n+2 into the stage S(n) has finished reading
-      if (mbar_wait(&k_full[st ^ 1], ((n + 1) >> 1) & 1, prm.status)) {
-        const uint32_t kb = smem_u32(k_t + (st ^ 1) * kTile);
+  } else if (warp >= 4) {
+    // ------------------------------------------------ MMA issuers: warp 4 S, warp 5 dP
+    if (lane == 0) {
+      const bool is_s = warp == 4;
+      uint64_t* full = is_s ? k_full : v_full;
+      const uint32_t a = smem_u32(is_s ? q_t : do_t);
+      const uint32_t stage = smem_u32(is_s ? k_t : v_t);
+      const uint32_t dcol = is_s ? 0u : 128u;
+      ok = mbar_wait(&q_full, 0, prm.status);
+      for (int n = 0; n < U && ok; ++n) {
+        const int b = n & 1;
+        // buffer b held block n - 2: the softmax warps must have read it
+        if (n >= 2) ok = !abort_flag && mbar_wait(&s_free[b], ((n - 2) >> 1) & 1, prm.status);
+        ok = ok && !abort_flag && mbar_wait(&full[b], (n >> 1) & 1, prm.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t bsm = stage + b * kTile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + 64 * (st ^ 1), desc_k128(qa, kk), desc_k128(kb, kk), kIdescKK64,
+          mma_bf16(tmem + dcol + 64 * b, desc_k128(a, kk), desc_k128(bsm, kk), kIdescKK64,
                    kk > 0 ? 1u : 0u);
-        mma_commit(&s_done[st ^ 1]);
+        mma_commit(&s_done[b]);
       }
-      if (n + 2 < U) {
-        mbar_arrive_expect_tx(&k_full[st], kTile);
-        load_tile(k_t + st * kTile, &tm_k, &k_full[st], blk0 + __ldg(klist + n + 2));
-      }
+      if (!ok) abort_flag = 1;
     }
-    const int valid = (j == prm.nb - 1) ? prm.n_last - 32 * kh : 32;   // real keys of this thread
-    float x[32], mx = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      x[e] = e < valid ? __uint_as_float(sr[e]) * c2 : -INFINITY;
-      mx = fmaxf(mx, x[e]);
-    }
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    const float alpha = exp2f(m_run - m_new);
-    float rs = 0.f;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) { x[e] = exp2f(x[e] - m_new); rs += x[e]; }
-    l_part = alpha * l_part + rs;
-    m_run = m_new;
-    // P.V(n-1) done: frees the P tile and the V stage of block n+1, and O is stable
-    ok = ok && (n == 0 || mbar_wait(&pv_done, (n - 1) & 1, prm.status));
-    tc_fence_after();
-    if (ok && threadIdx.x == 0 && n + 1 < U) {
-      mbar_arrive_expect_tx(&v_full[st ^ 1], kTile);
-      load_tile(v_t + (st ^ 1) * kTile, &tm_v, &v_full[st ^ 1], blk0 + __ldg(klist + n + 1));
-    }
-    if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t o[32];
-        tmem_ld16x64(tmem + lane_s + 128 + 64 * cc, o);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-        tmem_st16x64(tmem + lane_s + 128 + 64 * cc, o);
-      }
-      tmem_st_wait();
-    }
-    store_row_operand(p_t, row, kh, x);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (!ok) abort_flag = 1;
-    __syncthreads();
-    if (abort_flag) { ok = false; break; }
-    if (threadIdx.x == 32) {
+  } else {
+    // ------------------------------------------------ softmax warps
+    const int row = frag_row(warp, lane);
+    const int kh = (lane >> 1) & 1;
+    const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
+    const float c2 = kScale * kLog2e;
+    float m_run = -INFINITY, l_part = 0.f, d_part = 0.f;
+    for (int n = 0; n < U; ++n) {
+      const int st = n & 1;
+      ok = !abort_flag && mbar_wait(&s_done[st], (n >> 1) & 1, prm.status);
+      ok = __all_sync(0xffffffffu, ok) != 0;      // the warp leaves together
+      if (!ok) break;
       tc_fence_after();
-      if (mbar_wait(&v_full[st], (n >> 1) & 1, prm.status)) {
-        const uint32_t pa = smem_u32(p_t), vb = smem_u32(v_t + st * kTile);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 128, desc_k64(pa, kk), desc_mn128(vb, kk), kIdescKM128,
-                   (n > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&pv_done);
-      }
-    }
-  }
-  if (ok) ok = mbar_wait(&pv_done, (U - 1) & 1, prm.status);
-  tc_fence_after();
-  // O_s = O / l; D = dO . O_s over the row (this thread: columns kh + 2e and 64 + kh + 2e)
-  const float l_row = l_part + __shfl_xor_sync(0xffffffffu, l_part, 2);
-  const int tok = tile_token(row);
-  const int64_t grow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + tok;
-  float dsum = 0.f;
-  if (ok) {
-    const uint4* drow = reinterpret_cast<const uint4*>(prm.dn + grow * 128);
-#pragma unroll 1
-    for (int cc = 0; cc < 2; ++cc) {
-      uint32_t o[32];
-      tmem_ld16x64(tmem + lane_s + 128 + 64 * cc, o);
+      uint32_t sr[32], pr[32];
+      tmem_ld16x64(tmem + lane_s + 64 * st, sr);
+      tmem_ld16x64(tmem + lane_s + 128 + 64 * st, pr);
       tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[st]);
+      const int j = __ldg(klist + n);
+      const int valid = (j == prm.nb - 1) ? prm.n_last - 32 * kh : 32;   // real keys of this thread
+      float x[32], mx = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint4 w = __ldg(drow + 8 * cc + u);    // columns 64cc + 8u .. +7
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int z = 0; z < 4; ++z) {   // element pair (2e, 2e + 1), e = 4u + z
-          const float dv = bf16_bits_to_f32(kh ? (ww[z] >> 16) : (ww[z] & 0xFFFFu));
-          dsum = fmaf(dv, __uint_as_float(o[4 * u + z]), dsum);
-        }
+      for (int e = 0; e < 32; ++e) {
+        x[e] = e < valid ? __uint_as_float(sr[e]) * c2 : -INFINITY;
+        mx = fmaxf(mx, x[e]);
       }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m_run, mx);
+      const float alpha = exp2f(m_run - m_new);
+      float rs = 0.f, pd = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float p = exp2f(x[e] - m_new);
+        rs += p;
+        pd = fmaf(p, __uint_as_float(pr[e]), pd);
+      }
+      l_part = alpha * l_part + rs;
+      d_part = alpha * d_part + pd;
+      m_run = m_new;
     }
-  }
-  dsum += __shfl_xor_sync(0xffffffffu, dsum, 2);
-  if (ok && kh == 0) {
-    prm.lse[grow] = m_run + log2f(l_row);
-    prm.dd[grow] = dsum / l_row;
+    if (!ok) abort_flag = 1;
+    const float l_row = l_part + __shfl_xor_sync(0xffffffffu, l_part, 2);
+    const float d_row = d_part + __shfl_xor_sync(0xffffffffu, d_part, 2);
+    const int tok = tile_token(row);
+    const int64_t grow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + tok;
+    if (ok && kh == 0) {
+      prm.lse[grow] = m_run + log2f(l_row);
+      prm.dd[grow] = d_row / l_row;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -1271,20 +1241,17 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
   prm.n_last = p.n_last;
   prm.H = static_cast<int>(p.H);
   const dim3 grid(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.BH));
-  const int smem_lse = 1024 + 5 * kTile + kPTile;
+  const int smem_lse = 1024 + 6 * kTile;
   const int smem_dq = 1024 + 6 * kTile + kPTile;
   const int smem_dkv = 1024 + 4 * kTile + 2 * kPTile;
-  static bool configured = false;
-  if (!configured) {
-    if ((e = cudaFuncSetAttribute(k_bwd_lse, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_lse)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(k_bwd_dq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(k_bwd_dkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(k_bwd_lin_query, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(k_bwd_lin_key, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem)) != cudaSuccess)
-      return e;
-    configured = true;
-  }
-  k_bwd_lse<<<grid, kBwdThreads, smem_lse, stream>>>(tq, tk, tv, prm);
+  // set on every call: the attribute belongs to the current device
+  if ((e = cudaFuncSetAttribute(k_bwd_lse, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_lse)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(k_bwd_dq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(k_bwd_dkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(k_bwd_lin_query, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(k_bwd_lin_key, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem)) != cudaSuccess)
+    return e;
+  k_bwd_lse<<<grid, kLseThreads, smem_lse, stream>>>(tq, td, tk, tv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (!p.linear_empty) {
     CUtensorMap tg, th, tvn;

@@ -174,13 +174,10 @@ cudaError_t launch_mask_gemm(const void* a, const void* b, void* c, int64_t BH, 
       !encode_tmap_2d(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kHFlat, BH * M,
                       static_cast<uint64_t>(kHFlat) * 2, c, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_complement_gemm,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // set on every call: the attribute belongs to the current device
+  cudaError_t e = cudaFuncSetAttribute(k_complement_gemm,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e != cudaSuccess) return e;
   dim3 grid((kHFlat + kTileN - 1) / kTileN, static_cast<unsigned>((M + kTileM - 1) / kTileM),
             static_cast<unsigned>(BH));
   k_complement_gemm<<<grid, kGemmThreads, kGemmSmem, stream>>>(

@@ -406,15 +406,12 @@ k_quant(TensorArg Q, TensorArg K, TensorArg V, int N, int nb, int n_pad, int nbq
 
 cudaError_t launch_stats(const ForwardPlan& p, TensorArg k, TensorArg v, char* ws,
                          cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    for (const void* f : {reinterpret_cast<const void*>(k_stats<true>),
-                          reinterpret_cast<const void*>(k_stats<false>)}) {
-      cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kStatsSmem);
-      if (e != cudaSuccess) return e;
-    }
-    configured = true;
+  // set on every call: the attribute belongs to the current device
+  for (const void* f : {reinterpret_cast<const void*>(k_stats<true>),
+                        reinterpret_cast<const void*>(k_stats<false>)}) {
+    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kStatsSmem);
+    if (e != cudaSuccess) return e;
   }
   const auto& L = p.lay;
   dim3 grid(static_cast<unsigned>(p.nb_k_pad), static_cast<unsigned>(p.BH));

@@ -344,13 +344,10 @@ extern "C" sagesla_status sagesla_w8a8_gemm(const int8_t* x8, const float* x_sca
                       N, M, y_stride * esz, y, y_dtype == SAGESLA_F32 ? 32 : 64, 32,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return SAGESLA_ERR_CUDA;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(k_w8a8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem) !=
-        cudaSuccess)
-      return SAGESLA_ERR_CUDA;
-    configured = true;
-  }
+  // set on every call: the attribute belongs to the current device
+  if (cudaFuncSetAttribute(k_w8a8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem) !=
+      cudaSuccess)
+    return SAGESLA_ERR_CUDA;
   GemmParams p;
   p.x_scale = x_scale;
   p.w_scale = w_scale;

@@ -24,10 +24,11 @@
 // exchange. The sparse branch runs on tcgen05 BF16 MMAs (fp32 accumulators in TMEM):
 //   k_bwd_lse     per query block: the scores again (online softmax), giving the base-2
 //                 log-sum-exp L and D = rowsum(dO * O_s), taken as rowsum(P * dO V^T)
-//   k_bwd_dq      per query block over its kept blocks: S, dP, dS, dQ; adds the linear dq
+//   k_bwd_dq      per query block over its kept blocks: S, dP, dS, dQ (role warps: softmax,
+//                 S / dP / dQ issuers, TMA producer); adds the linear dq
 //   k_bwd_dkv     per key block over the query blocks that keep it (compressed per-head lists
-//                 built from the kept bitmask): S^T, dP^T, dV, dK; adds
-//                 the linear dk, dv
+//                 built from the kept bitmask): S^T, dP^T, dV, dK (role warps, a two-stage
+//                 Q / dO ring); adds the linear dk, dv
 // The linear branch runs on the CUDA cores (k_bwd_lin_query, k_bwd_lin_key) around one
 // complement GEMM on the tensor cores (dH = (1 - M)^T dG, the forward's GEMM on the
 // transposed mask).
@@ -278,7 +279,6 @@ struct BwdParams {
   int N, nb, n_pad, k, n_last, H;
 };
 
-constexpr int kBwdThreads = 128;
 
 // Online-softmax pass of one query block over its kept key blocks (bf16 MMAs): writes the
 // base-2 log-sum-exp L of the scaled scores and D = rowsum(dO * O_s) of its 64 rows. D is
@@ -471,11 +471,16 @@ __device__ __forceinline__ void* grad_row(void* base, int32_t dtype, int64_t sb,
   return static_cast<char*>(base) + off * (dtype == SAGESLA_F32 ? 4 : 2);
 }
 
-// dQ of one query block over its kept key blocks: S = Q K^T and dP = dO V^T (one M=64 N=64
-// group each; S in TMEM lanes 0-15 and dP in lanes 16-31 of each quadrant, columns [0, 64)),
-// dS = P (dP - D) with P = 2^(S c - L), dQ += dS K (columns [64, 192)). The linear-branch dq
-// is added before the store.
-__global__ void __launch_bounds__(kBwdThreads, 2)
+// dQ of one query block over its kept key blocks: S = Q K^T and dP = dO V^T (M=64 N=64 each;
+// S in TMEM lanes 0-15 and dP in lanes 16-31 of each quadrant, double-buffered in columns
+// [0, 64) and [64, 128)), dS = P (dP - D) with P = 2^(S c - L), dQ += dS K (columns
+// [128, 256)). Role warps ordered by mbarriers: warps 0-3 the softmax (dS into the shared
+// tile), warp 4 issues S and warp 5 dP one block ahead, warp 6 dQ, warp 7 loads K and V of
+// each block into a two-stage ring, refilling a stage once the dQ of its block (the last
+// reader of K) has completed. The linear-branch dq is added before the store.
+constexpr int kDqThreads = 256;
+
+__global__ void __launch_bounds__(kDqThreads, 2)
 k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
          BwdParams prm) {
@@ -486,9 +491,9 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   uint8_t* k_t = smem + 2 * kTile;       // 2 K stages
   uint8_t* v_t = smem + 4 * kTile;       // 2 V stages
   uint8_t* s_t = smem + 6 * kTile;       // dS tile
-  __shared__ uint64_t q_full, kv_full[2], s_done, dq_done;
+  __shared__ uint64_t q_full, kv_full[2], s_done[2], s_free[2], ds_full, dq_done[2];
   __shared__ uint32_t tmem_slot;
-  __shared__ volatile int abort_flag;   // set by any thread whose wait timed out
+  __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x;
@@ -502,9 +507,13 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   }
   if (threadIdx.x == 32) {
     mbar_init(&q_full, 1);
-    for (int s = 0; s < 2; ++s) mbar_init(&kv_full[s], 1);
-    mbar_init(&s_done, 2);               // S from warp 0, dP from warp 1
-    mbar_init(&dq_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&s_done[s], 2);          // the S and the dP commit of a block
+      mbar_init(&s_free[s], 4);          // the four softmax warps have read S and dP
+      mbar_init(&dq_done[s], 1);
+    }
+    mbar_init(&ds_full, 4);              // the four softmax warps have stored dS
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -512,99 +521,130 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_do);
-    mbar_arrive_expect_tx(&q_full, 2 * kTile);
-    load_tile(q_t, &tm_q, &q_full, blk0 + i);
-    load_tile(o_t, &tm_do, &q_full, blk0 + i);
-    const int j0 = __ldg(klist);
-    mbar_arrive_expect_tx(&kv_full[0], 2 * kTile);
-    load_tile(k_t, &tm_k, &kv_full[0], blk0 + j0);
-    load_tile(v_t, &tm_v, &kv_full[0], blk0 + j0);
-  }
-  const int row = frag_row(warp, lane);
-  const int kh = (lane >> 1) & 1;
-  const int tok = tile_token(row);
-  const int64_t grow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + tok;
-  const float l2 = prm.lse[grow], dterm = prm.dd[grow];
-  const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
-  const uint32_t lane_p = static_cast<uint32_t>(32 * warp + 16) << 16;
-  const float c2 = kScale * kLog2e;
   bool ok = true;
-  int j_next = __ldg(klist);
-  for (int n = 0; n < U; ++n) {
-    const int st = n & 1;
-    if (n + 1 < U) j_next = __ldg(klist + n + 1);
-    if (ok && (threadIdx.x == 0 || threadIdx.x == 32)) {   // S (warp 0) and dP (warp 1)
-      ok = (n > 0 || mbar_wait(&q_full, 0, prm.status)) &&
-           mbar_wait(&kv_full[st], (n >> 1) & 1, prm.status);
-      if (ok) {
+  if (warp == 7) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_do);
+      mbar_arrive_expect_tx(&q_full, 2 * kTile);
+      load_tile(q_t, &tm_q, &q_full, blk0 + i);
+      load_tile(o_t, &tm_do, &q_full, blk0 + i);
+      for (int m = 0; m < U; ++m) {
+        const int b = m & 1;
+        // stage b held block m - 2: its dQ (after its S and dP) must have completed
+        if (m >= 2 && (abort_flag || !mbar_wait(&dq_done[b], ((m - 2) >> 1) & 1, prm.status))) {
+          ok = false;
+          break;
+        }
+        const int jm = blk0 + __ldg(klist + m);
+        mbar_arrive_expect_tx(&kv_full[b], 2 * kTile);
+        load_tile(k_t + b * kTile, &tm_k, &kv_full[b], jm);
+        load_tile(v_t + b * kTile, &tm_v, &kv_full[b], jm);
+      }
+      if (!ok) abort_flag = 1;
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------ dQ issuer
+    if (lane == 0) {
+      const uint32_t sa = smem_u32(s_t);
+      for (int n = 0; n < U; ++n) {
+        ok = !abort_flag && mbar_wait(&ds_full, n & 1, prm.status);
+        if (!ok) break;
         tc_fence_after();
-        const bool is_s = threadIdx.x == 0;
-        const uint32_t a = smem_u32(is_s ? q_t : o_t);
-        const uint32_t b = smem_u32((is_s ? k_t : v_t) + st * kTile);
-        const uint32_t d = is_s ? tmem : tmem + (16u << 16);
+        const uint32_t kb = smem_u32(k_t + (n & 1) * kTile);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + 128, desc_k64(sa, kk), desc_mn128(kb, kk), kIdescKM128,
+                   (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&dq_done[n & 1]);
+      }
+      if (!ok) abort_flag = 1;
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------ S (warp 4) and dP (warp 5) issuers
+    if (lane == 0) {
+      const bool is_s = warp == 4;
+      const uint32_t a = smem_u32(is_s ? q_t : o_t);
+      const uint32_t stage = smem_u32(is_s ? k_t : v_t);
+      const uint32_t dbase = is_s ? tmem : tmem + (16u << 16);
+      ok = mbar_wait(&q_full, 0, prm.status);
+      for (int n = 0; n < U && ok; ++n) {
+        const int b = n & 1;
+        // buffer b held block n - 2: the softmax warps must have read it
+        if (n >= 2) ok = !abort_flag && mbar_wait(&s_free[b], ((n - 2) >> 1) & 1, prm.status);
+        ok = ok && !abort_flag && mbar_wait(&kv_full[b], (n >> 1) & 1, prm.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t bsm = stage + b * kTile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(d, desc_k128(a, kk), desc_k128(b, kk), kIdescKK64, kk > 0 ? 1u : 0u);
-        mma_commit(&s_done);
+          mma_bf16(dbase + 64 * b, desc_k128(a, kk), desc_k128(bsm, kk), kIdescKK64,
+                   kk > 0 ? 1u : 0u);
+        mma_commit(&s_done[b]);
       }
+      if (!ok) abort_flag = 1;
     }
-    // a failed wait only clears ok: every thread leaves the loop together after its barrier
-    ok = ok && mbar_wait(&s_done, n & 1, prm.status);
-    tc_fence_after();
-    uint32_t sr[32], pr[32];
-    tmem_ld16x64(tmem + lane_s, sr);
-    tmem_ld16x64(tmem + lane_p, pr);
-    tmem_ld_wait();
-    float ds[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
-      ds[e] = p * (__uint_as_float(pr[e]) - dterm);
-    }
-    // dQ(n-1) has read the dS tile and the K / V stage of block n+1
-    ok = ok && (n == 0 || mbar_wait(&dq_done, (n - 1) & 1, prm.status));
-    tc_fence_after();
-    if (ok && threadIdx.x == 0 && n + 1 < U) {
-      mbar_arrive_expect_tx(&kv_full[st ^ 1], 2 * kTile);
-      load_tile(k_t + (st ^ 1) * kTile, &tm_k, &kv_full[st ^ 1], blk0 + j_next);
-      load_tile(v_t + (st ^ 1) * kTile, &tm_v, &kv_full[st ^ 1], blk0 + j_next);
-    }
-    store_row_operand(s_t, row, kh, ds);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (!ok) abort_flag = 1;
-    __syncthreads();
-    if (abort_flag) { ok = false; break; }
-    if (threadIdx.x == 64) {
+  } else {
+    // ------------------------------------------------ softmax warps
+    const int row = frag_row(warp, lane);
+    const int kh = (lane >> 1) & 1;
+    const int tok = tile_token(row);
+    const int64_t grow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + tok;
+    const float l2 = prm.lse[grow], dterm = prm.dd[grow];
+    const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
+    const uint32_t lane_p = static_cast<uint32_t>(32 * warp + 16) << 16;
+    const float c2 = kScale * kLog2e;
+    for (int n = 0; n < U; ++n) {
+      const int b = n & 1;
+      ok = !abort_flag && mbar_wait(&s_done[b], (n >> 1) & 1, prm.status);
+      ok = __all_sync(0xffffffffu, ok) != 0;      // the warp leaves together
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t sa = smem_u32(s_t), kb = smem_u32(k_t + st * kTile);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 64, desc_k64(sa, kk), desc_mn128(kb, kk), kIdescKM128,
-                 (n > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(&dq_done);
-    }
-  }
-  if (ok) ok = mbar_wait(&dq_done, (U - 1) & 1, prm.status);
-  tc_fence_after();
-  if (ok) {
-    const float* lin = prm.lin_q ? prm.lin_q + grow * 128 : nullptr;
-    const int t = 64 * i + tok;
-    void* dst = t < prm.N ? grad_row(prm.dq, prm.g_dtype, prm.dq_sb, prm.dq_sh, prm.dq_sn, bh,
-                                     prm.H, t)
-                          : nullptr;
-#pragma unroll 1
-    for (int cb = 0; cb < 2; ++cb) {
-      uint32_t o[32];
-      tmem_ld16x64(tmem + lane_s + 64 + 64 * cb, o);
+      uint32_t sr[32], pr[32];
+      tmem_ld16x64(tmem + lane_s + 64 * b, sr);
+      tmem_ld16x64(tmem + lane_p + 64 * b, pr);
       tmem_ld_wait();
-      float g[32];
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);
+      float ds[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        g[e] = __uint_as_float(o[e]) * kScale + (lin ? lin[64 * cb + kh + 2 * e] : 0.f);
-      store_grad_chunk(g, cb, kh, dst, prm.g_dtype);
+      for (int e = 0; e < 32; ++e) {
+        const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
+        ds[e] = p * (__uint_as_float(pr[e]) - dterm);
+      }
+      // dQ of block n - 1 has read the dS tile
+      if (n >= 1) {
+        ok = !abort_flag && mbar_wait(&dq_done[(n - 1) & 1], ((n - 1) >> 1) & 1, prm.status);
+        ok = __all_sync(0xffffffffu, ok) != 0;
+        if (!ok) break;
+      }
+      store_row_operand(s_t, row, kh, ds);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_full);
+    }
+    if (ok) ok = mbar_wait(&dq_done[(U - 1) & 1], ((U - 1) >> 1) & 1, prm.status);
+    ok = __all_sync(0xffffffffu, ok) != 0;
+    if (!ok) abort_flag = 1;
+    tc_fence_after();
+    if (ok) {
+      const float* lin = prm.lin_q ? prm.lin_q + grow * 128 : nullptr;
+      const int t = 64 * i + tok;
+      void* dst = t < prm.N ? grad_row(prm.dq, prm.g_dtype, prm.dq_sb, prm.dq_sh, prm.dq_sn, bh,
+                                       prm.H, t)
+                            : nullptr;
+#pragma unroll 1
+      for (int cb = 0; cb < 2; ++cb) {
+        uint32_t o[32];
+        tmem_ld16x64(tmem + lane_s + 128 + 64 * cb, o);
+        tmem_ld_wait();
+        float g[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          g[e] = __uint_as_float(o[e]) * kScale + (lin ? lin[64 * cb + kh + 2 * e] : 0.f);
+        store_grad_chunk(g, cb, kh, dst, prm.g_dtype);
+      }
     }
   }
   tc_fence_before();
@@ -613,27 +653,42 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
 }
 
 // dK, dV of one key block over the query blocks that keep it: S^T = K Q^T and dP^T = V dO^T
-// (lanes 0-15 / 16-31, columns [0, 64)), P^T = 2^(S^T c - L), dS^T = P^T (dP^T - D),
-// dV += P^T dO (lanes 0-15) and dK += dS^T Q (lanes 16-31), columns [64, 192). The
-// linear-branch dk, dv are added before the stores. A failed (timed-out) wait only clears a
-// thread's ok flag; the flags are ANDed at the loop's barrier, so every thread leaves the loop
-// at the same iteration.
-__global__ void __launch_bounds__(kBwdThreads, 2)
+// (TMEM lanes 0-15 / 16-31, double-buffered in columns [0, 64) and [64, 128)),
+// P^T = 2^(S^T c - L), dS^T = P^T (dP^T - D), dV += P^T dO (lanes 0-15) and dK += dS^T Q
+// (lanes 16-31), columns [128, 256). Role warps ordered by mbarriers: warps 0-3 the softmax
+// (P^T and dS^T into shared tiles), warp 4 issues S^T and warp 5 dP^T one query block ahead,
+// warp 6 dV and dK, warp 7 loads K and V once and the Q / dO tiles of each query block into a
+// two-stage ring, refilling a stage once the dV / dK MMAs of its block have completed. The
+// softmax warpgroup takes 168 registers and the role warpgroup 56 (setmaxnreg; 4 x 32 x 168 +
+// 4 x 32 x 56 = 28672 of the 256 x 128 a CTA is launched with). The seven tiles fill 112 KB
+// exactly, so that two CTAs share an SM: the dynamic shared memory is declared 1024-byte
+// aligned instead of being aligned by hand, and the kernel checks it. The linear-branch dk,
+// dv are added before the stores.
+constexpr int kDkvThreads = 256;
+constexpr int kDkvSmem = 6 * kTile + 2 * kPTile;   // K, V, Q x 2, dO x 2, P^T, dS^T
+constexpr int kDkvSoftmaxRegs = 168, kDkvRoleRegs = 56;
+static_assert(4 * 32 * kDkvSoftmaxRegs + 4 * 32 * kDkvRoleRegs <= kDkvThreads * 128,
+              "register split exceeds the launch's registers");
+
+__global__ void __launch_bounds__(kDkvThreads, 2)
 k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
           BwdParams prm) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint8_t* k_t = smem;                   // K tile
-  uint8_t* v_t = smem + kTile;           // V tile
-  uint8_t* q_t = smem + 2 * kTile;       // Q tile of the current query block
-  uint8_t* o_t = smem + 3 * kTile;       // dO tile
-  uint8_t* p_t = smem + 4 * kTile;       // P^T tile
-  uint8_t* s_t = smem + 4 * kTile + kPTile;   // dS^T tile
-  __shared__ uint64_t kv_full, qo_full, s_done, acc_done;
+  extern __shared__ __align__(1024) uint8_t smem_dkv[];
+  uint8_t* k_t = smem_dkv;                     // K tile
+  uint8_t* v_t = smem_dkv + kTile;             // V tile
+  uint8_t* q_t = smem_dkv + 2 * kTile;         // 2 Q stages
+  uint8_t* o_t = smem_dkv + 4 * kTile;         // 2 dO stages
+  uint8_t* p_t = smem_dkv + 6 * kTile;         // P^T tile
+  uint8_t* s_t = smem_dkv + 6 * kTile + kPTile;   // dS^T tile
+  __shared__ uint64_t kv_full, qo_full[2], s_done[2], s_free[2], p_full, acc_done[2];
   __shared__ uint32_t tmem_slot;
-  __shared__ volatile int abort_flag;   // set by any thread whose wait timed out
+  __shared__ volatile int abort_flag;
 
+  if (smem_u32(smem_dkv) & 1023u) {          // same for every thread of the CTA
+    if (threadIdx.x == 0) record_error(prm.status, SAGESLA_ERR_DEVICE_CHECK);
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x;
   const int64_t bh = blockIdx.y;
@@ -647,9 +702,13 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   }
   if (threadIdx.x == 32) {
     mbar_init(&kv_full, 1);
-    mbar_init(&qo_full, 1);
-    mbar_init(&s_done, 2);               // S^T from warp 0, dP^T from warp 1
-    mbar_init(&acc_done, 2);             // dV from warp 2, dK from warp 3
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&qo_full[s], 1);
+      mbar_init(&s_done[s], 2);          // the S^T and the dP^T commit of a query block
+      mbar_init(&s_free[s], 4);          // the four softmax warps have read S^T and dP^T
+      mbar_init(&acc_done[s], 1);
+    }
+    mbar_init(&p_full, 4);               // the four softmax warps have stored P^T and dS^T
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -657,123 +716,163 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_do);
-    mbar_arrive_expect_tx(&kv_full, 2 * kTile);
-    load_tile(k_t, &tm_k, &kv_full, blk0 + j);
-    load_tile(v_t, &tm_v, &kv_full, blk0 + j);
-    if (T > 0) {
-      const int i0 = __ldg(ilist);
-      mbar_arrive_expect_tx(&qo_full, 2 * kTile);
-      load_tile(q_t, &tm_q, &qo_full, blk0 + i0);
-      load_tile(o_t, &tm_do, &qo_full, blk0 + i0);
-    }
-  }
-  const int row = frag_row(warp, lane);
-  const int kh = (lane >> 1) & 1;
-  const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
-  const uint32_t lane_p = static_cast<uint32_t>(32 * warp + 16) << 16;
-  const float c2 = kScale * kLog2e;
   bool ok = true;
-  for (int t = 0; t < T; ++t) {
-    const int i = __ldg(ilist + t);
-    if (ok && (threadIdx.x == 0 || threadIdx.x == 32)) {   // S^T (warp 0) and dP^T (warp 1)
-      ok = (t > 0 || mbar_wait(&kv_full, 0, prm.status)) &&
-           mbar_wait(&qo_full, t & 1, prm.status);
-      if (ok) {
-        tc_fence_after();
-        const bool is_s = threadIdx.x == 0;
-        const uint32_t a = smem_u32(is_s ? k_t : v_t), b = smem_u32(is_s ? q_t : o_t);
-        const uint32_t d = is_s ? tmem : tmem + (16u << 16);
+  if (warp >= 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDkvRoleRegs));
+    if (warp == 7) {
+      // ---------------------------------------------- TMA producer
+      if (lane == 0 && T > 0) {
+        prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_do);
+        mbar_arrive_expect_tx(&kv_full, 2 * kTile);
+        load_tile(k_t, &tm_k, &kv_full, blk0 + j);
+        load_tile(v_t, &tm_v, &kv_full, blk0 + j);
+        for (int m = 0; m < T; ++m) {
+          const int b = m & 1;
+          // stage b held query block m - 2: its dV / dK MMAs must have completed
+          if (m >= 2 && (abort_flag || !mbar_wait(&acc_done[b], ((m - 2) >> 1) & 1, prm.status))) {
+            ok = false;
+            break;
+          }
+          const int im = blk0 + __ldg(ilist + m);
+          mbar_arrive_expect_tx(&qo_full[b], 2 * kTile);
+          load_tile(q_t + b * kTile, &tm_q, &qo_full[b], im);
+          load_tile(o_t + b * kTile, &tm_do, &qo_full[b], im);
+        }
+        if (!ok) abort_flag = 1;
+      }
+    } else if (warp == 6) {
+      // ---------------------------------------------- dV and dK issuer
+      if (lane == 0) {
+        const uint32_t pa = smem_u32(p_t), sa = smem_u32(s_t);
+        for (int n = 0; n < T; ++n) {
+          ok = !abort_flag && mbar_wait(&p_full, n & 1, prm.status);
+          if (!ok) break;
+          tc_fence_after();
+          const int b = n & 1;
+          const uint32_t ob = smem_u32(o_t + b * kTile), qb = smem_u32(q_t + b * kTile);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(d, desc_k128(a, kk), desc_k128(b, kk), kIdescKK64, kk > 0 ? 1u : 0u);
-        mma_commit(&s_done);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + 128, desc_k64(pa, kk), desc_mn128(ob, kk), kIdescKM128,
+                     (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + (16u << 16) + 128, desc_k64(sa, kk), desc_mn128(qb, kk), kIdescKM128,
+                     (n > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&acc_done[b]);
+        }
+        if (!ok) abort_flag = 1;
+      }
+    } else {
+      // ---------------------------------------------- S^T (warp 4) and dP^T (warp 5) issuers
+      if (lane == 0 && T > 0) {
+        const bool is_s = warp == 4;
+        const uint32_t a = smem_u32(is_s ? k_t : v_t);
+        const uint32_t stage = smem_u32(is_s ? q_t : o_t);
+        const uint32_t dbase = is_s ? tmem : tmem + (16u << 16);
+        ok = mbar_wait(&kv_full, 0, prm.status);
+        for (int n = 0; n < T && ok; ++n) {
+          const int b = n & 1;
+          // buffer b held query block n - 2: the softmax warps must have read it
+          if (n >= 2) ok = !abort_flag && mbar_wait(&s_free[b], ((n - 2) >> 1) & 1, prm.status);
+          ok = ok && !abort_flag && mbar_wait(&qo_full[b], (n >> 1) & 1, prm.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t bsm = stage + b * kTile;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(dbase + 64 * b, desc_k128(a, kk), desc_k128(bsm, kk), kIdescKK64,
+                     kk > 0 ? 1u : 0u);
+          mma_commit(&s_done[b]);
+        }
+        if (!ok) abort_flag = 1;
       }
     }
-    // L and D of the query tokens 32kh + e of block i (this thread's columns)
-    const int64_t qrow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + 32 * kh;
-    float lq[32], dq_[32];
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDkvSoftmaxRegs));
+    // ------------------------------------------------ softmax warps
+    const int row = frag_row(warp, lane);
+    const int kh = (lane >> 1) & 1;
+    const uint32_t lane_s = static_cast<uint32_t>(32 * warp) << 16;
+    const uint32_t lane_p = static_cast<uint32_t>(32 * warp + 16) << 16;
+    const float c2 = kScale * kLog2e;
+    for (int n = 0; n < T; ++n) {
+      const int b = n & 1;
+      const int i = __ldg(ilist + n);
+      // L and D of the query tokens 32kh + e of block i (this thread's columns)
+      const int64_t qrow = bh * prm.n_pad + 64 * static_cast<int64_t>(i) + 32 * kh;
+      float lq[32], dq_[32];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(prm.lse + qrow) + u);
-      const float4 b = __ldg(reinterpret_cast<const float4*>(prm.dd + qrow) + u);
-      lq[4 * u] = a.x; lq[4 * u + 1] = a.y; lq[4 * u + 2] = a.z; lq[4 * u + 3] = a.w;
-      dq_[4 * u] = b.x; dq_[4 * u + 1] = b.y; dq_[4 * u + 2] = b.z; dq_[4 * u + 3] = b.w;
-    }
-    // a failed wait only clears ok: every thread leaves the loop together after its barrier
-    ok = ok && mbar_wait(&s_done, t & 1, prm.status);
-    tc_fence_after();
-    uint32_t sr[32], pr[32];
-    tmem_ld16x64(tmem + lane_s, sr);
-    tmem_ld16x64(tmem + lane_p, pr);
-    tmem_ld_wait();
-    float pt[32], ds[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      pt[e] = exp2f(__uint_as_float(sr[e]) * c2 - lq[e]);
-      ds[e] = pt[e] * (__uint_as_float(pr[e]) - dq_[e]);
-    }
-    // the previous dV / dK MMAs have read the P^T and dS^T tiles and the Q / dO tiles
-    ok = ok && (t == 0 || mbar_wait(&acc_done, (t - 1) & 1, prm.status));
-    store_row_operand(p_t, row, kh, pt);
-    store_row_operand(s_t, row, kh, ds);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (!ok) abort_flag = 1;
-    __syncthreads();
-    if (abort_flag) { ok = false; break; }
-    if (threadIdx.x == 64 || threadIdx.x == 96) {  // dV (warp 2) and dK (warp 3)
+      for (int u = 0; u < 8; ++u) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(prm.lse + qrow) + u);
+        const float4 c = __ldg(reinterpret_cast<const float4*>(prm.dd + qrow) + u);
+        lq[4 * u] = a.x; lq[4 * u + 1] = a.y; lq[4 * u + 2] = a.z; lq[4 * u + 3] = a.w;
+        dq_[4 * u] = c.x; dq_[4 * u + 1] = c.y; dq_[4 * u + 2] = c.z; dq_[4 * u + 3] = c.w;
+      }
+      ok = !abort_flag && mbar_wait(&s_done[b], (n >> 1) & 1, prm.status);
+      ok = __all_sync(0xffffffffu, ok) != 0;      // the warp leaves together
+      if (!ok) break;
       tc_fence_after();
-      const bool is_v = threadIdx.x == 64;
-      const uint32_t a = smem_u32(is_v ? p_t : s_t), b = smem_u32(is_v ? o_t : q_t);
-      const uint32_t d = is_v ? tmem + 64 : tmem + (16u << 16) + 64;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(d, desc_k64(a, kk), desc_mn128(b, kk), kIdescKM128, (t > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(&acc_done);
-    }
-    if (threadIdx.x == 0 && t + 1 < T && mbar_wait(&acc_done, t & 1, prm.status)) {
-      // next query block's Q and dO once these MMAs have read the tiles
-      const int i1 = __ldg(ilist + t + 1);
-      mbar_arrive_expect_tx(&qo_full, 2 * kTile);
-      load_tile(q_t, &tm_q, &qo_full, blk0 + i1);
-      load_tile(o_t, &tm_do, &qo_full, blk0 + i1);
-    }
-  }
-  if (ok && T > 0) ok = mbar_wait(&acc_done, (T - 1) & 1, prm.status);
-  tc_fence_after();
-  if (ok) {
-    const int tok = tile_token(row);
-    const int t_key = 64 * j + tok;
-    const int64_t grow = bh * prm.n_pad + t_key;
-    const bool real = t_key < prm.N;
-    void* dst_k = real ? grad_row(prm.dk, prm.g_dtype, prm.dk_sb, prm.dk_sh, prm.dk_sn, bh, prm.H,
-                                  t_key)
-                       : nullptr;
-    void* dst_v = real ? grad_row(prm.dv, prm.g_dtype, prm.dv_sb, prm.dv_sh, prm.dv_sn, bh, prm.H,
-                                  t_key)
-                       : nullptr;
-#pragma unroll 1
-    for (int cb = 0; cb < 2; ++cb) {
-      uint32_t ov[32], okk[32];
-      if (T > 0) {
-        tmem_ld16x64(tmem + lane_s + 64 + 64 * cb, ov);
-        tmem_ld16x64(tmem + lane_p + 64 + 64 * cb, okk);
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) { ov[e] = 0u; okk[e] = 0u; }
-      }
-      float gk[32], gv[32];
+      uint32_t sr[32], pr[32];
+      tmem_ld16x64(tmem + lane_s + 64 * b, sr);
+      tmem_ld16x64(tmem + lane_p + 64 * b, pr);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);
+      float pt[32], ds[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const int c = 64 * cb + kh + 2 * e;
-        gv[e] = __uint_as_float(ov[e]) + (prm.lin_v ? prm.lin_v[grow * 128 + c] : 0.f);
-        gk[e] = __uint_as_float(okk[e]) * kScale + (prm.lin_k ? prm.lin_k[grow * 128 + c] : 0.f);
+        pt[e] = exp2f(__uint_as_float(sr[e]) * c2 - lq[e]);
+        ds[e] = pt[e] * (__uint_as_float(pr[e]) - dq_[e]);
       }
-      store_grad_chunk(gk, cb, kh, dst_k, prm.g_dtype);
-      store_grad_chunk(gv, cb, kh, dst_v, prm.g_dtype);
+      // dV / dK of query block n - 1 have read the P^T and dS^T tiles
+      if (n >= 1) {
+        ok = !abort_flag && mbar_wait(&acc_done[(n - 1) & 1], ((n - 1) >> 1) & 1, prm.status);
+        ok = __all_sync(0xffffffffu, ok) != 0;
+        if (!ok) break;
+      }
+      store_row_operand(p_t, row, kh, pt);
+      store_row_operand(s_t, row, kh, ds);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full);
+    }
+    if (ok && T > 0) ok = mbar_wait(&acc_done[(T - 1) & 1], ((T - 1) >> 1) & 1, prm.status);
+    ok = __all_sync(0xffffffffu, ok) != 0;
+    if (!ok) abort_flag = 1;
+    tc_fence_after();
+    if (ok) {
+      const int tok = tile_token(row);
+      const int t_key = 64 * j + tok;
+      const int64_t grow = bh * prm.n_pad + t_key;
+      const bool real = t_key < prm.N;
+      void* dst_k = real ? grad_row(prm.dk, prm.g_dtype, prm.dk_sb, prm.dk_sh, prm.dk_sn, bh,
+                                    prm.H, t_key)
+                         : nullptr;
+      void* dst_v = real ? grad_row(prm.dv, prm.g_dtype, prm.dv_sb, prm.dv_sh, prm.dv_sn, bh,
+                                    prm.H, t_key)
+                         : nullptr;
+#pragma unroll 1
+      for (int cb = 0; cb < 2; ++cb) {
+        uint32_t ov[32], okk[32];
+        if (T > 0) {
+          tmem_ld16x64(tmem + lane_s + 128 + 64 * cb, ov);
+          tmem_ld16x64(tmem + lane_p + 128 + 64 * cb, okk);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) { ov[e] = 0u; okk[e] = 0u; }
+        }
+        float gk[32], gv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = 64 * cb + kh + 2 * e;
+          gv[e] = __uint_as_float(ov[e]) + (prm.lin_v ? prm.lin_v[grow * 128 + c] : 0.f);
+          gk[e] = __uint_as_float(okk[e]) * kScale + (prm.lin_k ? prm.lin_k[grow * 128 + c] : 0.f);
+        }
+        store_grad_chunk(gk, cb, kh, dst_k, prm.g_dtype);
+        store_grad_chunk(gv, cb, kh, dst_v, prm.g_dtype);
+      }
     }
   }
   tc_fence_before();
@@ -1243,7 +1342,7 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
   const dim3 grid(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.BH));
   const int smem_lse = 1024 + 6 * kTile;
   const int smem_dq = 1024 + 6 * kTile + kPTile;
-  const int smem_dkv = 1024 + 4 * kTile + 2 * kPTile;
+  const int smem_dkv = kDkvSmem;
   // set on every call: the attribute belongs to the current device
   if ((e = cudaFuncSetAttribute(k_bwd_lse, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_lse)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(k_bwd_dq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq)) != cudaSuccess ||
@@ -1289,9 +1388,9 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
         reinterpret_cast<float*>(ws + bl.lin_v), prm.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  k_bwd_dq<<<grid, kBwdThreads, smem_dq, stream>>>(tq, tk, tv, td, prm);
+  k_bwd_dq<<<grid, kDqThreads, smem_dq, stream>>>(tq, tk, tv, td, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  k_bwd_dkv<<<grid, kBwdThreads, smem_dkv, stream>>>(tq, tk, tv, td, prm);
+  k_bwd_dkv<<<grid, kDkvThreads, smem_dkv, stream>>>(tq, tk, tv, td, prm);
   return cudaGetLastError();
 }
 

@@ -497,7 +497,7 @@ def _time_w8a8(sba, torch, steps, warmup, M=75600, K=5120, N=5120):
 
 def backward_tensor_flops(B, H, nb, k):
     """Tensor-core FLOPs of the SLA backward's sparse branch: per kept (query block, key block)
-    pair nine 64x64x128 products (S and P.V again for the log-sum-exp; S, dP and dQ; S^T, dP^T,
+    pair nine 64x64x128 products (S and dP = dO V^T for the log-sum-exp and D; S, dP and dQ; S^T, dP^T,
     dV and dK), 2 FLOPs per multiply-add; plus the two complement GEMMs (G and dH), each
     2 nb_pad^2 16512 per head."""
     nb_pad = -(-nb // 128) * 128

@@ -114,3 +114,22 @@ def test_query_side_projection_vanishes():
         da = dnum @ g[:, :d].T + dden[:, None] * g[:, d][None, :]
         proj = (a * da).sum(axis=1)
         assert np.all(np.abs(proj) <= 1e-12 * (np.abs(a) @ np.abs(da).T).diagonal())
+
+
+def test_d_is_rowsum_of_p_times_dp():
+    """D = rowsum(dO * O_s) equals rowsum(P * dP) with dP = dO V^T (O_s = P V), the form the
+    GPU's log-sum-exp pass accumulates; checked on the oracle's forward state, per query block
+    over its kept tokens."""
+    n = 200
+    q, k, v, d_out, kept = _inputs(n, 17, 2)
+    _, st = sbo.sla_forward_head(q, k, v, kept)
+    for i in range(orc.n_blocks(n)):
+        rows = orc.block_rows(i, n)
+        toks = np.concatenate([np.arange(orc.block_rows(int(j), n).start,
+                                         orc.block_rows(int(j), n).stop)
+                               for j in sorted(int(x) for x in kept[i])])
+        s = (q[rows] @ k[toks].T) / math.sqrt(q.shape[1])
+        p = np.exp(s - st["lse"][rows][:, None])
+        d_def = (d_out[rows] * st["o_s"][rows]).sum(axis=1)
+        d_alt = (p * (d_out[rows] @ v[toks].T)).sum(axis=1)
+        np.testing.assert_allclose(d_alt, d_def, rtol=1e-12, atol=1e-12 * np.abs(d_def).max())

@@ -474,26 +474,32 @@ __device__ __forceinline__ void* grad_row(void* base, int32_t dtype, int64_t sb,
 // dQ of one query block over its kept key blocks: S = Q K^T and dP = dO V^T (M=64 N=64 each;
 // S in TMEM lanes 0-15 and dP in lanes 16-31 of each quadrant, double-buffered in columns
 // [0, 64) and [64, 128)), dS = P (dP - D) with P = 2^(S c - L), dQ += dS K (columns
-// [128, 256)). Role warps ordered by mbarriers: warps 0-3 the softmax (dS into the shared
-// tile), warp 4 issues S and warp 5 dP one block ahead, warp 6 dQ, warp 7 loads K and V of
-// each block into a two-stage ring, refilling a stage once the dQ of its block (the last
-// reader of K) has completed. The linear-branch dq is added before the store.
+// [128, 256)). Role warps ordered by mbarriers: warps 0-3 the softmax (dS into two shared
+// tiles, so that storing dS of block n waits only for the dQ of block n - 2), warp 4 issues S
+// and warp 5 dP one block ahead, warp 6 dQ, warp 7 loads K and V of each block into a
+// two-stage ring, refilling a stage once the dQ of its block (the last reader of K) has
+// completed. The tiles take 112 KB (dynamic shared memory declared 1024-byte aligned and
+// checked, as in k_bwd_dkv). The linear-branch dq is added before the store.
 constexpr int kDqThreads = 256;
 
 __global__ void __launch_bounds__(kDqThreads, 2)
 k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
          BwdParams prm) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint8_t* q_t = smem;                   // Q tile
-  uint8_t* o_t = smem + kTile;           // dO tile
-  uint8_t* k_t = smem + 2 * kTile;       // 2 K stages
-  uint8_t* v_t = smem + 4 * kTile;       // 2 V stages
-  uint8_t* s_t = smem + 6 * kTile;       // dS tile
-  __shared__ uint64_t q_full, kv_full[2], s_done[2], s_free[2], ds_full, dq_done[2];
+  extern __shared__ __align__(1024) uint8_t smem_dq[];
+  uint8_t* q_t = smem_dq;                // Q tile
+  uint8_t* o_t = smem_dq + kTile;        // dO tile
+  uint8_t* k_t = smem_dq + 2 * kTile;    // 2 K stages
+  uint8_t* v_t = smem_dq + 4 * kTile;    // 2 V stages
+  uint8_t* s_t = smem_dq + 6 * kTile;    // 2 dS tiles
+  __shared__ uint64_t q_full, kv_full[2], s_done[2], s_free[2], ds_full[2], dq_done[2];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
+
+  if (smem_u32(smem_dq) & 1023u) {           // same for every thread of the CTA
+    if (threadIdx.x == 0) record_error(prm.status, SAGESLA_ERR_DEVICE_CHECK);
+    return;
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x;
@@ -512,8 +518,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       mbar_init(&s_done[s], 2);          // the S and the dP commit of a block
       mbar_init(&s_free[s], 4);          // the four softmax warps have read S and dP
       mbar_init(&dq_done[s], 1);
+      mbar_init(&ds_full[s], 4);         // the four softmax warps have stored dS
     }
-    mbar_init(&ds_full, 4);              // the four softmax warps have stored dS
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -546,11 +552,11 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
   } else if (warp == 6) {
     // ------------------------------------------------ dQ issuer
     if (lane == 0) {
-      const uint32_t sa = smem_u32(s_t);
       for (int n = 0; n < U; ++n) {
-        ok = !abort_flag && mbar_wait(&ds_full, n & 1, prm.status);
+        ok = !abort_flag && mbar_wait(&ds_full[n & 1], (n >> 1) & 1, prm.status);
         if (!ok) break;
         tc_fence_after();
+        const uint32_t sa = smem_u32(s_t + (n & 1) * kPTile);
         const uint32_t kb = smem_u32(k_t + (n & 1) * kTile);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -613,16 +619,16 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
         ds[e] = p * (__uint_as_float(pr[e]) - dterm);
       }
-      // dQ of block n - 1 has read the dS tile
-      if (n >= 1) {
-        ok = !abort_flag && mbar_wait(&dq_done[(n - 1) & 1], ((n - 1) >> 1) & 1, prm.status);
+      // dQ of block n - 2 has read dS tile b
+      if (n >= 2) {
+        ok = !abort_flag && mbar_wait(&dq_done[b], ((n - 2) >> 1) & 1, prm.status);
         ok = __all_sync(0xffffffffu, ok) != 0;
         if (!ok) break;
       }
-      store_row_operand(s_t, row, kh, ds);
+      store_row_operand(s_t + b * kPTile, row, kh, ds);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_full);
+      if (lane == 0) mbar_arrive(&ds_full[b]);
     }
     if (ok) ok = mbar_wait(&dq_done[(U - 1) & 1], ((U - 1) >> 1) & 1, prm.status);
     ok = __all_sync(0xffffffffu, ok) != 0;
@@ -1341,7 +1347,7 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
   prm.H = static_cast<int>(p.H);
   const dim3 grid(static_cast<unsigned>(p.nb), static_cast<unsigned>(p.BH));
   const int smem_lse = 1024 + 6 * kTile;
-  const int smem_dq = 1024 + 6 * kTile + kPTile;
+  const int smem_dq = 6 * kTile + 2 * kPTile;
   const int smem_dkv = kDkvSmem;
   // set on every call: the attribute belongs to the current device
   if ((e = cudaFuncSetAttribute(k_bwd_lse, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_lse)) != cudaSuccess ||

@@ -41,6 +41,15 @@ namespace sagesla {
 
 namespace {
 
+
+// 2^x by the MUFU approximation (subnormal results flushed to zero): the probabilities here
+// are compared with a tolerance of 2^-5 of each gradient's magnitude
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kScale = 0.08838834764831845f;   // 1 / sqrt(128)
 constexpr uint32_t kTile = 64 * 128 * 2;         // one 64-row bf16 tile (two 8 KB d-chunks)
@@ -409,11 +418,11 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       }
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float m_new = fmaxf(m_run, mx);
-      const float alpha = exp2f(m_run - m_new);
+      const float alpha = ex2_approx(m_run - m_new);
       float rs = 0.f, pd = 0.f;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p = exp2f(x[e] - m_new);
+        const float p = ex2_approx(x[e] - m_new);
         rs += p;
         pd = fmaf(p, __uint_as_float(pr[e]), pd);
       }
@@ -616,7 +625,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       float ds[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p = exp2f(__uint_as_float(sr[e]) * c2 - l2);
+        const float p = ex2_approx(__uint_as_float(sr[e]) * c2 - l2);
         ds[e] = p * (__uint_as_float(pr[e]) - dterm);
       }
       // dQ of block n - 2 has read dS tile b
@@ -828,7 +837,7 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       float pt[32], ds[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        pt[e] = exp2f(__uint_as_float(sr[e]) * c2 - lq[e]);
+        pt[e] = ex2_approx(__uint_as_float(sr[e]) * c2 - lq[e]);
         ds[e] = pt[e] * (__uint_as_float(pr[e]) - dq_[e]);
       }
       // dV / dK of query block n - 1 have read the P^T and dS^T tiles

@@ -29,9 +29,9 @@
 //   k_bwd_dkv     per key block over the query blocks that keep it (compressed per-head lists
 //                 built from the kept bitmask): S^T, dP^T, dV, dK (role warps, a two-stage
 //                 Q / dO ring); adds the linear dk, dv
-// The linear branch runs on the CUDA cores (k_bwd_lin_query, k_bwd_lin_key) around one
-// complement GEMM on the tensor cores (dH = (1 - M)^T dG, the forward's GEMM on the
-// transposed mask).
+// The linear branch: k_bwd_lin_query and k_bwd_lin_key put their products over channels on
+// tcgen05 (the column-128 and rank-one terms on the CUDA cores), around one complement GEMM
+// (dH = (1 - M)^T dG, the forward's GEMM on the transposed mask).
 #include <cuda_bf16.h>
 
 #include "common.cuh"

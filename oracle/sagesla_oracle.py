@@ -217,43 +217,78 @@ def quant_v_fp8(v_head: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 # The two branches
 # --------------------------------------------------------------------------------------
 
-# The P-tile code is a floating-point decision (which e4m3 code 448 p rounds to). Both sides
-# take it in binary32 with one formula: in base-2 units with the factor 448 folded in,
-#   c = fl32(fl32(sq_i * L) * sk_j),  L = fl32(fl32(log2 e) * fl32(1/sqrt(128)))
-#   m = max over the keys seen so far of fl32(S_max * c)        (running, per 64-key block)
-#   x = fl32(S * c + fl32(log2(448) - m))                        (one rounding, as an FMA)
-#   code = e4m3(2^x)
-# 2^x itself is taken exactly here. A binary32 exp2 evaluation (relative error up to
-# EXP2_REL_ERR) can round a value that lies that close to an e4m3 midpoint to the neighbouring
-# code: those codes are ambiguous, and the oracle reports how much choosing the other code
-# could change each output element (``o_s_ambig``). The row sums and the accumulation stay in
-# float64.
-P_LOG2_SCALE = np.float32(np.float32(1.4426950408889634) * np.float32(0.08838834764831845))
-P_LOG2_448 = np.float32(8.807354922057604)
+# The P tile holds e4m3(448 p) with p = e^{S - m'} (m' the running maximum after the block):
+# the oracle takes that code exactly, from the float64 value of 448 p. A kernel evaluates
+# 448 p in binary32 and through an approximate base-2 exponential, so where 448 p lies very
+# close to a rounding boundary of the e4m3 grid it may take the neighbouring code. The bound
+# on how far the kernel's value may sit from 448 p is a property of a binary32 evaluation of
+# the exponent, independent of any particular kernel:
+#   x = S c + (log2 448 - m)      with c = sq sk log2(e) / sqrt(128) and m = m' log2(e),
+# formed with at most nine binary32 roundings (the constant c from its four factors, the
+# block maximum times c, the difference with log2 448, one fused multiply-add), each of
+# relative size at most u = 2^-24 of the quantity rounded, gives
+#   |x - x_exact| <= u (6 |S c| + 8 |m| + 27)           (base-2 units),
+# and the exponential itself adds a relative error eps_exp. In natural-log units (s = S c
+# ln 2, the logit; m' the running maximum) the relative distance of the kernel's value from
+# 448 p is therefore at most
+#   w = 2^-21 (|s| + |m'| + 3) + eps_exp,
+# with room to spare (8u per unit of |s| and |m'|, and 24u for the constant terms). A code is
+# *ambiguous* when 448 p (1 - w) and 448 p (1 + w) round to different e4m3 values; the oracle
+# reports, per output element, how much choosing the other code could change it, and how much
+# the row sum l can move when every p carries its window.
+EXP2_REL_ERR = 2.0 ** -20        # eps_exp: the kernel's 2^x (a few units in the last place)
 
 
-def p_codes_binary32(s_int: np.ndarray, sq_i, sk_j, m_run32: np.ndarray):
-    """e4m3 values of the P tile (448 p) decided in binary32; returns (values, new m32, and
-    the exact 2^x that was rounded)."""
-    c = np.float32(np.float32(sq_i) * P_LOG2_SCALE) * np.float32(sk_j)
-    mx = (s_int.max(axis=1).astype(np.float32) * c).astype(np.float32)
-    m_new = np.maximum(m_run32, mx).astype(np.float32)
-    neg = (P_LOG2_448 - m_new).astype(np.float32)
-    # S * c is exact in float64 (|S| < 2^22, 24-bit c); one rounding to binary32 like an FMA
-    x = (s_int.astype(np.float64) * np.float64(c) + neg.astype(np.float64)[:, None]).astype(np.float32)
-    y = np.exp2(x.astype(np.float64))
-    return round_e4m3(y), m_new, y
+def p_code_window(s: np.ndarray, m_new: np.ndarray, exp_rel_err: float = EXP2_REL_ERR):
+    """Relative window w around 448 p for logits s [nq, nk] and running maxima m_new [nq]."""
+    return 2.0 ** -21 * (np.abs(s) + np.abs(m_new)[:, None] + 3.0) + exp_rel_err
 
 
-EXP2_REL_ERR = 1e-6
-
-
-def e4m3_ambiguity(y: np.ndarray, rel: float = EXP2_REL_ERR) -> np.ndarray:
-    """|code change| (as a value) when y, perturbed by up to rel relative, can round to the
-    neighbouring e4m3 value instead; 0 where the rounding is unambiguous."""
+def e4m3_ambiguity(y: np.ndarray, rel) -> np.ndarray:
+    """|code change| (as a value) when y, perturbed by up to rel relative (a scalar or an
+    array shaped like y), can round to the neighbouring e4m3 value instead; 0 where the
+    rounding is unambiguous."""
     lo = round_e4m3(y * (1.0 - rel))
     hi = round_e4m3(y * (1.0 + rel))
-    return np.maximum(np.abs(hi - round_e4m3(y)), np.abs(round_e4m3(y) - lo))
+    r = round_e4m3(y)
+    return np.maximum(np.abs(hi - r), np.abs(r - lo))
+
+
+def online_softmax_p8(blocks, exp_rel_err: float = EXP2_REL_ERR):
+    """The online loop of the sparse branch with the P tile in e4m3 (SPEC section 6).
+
+    ``blocks``: the kept key blocks in ascending order, each a pair (s, v8) of the logits
+    s [nq, nk] (float64, natural-log units) and the decoded V codes v8 [nk, D] of its keys.
+    For each block: m' = max(m, rowmax s); alpha = e^{m - m'} (0 while m = -inf);
+    p = e^{s - m'}; l <- alpha l + sum p (unquantized p); o <- alpha o + e4m3(448 p) . v8;
+    m <- m'. Returns (o [nq, D], l [nq], amb [nq, D], lw [nq]): amb bounds the change of o
+    from ambiguous codes (sum of the alternative code's distance times |v8|), and lw = the
+    same recurrence as l with every p weighted by its window w, so that lw / l bounds the
+    relative error of a row sum formed from values within their windows."""
+    nq = blocks[0][0].shape[0]
+    d = blocks[0][1].shape[1]
+    m = np.full(nq, -np.inf)
+    l = np.zeros(nq)
+    lw = np.zeros(nq)
+    o = np.zeros((nq, d))
+    amb = np.zeros((nq, d))
+    for s, v8 in blocks:
+        m_new = np.maximum(m, s.max(axis=1))
+        alpha = np.where(np.isneginf(m), 0.0, np.exp(m - m_new))
+        p = np.exp(s - m_new[:, None])
+        w = p_code_window(s, m_new, exp_rel_err)
+        y = E4M3_MAX * p
+        l = alpha * l + p.sum(axis=1)
+        lw = alpha * lw + (p * w).sum(axis=1)
+        o = alpha[:, None] * o + round_e4m3(y) @ v8
+        amb = alpha[:, None] * amb + e4m3_ambiguity(y, w) @ np.abs(v8)
+        m = m_new
+    return o, l, amb, lw
+
+
+def sparse_output(o: np.ndarray, l: np.ndarray, s_v: np.ndarray) -> np.ndarray:
+    """O_s = o s_v / (448 l): the P codes carry the scale 1/448, the V codes s_v per channel."""
+    return o * (np.asarray(s_v, dtype=np.float64)[None, :] / (E4M3_MAX * l[:, None]))
 
 
 def phi(x: np.ndarray) -> np.ndarray:
@@ -333,44 +368,44 @@ def key_block_states(k: np.ndarray, v: np.ndarray) -> np.ndarray:
 def sparse_block_row(prep: HeadPrep, i: int, q, k, v, quant: bool = True,
                      smooth_in_quant_off: bool = False, return_ambiguity: bool = False):
     """Sparse branch for the real query tokens of block i: online softmax over kept(i) in
-    ascending order, running max updated per key block (no lazy rescale)."""
+    ascending order, running max updated per key block (no lazy rescale).
+
+    With ``return_ambiguity`` also returns, per output element, the bound on what a kernel
+    may differ by through ambiguous P codes and the window of the row sum (zero with
+    quantization off)."""
     n = prep.n
     qrows = block_rows(i, n)
+    inv_sqrt_d = 1.0 / math.sqrt(q.shape[1])
+    if quant:
+        blocks = []
+        for j in prep.kept[i]:
+            krows = block_rows(int(j), n)
+            s_int = prep.q8[qrows].astype(np.float64) @ prep.k8[krows].astype(np.float64).T
+            blocks.append((s_int * (float(prep.sq[i]) * float(prep.sk[j])) * inv_sqrt_d,
+                           prep.v8[krows]))
+        o, l, amb, lw = online_softmax_p8(blocks)
+        o_s = sparse_output(o, l, prep.s_v)
+        if return_ambiguity:
+            return o_s, sparse_output(amb, l, prep.s_v) + np.abs(o_s) * (lw / l)[:, None]
+        return o_s
     nq = qrows.stop - qrows.start
     d = q.shape[1]
     m = np.full(nq, -np.inf)
-    m32 = np.full(nq, -np.inf, dtype=np.float32)
     l = np.zeros(nq)
     o = np.zeros((nq, d))
-    amb = np.zeros((nq, d))          # bound on |o| change from ambiguous P codes
-    inv_sqrt_d = 1.0 / math.sqrt(d)
-    if not quant and smooth_in_quant_off:
+    if smooth_in_quant_off:
         k_used = k - smoothing_mean(k)[None, :]
     else:
         k_used = k
     for j in prep.kept[i]:
         krows = block_rows(int(j), n)
-        if quant:
-            s_int = prep.q8[qrows].astype(np.float64) @ prep.k8[krows].astype(np.float64).T
-            s = s_int * (float(prep.sq[i]) * float(prep.sk[j])) * inv_sqrt_d
-        else:
-            s = (q[qrows] @ k_used[krows].T) * inv_sqrt_d
+        s = (q[qrows] @ k_used[krows].T) * inv_sqrt_d
         m_new = np.maximum(m, s.max(axis=1))
         alpha = np.where(np.isneginf(m), 0.0, np.exp(m - m_new))
         p = np.exp(s - m_new[:, None])
         l = alpha * l + p.sum(axis=1)
-        if quant:
-            p8, m32, y32 = p_codes_binary32(s_int, prep.sq[i], prep.sk[j], m32)
-            o = alpha[:, None] * o + p8 @ prep.v8[krows]
-            amb = alpha[:, None] * amb + e4m3_ambiguity(y32) @ np.abs(prep.v8[krows])
-        else:
-            o = alpha[:, None] * o + p @ v[krows]
+        o = alpha[:, None] * o + p @ v[krows]
         m = m_new
-    if quant:
-        scale = prep.s_v.astype(np.float64)[None, :] / (E4M3_MAX * l[:, None])
-        if return_ambiguity:
-            return o * scale, amb * scale
-        return o * scale
     if return_ambiguity:
         return o / l[:, None], np.zeros_like(o)
     return o / l[:, None]

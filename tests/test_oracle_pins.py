@@ -259,36 +259,103 @@ def test_quantized_forward_is_close_to_exact():
     assert 1e-4 < err < 0.08
 
 
-def test_p_code_decision_in_binary32_matches_float64_away_from_midpoints():
-    """The P-tile codes decided in binary32 differ from the float64 decision e4m3(448 p) only
-    where 448 p lies within 1e-5 (relative) of a rounding midpoint of the e4m3 grid."""
+def _golden_two_blocks():
+    rows, cur, s_v = {}, None, None
+    for line in open(os.path.join(GOLDEN, "p8_two_blocks.txt")):
+        f = line.split()
+        if not f or f[0].startswith("#"):
+            continue
+        if f[0] == "s_v":
+            s_v = np.array([float(x) for x in f[1:]])
+        elif f[0] == "row":
+            cur = rows.setdefault(f[1], {"blocks": []})
+        elif f[0] == "block":
+            cur["blocks"].append([])
+        elif f[0] == "key":
+            cur["blocks"][-1].append((float(f[1]), int(f[2])))
+        elif f[0] == "expect_l":
+            cur["l"] = float(f[1])
+        elif f[0] == "expect_o":
+            cur["o"] = np.array([float(x) for x in f[1:]])
+    return rows, s_v
+
+
+def test_online_loop_golden_two_blocks():
+    """The hand-derived two-block rows of tests/golden/p8_two_blocks.txt: codes against the
+    running maximum of each block, the row sum of the unquantized p, the 1/448 and s_v
+    scales. Row A fails if codes are taken against the final maximum or l sums the codes;
+    row B fails if codes are taken against each block's own maximum."""
+    rows, s_v = _golden_two_blocks()
+    for name, r in rows.items():
+        blocks = []
+        for keys in r["blocks"]:
+            s = np.array([[lg for lg, _ in keys]])
+            v8 = np.zeros((len(keys), s_v.size))
+            for u, (_, ch) in enumerate(keys):
+                v8[u, ch] = 1.0
+            blocks.append((s, v8))
+        o, l, amb, lw = orc.online_softmax_p8(blocks)
+        assert abs(l[0] - r["l"]) <= 1e-13, (name, l)
+        np.testing.assert_allclose(orc.sparse_output(o, l, s_v)[0], r["o"], rtol=0, atol=1e-13)
+        assert not amb.any(), name          # no code of the example is near a midpoint
+        assert 0 < lw[0] / l[0] < 1e-5
+
+
+def _binary32_codes(s_blocks, sq, sk_list, eps, rng):
+    """An independent binary32 evaluation of the P codes (the way a kernel forms them): the
+    exponent in base 2 with the factor 448 folded in, from a float32 constant, a float32 running
+    maximum and one fused rounding, then 2^x with a random relative error of up to eps."""
+    L = np.float32(np.float32(1.4426950408889634) * np.float32(1.0 / math.sqrt(128.0)))
+    lg448 = np.float32(math.log2(448.0))
+    m32 = np.full(s_blocks[0].shape[0], -np.inf, dtype=np.float32)
+    out = []
+    for s_int, sk in zip(s_blocks, sk_list):
+        c = np.float32(np.float32(np.float32(sq) * L) * np.float32(sk))
+        mx = (s_int.max(axis=1).astype(np.float32) * c).astype(np.float32)
+        m32 = np.maximum(m32, mx)
+        neg = (lg448 - m32).astype(np.float32)
+        x = (s_int.astype(np.float64) * np.float64(c) + neg.astype(np.float64)[:, None]).astype(np.float32)
+        y = np.exp2(x.astype(np.float64)) * (1.0 + rng.uniform(-eps, eps, x.shape))
+        out.append(orc.round_e4m3(y))
+    return out
+
+
+@pytest.mark.parametrize("scale,offset", [(1.0, 0), (30.0, 0), (30.0, 190000)])
+def test_p_code_window_covers_a_binary32_evaluation(scale, offset):
+    """Wherever a binary32 evaluation (written here, not in the oracle) picks another e4m3 code
+    than the oracle's exact e4m3(448 p), the oracle's window marks that code ambiguous; and the
+    window is narrow (few codes ambiguous). Three blocks in sequence, so that the running
+    maximum moves; ordinary logits, large logits, and large logits close to each other (many
+    codes near the top of the grid computed from large binary32 operands)."""
     rng = np.random.default_rng(16)
-    grid = orc.e4m3_decode(np.arange(0, 127))
-    mids = (grid[:-1] + grid[1:]) / 2
-    checked = flips = 0
-    for trial in range(40):
-        s_int = rng.integers(-30000, 30000, size=(64, 64))
-        sq, sk = np.float32(rng.uniform(0.01, 0.5)), np.float32(rng.uniform(0.01, 0.5))
-        m0 = np.full(64, -np.inf, dtype=np.float32)
-        p8, m32, _ = orc.p_codes_binary32(s_int, sq, sk, m0)
-        s = s_int * (float(sq) * float(sk)) / math.sqrt(128)
-        y = 448.0 * np.exp(s - s.max(axis=1, keepdims=True))
-        ref = orc.round_e4m3(y)
-        near = np.min(np.abs(y[..., None] - mids[None, None, :]), axis=-1) <= 1e-5 * y
-        diff = p8 != ref
-        assert not np.any(diff & ~near)
-        checked += diff.size
-        flips += int(diff.sum())
-        # the running maximum is the binary32 image of the row maximum
-        np.testing.assert_allclose(m32, s.max(axis=1) * math.log2(math.e), rtol=1e-6)
-    assert flips < checked * 1e-3
+    flagged = total = differ = 0
+    for trial in range(30):
+        sq = np.float32(rng.uniform(0.005, 0.05) * scale)
+        sks = [np.float32(rng.uniform(0.005, 0.05)) for _ in range(3)]
+        spread = 3000 if offset else 127 * 127 * 12
+        s_ints = [offset + rng.integers(-spread, spread, size=(64, 64)) for _ in range(3)]
+        ref_codes = _binary32_codes(s_ints, sq, sks, 2.0 ** -21, rng)
+        m = np.full(64, -np.inf)
+        for s_int, sk, code32 in zip(s_ints, sks, ref_codes):
+            s = s_int * (float(sq) * float(sk)) / math.sqrt(128.0)
+            m = np.maximum(m, s.max(axis=1))
+            y = 448.0 * np.exp(s - m[:, None])
+            amb = orc.e4m3_ambiguity(y, orc.p_code_window(s, m))
+            differs = code32 != orc.round_e4m3(y)
+            assert not np.any(differs & (amb == 0))
+            flagged += int((amb > 0).sum())
+            differ += int(differs.sum())
+            total += amb.size
+    assert flagged < 2e-2 * total
+    if offset:
+        assert differ > 0        # the case does move codes: the window is exercised
 
 
 def test_e4m3_ambiguity_bound():
     """Zero away from midpoints; exactly one grid step at a midpoint."""
     grid = orc.e4m3_decode(np.arange(0, 127))
     mids = (grid[:-1] + grid[1:]) / 2
-    amb = orc.e4m3_ambiguity(mids)
+    amb = orc.e4m3_ambiguity(mids, 1e-6)
     np.testing.assert_allclose(amb, np.diff(grid))
-    off = orc.e4m3_ambiguity(grid[1:])           # on the grid: unambiguous
+    off = orc.e4m3_ambiguity(grid[1:], 1e-6)     # on the grid: unambiguous
     assert not off.any()

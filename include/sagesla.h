@@ -77,6 +77,16 @@ typedef struct {
    * and key-block states, statistics finalize, quantization, block scores, Top-K selection,
    * complement sums (skipped when every block is kept), sparse attention + linear branch. */
   void** stage_events;
+  /* Test hooks of the failure path; leave both 0 in normal use.
+   *   debug_spin_limit_us > 0 replaces the 2 s limit of every wait of the attention kernel by
+   *   that many microseconds for this call.
+   *   debug_skip_tile = 1 makes the attention kernel's first CTA skip one tile load (and the
+   *   byte count announced for it), so that the waits for that tile run out: the call then
+   *   ends normally with SAGESLA_ERR_TIMEOUT in the workspace's status word and that CTA's
+   *   output rows unwritten. Nothing is left in flight, and the next call on the same
+   *   workspace starts clean. */
+  uint32_t debug_spin_limit_us;
+  int32_t debug_skip_tile;
 } sagesla_options;
 
 #define SAGESLA_N_STAGES 7
@@ -174,7 +184,9 @@ sagesla_status sagesla_forward_host(const uint16_t* q_host, const uint16_t* k_ho
  *   - Problems whose sagesla_workspace_size() exceeds SAGESLA_NO_ALLOC_SCRATCH_BYTES are
  *     rejected with SAGESLA_ERR_WORKSPACE before anything is launched.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current); make that first call before any stream capture.
+ *     with that device current); make that first call before any stream capture. The address
+ *     is kept until the process exits: after a cudaDeviceReset of that device it is stale, so
+ *     do not use this call on a device after resetting it.
  *   - Every call shares the one array, which keeps the last call's contents; calls whose GPU
  *     work overlaps (different streams, or threads without ordering) race on it.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.

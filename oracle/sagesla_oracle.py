@@ -223,25 +223,28 @@ def quant_v_fp8(v_head: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 # close to a rounding boundary of the e4m3 grid it may take the neighbouring code. The bound
 # on how far the kernel's value may sit from 448 p is a property of a binary32 evaluation of
 # the exponent, independent of any particular kernel:
-#   x = S c + (log2 448 - m)      with c = sq sk log2(e) / sqrt(128) and m = m' log2(e),
-# formed with at most nine binary32 roundings (the constant c from its four factors, the
-# block maximum times c, the difference with log2 448, one fused multiply-add), each of
-# relative size at most u = 2^-24 of the quantity rounded, gives
-#   |x - x_exact| <= u (6 |S c| + 8 |m| + 27)           (base-2 units),
+#   x = S c + (log2 448 - m)      c = sq sk log2(e) / sqrt(128),  m = m' log2(e).
+# The factor of c common to all blocks of a row (sq log2(e) / sqrt(128)) is rounded at most
+# four times; that common relative error scales every exponent of the row alike, so it moves
+# x by at most 4u |S c - m|. Each block's c takes one more rounding (u |S c|), the block
+# maximum times c one and the running maximum is one of those (2u |m|), the difference with
+# log2 448 two (u (2 log2 448 + |m|)) and the fused multiply-add one (u |x|). With u = 2^-24:
+#   |x - x_exact| <= u (5 |S c - m| + |S c| + 3 |m| + 27)     (base-2 units),
 # and the exponential itself adds a relative error eps_exp. In natural-log units (s = S c
 # ln 2, the logit; m' the running maximum) the relative distance of the kernel's value from
 # 448 p is therefore at most
-#   w = 2^-21 (|s| + |m'| + 3) + eps_exp,
-# with room to spare (8u per unit of |s| and |m'|, and 24u for the constant terms). A code is
-# *ambiguous* when 448 p (1 - w) and 448 p (1 + w) round to different e4m3 values; the oracle
-# reports, per output element, how much choosing the other code could change it, and how much
-# the row sum l can move when every p carries its window.
+#   w = 2^-21 (|s - m'| + (|s| + 3 |m'|) / 4 + 3) + eps_exp,
+# a factor of two or more above each term (2^-21 = 8u). A code is *ambiguous* when
+# 448 p (1 - w) and 448 p (1 + w) round to different e4m3 values; the oracle reports, per
+# output element, how much choosing the other code could change it, and how much the row sum l
+# can move when every p carries its window.
 EXP2_REL_ERR = 2.0 ** -20        # eps_exp: the kernel's 2^x (a few units in the last place)
 
 
 def p_code_window(s: np.ndarray, m_new: np.ndarray, exp_rel_err: float = EXP2_REL_ERR):
     """Relative window w around 448 p for logits s [nq, nk] and running maxima m_new [nq]."""
-    return 2.0 ** -21 * (np.abs(s) + np.abs(m_new)[:, None] + 3.0) + exp_rel_err
+    m = m_new[:, None]
+    return 2.0 ** -21 * (np.abs(s - m) + (np.abs(s) + 3.0 * np.abs(m)) / 4.0 + 3.0) + exp_rel_err
 
 
 def e4m3_ambiguity(y: np.ndarray, rel) -> np.ndarray:

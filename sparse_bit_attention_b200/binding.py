@@ -47,7 +47,8 @@ STAGE_NAMES = ["stats", "finalize", "quant", "scores", "topk", "complement_gemm"
 class SageslaOptions(ctypes.Structure):
     _fields_ = [("kept_idx_out", ctypes.c_void_p), ("mask_out", ctypes.c_void_p),
                 ("scores_out", ctypes.c_void_p), ("sparse_out", ctypes.c_void_p),
-                ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p)),
+                ("debug_spin_limit_us", ctypes.c_uint32), ("debug_skip_tile", ctypes.c_int32)]
 
 
 _LAYOUT_FIELDS = ["status", "q8", "k8", "v8", "sq", "sk", "s_v", "inv_v", "mu", "qbar", "kbar",
@@ -196,11 +197,14 @@ def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_rati
                     block: int = BLOCK, out: torch.Tensor | None = None,
                     workspace: torch.Tensor | None = None, stream=None,
                     out_dtype: torch.dtype = torch.float32, kept_idx_out=None, mask_out=None,
-                    scores_out=None, sparse_out=None, stage_events=None) -> torch.Tensor:
+                    scores_out=None, sparse_out=None, stage_events=None,
+                    debug_spin_limit_us: int = 0, debug_skip_tile: bool = False) -> torch.Tensor:
     """SageSLA forward on device tensors q, k, v (bf16 [B, H, N, 128]); returns ``out``.
 
     ``stage_events``: optional list of N_STAGES + 1 torch.cuda.Event(enable_timing=True)
-    recorded around each kernel of the forward on the launching stream."""
+    recorded around each kernel of the forward on the launching stream.
+    ``debug_spin_limit_us`` / ``debug_skip_tile``: the failure-path test hooks of
+    sagesla_options (0 / False in normal use)."""
     lib = load_library()
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
@@ -213,8 +217,11 @@ def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_rati
     args = (ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), float(topk_ratio), int(block),
             ctypes.byref(vo), ctypes.c_void_p(workspace.data_ptr()),
             workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_ptr(stream)))
-    if any(x is not None for x in extra) or stage_events is not None:
+    if (any(x is not None for x in extra) or stage_events is not None or debug_spin_limit_us
+            or debug_skip_tile):
         opt = SageslaOptions(*[None if x is None else x.data_ptr() for x in extra])
+        opt.debug_spin_limit_us = int(debug_spin_limit_us)
+        opt.debug_skip_tile = 1 if debug_skip_tile else 0
         if stage_events is not None:
             if len(stage_events) != N_STAGES + 1:
                 raise ValueError(f"stage_events needs {N_STAGES + 1} events")

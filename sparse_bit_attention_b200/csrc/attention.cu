@@ -130,12 +130,14 @@ struct AttnParams {
   int* status;
   int N, nb, nbq, n_pad, k, nb_m_pad, n_last;
   int linear;                 // 0 when every key block is kept
+  unsigned long long spin_ns; // limit of every wait (a shorter one only in failure-path tests)
+  int skip_tile;              // failure-path test: CTA (0, 0) never loads its first K8 pair
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ctl* ctl,
-                                              int* status) {
+                                              int* status, unsigned long long limit_ns) {
   if (ctl->abort) return false;
-  if (!mbar_wait(bar, parity, status)) {
+  if (!mbar_wait(bar, parity, status, limit_ns)) {
     ctl->abort = 1;
     return false;
   }
@@ -308,9 +310,12 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int h = 0; h < 2 && ok; ++h) {
           if (n0 >= U[h]) continue;
           HalfCtl& c = ctl->hc[h];
-          if (n0 > 0 && !(ok = wait_or_abort(&c.s_full, ((n0 >> 1) - 1) & 1, ctl, status))) break;
+          if (n0 > 0 && !(ok = wait_or_abort(&c.s_full, ((n0 >> 1) - 1) & 1, ctl, status, prm.spin_ns))) break;
           const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) : nullptr;
           const int two = n0 + 1 < U[h] ? 2 : 1;
+          // Failure-path test: the first pair of CTA (0, 0) is never loaded, so the waits for
+          // it run out (nothing is left in flight: neither its bytes nor its copies exist).
+          if (prm.skip_tile && n0 == 0 && h == 0 && pair == 0 && bh == 0) continue;
           mbar_arrive_expect_tx(&c.k_full, two * kKVBytes);
           uint8_t* kst = smem + h * kHalfBytes + kHK;
           tma_load_2d(kst, &tm_k, &c.k_full, 0, row_base + 64 * kept_at(ctl, h, klist, n0));
@@ -322,7 +327,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (n >= U[h]) continue;
             HalfCtl& c = ctl->hc[h];
             const int s = n % kNV;
-            if (n >= kNV && !(ok = wait_or_abort(&c.v_empty[s], ((n / kNV) - 1) & 1, ctl, status))) break;
+            if (n >= kNV && !(ok = wait_or_abort(&c.v_empty[s], ((n / kNV) - 1) & 1, ctl, status, prm.spin_ns))) break;
             const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) : nullptr;
             mbar_arrive_expect_tx(&c.v_full[s], kKVBytes);
             tma_load_2d(smem + h * kHalfBytes + kHV + s * kKVBytes, &tm_v, &c.v_full[s], 0,
@@ -333,7 +338,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       for (int h = 0; h < 2 && ok && prm.linear; ++h) {
         if (U[h] == 0) continue;
         HalfCtl& c = ctl->hc[h];
-        if (!(ok = wait_or_abort(&c.mma_done, 0, ctl, status))) break;
+        if (!(ok = wait_or_abort(&c.mma_done, 0, ctl, status, prm.spin_ns))) break;
         const int gy = static_cast<int>((bh * prm.nb_m_pad + ia + h) * 129);
         uint8_t* hb = smem + h * kHalfBytes;
         mbar_arrive_expect_tx(&c.g_full, 32768u);
@@ -349,7 +354,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       constexpr uint32_t idesc_l = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 64, 128);
       bool ok = true;
       for (int h = 0; h < 2 && ok; ++h)
-        if (U[h] > 0) ok = wait_or_abort(&ctl->hc[h].q_full, 0, ctl, status);
+        if (U[h] > 0) ok = wait_or_abort(&ctl->hc[h].q_full, 0, ctl, status, prm.spin_ns);
       // Q rows and K pair descriptors; the K-steps of 32 bytes add 2 to the address field.
       uint64_t dq[2], dk[2];
 #pragma unroll
@@ -364,8 +369,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           if (n0 >= U[h]) continue;
           HalfCtl& c = ctl->hc[h];
           const int p = n0 >> 1;
-          if (!(ok = wait_or_abort(&c.k_full, p & 1, ctl, status))) break;
-          if (p > 0 && !(ok = wait_or_abort(&c.s_free, (p - 1) & 1, ctl, status))) break;
+          if (!(ok = wait_or_abort(&c.k_full, p & 1, ctl, status, prm.spin_ns))) break;
+          if (p > 0 && !(ok = wait_or_abort(&c.s_free, (p - 1) & 1, ctl, status, prm.spin_ns))) break;
           tc_fence_after();
           const uint32_t d = tmem + (static_cast<uint32_t>(16 * h) << 16) + kTmemS;
           mma_i8(d, dq[h], dk[h], idesc_s, 0u);
@@ -379,8 +384,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // phi(Q_i) . G_i into this half's S columns, once the loop's P.V are done
         if (U[h] == 0) continue;
         HalfCtl& c = ctl->hc[h];
-        if (!(ok = wait_or_abort(&c.mma_done, 0, ctl, status) && wait_or_abort(&c.a_full, 0, ctl, status) &&
-                   wait_or_abort(&c.g_full, 0, ctl, status))) break;
+        if (!(ok = wait_or_abort(&c.mma_done, 0, ctl, status, prm.spin_ns) && wait_or_abort(&c.a_full, 0, ctl, status, prm.spin_ns) &&
+                   wait_or_abort(&c.g_full, 0, ctl, status, prm.spin_ns))) break;
         tc_fence_after();
         const uint32_t dlane = static_cast<uint32_t>(16 * h) << 16;
         const uint32_t hb = smem_u32(smem + h * kHalfBytes);
@@ -407,8 +412,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       const uint32_t d = tmem + (static_cast<uint32_t>(16 * h) << 16);
       for (int n = 0; n < U[h]; ++n) {
         const int s = n % kNV;
-        if (!wait_or_abort(&c.p_full, n & 1, ctl, status)) break;
-        if (!wait_or_abort(&c.v_full[s], (n / kNV) & 1, ctl, status)) break;
+        if (!wait_or_abort(&c.p_full, n & 1, ctl, status, prm.spin_ns)) break;
+        if (!wait_or_abort(&c.v_full[s], (n / kNV) & 1, ctl, status, prm.spin_ns)) break;
         tc_fence_after();
         // P: K-major, no swizzle (layout above). V: MN-major (d contiguous), 128-byte
         // swizzle, 8-key groups 1024 B apart.
@@ -458,7 +463,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           j_cur = j_ahead;
           if (n + 2 < Uh) j_ahead = kept_block(klist, n + 2);
         }
-        if (b == 0 && !wait_or_abort(&c.s_full, (n >> 1) & 1, ctl, status)) { ok = false; break; }
+        if (b == 0 && !wait_or_abort(&c.s_full, (n >> 1) & 1, ctl, status, prm.spin_ns)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[32];
         tmem_ld16x64(tmem + lane16 + kTmemS + 64 * b, sr);
@@ -482,7 +487,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         m_run = m_new;
         // P.V(n-1) must be done: it frees P buffer b (read by P.V(n-2) before it), makes O
         // stable for the rescale, and orders the P.V MMAs issued from different warps.
-        if (n >= 1 && !wait_or_abort(&c.pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status)) { ok = false; break; }
+        if (n >= 1 && !wait_or_abort(&c.pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status, prm.spin_ns)) { ok = false; break; }
         tc_fence_after();
         uint8_t* pb = smem + kOffP + h * kPBytes + (r >> 3) * kPGroup + (r & 7) * 16 + 2 * kh * kPChunk;
         *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -512,7 +517,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncwarp();
         if (lane == 0) mbar_arrive(&c.p_full);
       }
-      if (ok) ok = wait_or_abort(&c.pv_done[(Uh - 1) & 1], ((Uh - 1) >> 1) & 1, ctl, status);
+      if (ok) ok = wait_or_abort(&c.pv_done[(Uh - 1) & 1], ((Uh - 1) >> 1) & 1, ctl, status, prm.spin_ns);
       tc_fence_after();
     }
 
@@ -579,7 +584,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.a_full);
-      ok = wait_or_abort(&c.l_done, 0, ctl, status);
+      ok = wait_or_abort(&c.l_done, 0, ctl, status, prm.spin_ns);
       tc_fence_after();
     }
     const float inv_l = 1.f / l448;
@@ -644,7 +649,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
 cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32_t out_dtype,
                              int64_t out_sb, int64_t out_sh, int64_t out_sn, float* sparse_out,
-                             char* ws, cudaStream_t stream) {
+                             char* ws, const AttnTestHooks& hooks, cudaStream_t stream) {
   const auto& L = p.lay;
   CUtensorMap tq, tk, tv, tg;
   const uint64_t rows = static_cast<uint64_t>(p.BH * p.n_pad);
@@ -680,15 +685,14 @@ cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32
   prm.nb_m_pad = static_cast<int>(p.nb_m_pad);
   prm.n_last = p.n_last;
   prm.linear = p.linear_empty ? 0 : 1;
+  prm.spin_ns = hooks.spin_limit_us ? 1000ull * hooks.spin_limit_us : kSpinLimitNs;
+  prm.skip_tile = hooks.skip_tile;
   // The register split (setmaxnreg) must fit the registers the CTA is launched with, or the
-  // softmax warps would wait for registers forever.
-  static int regs = -1;
-  if (regs < 0) {
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, k_attention) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
-    regs = fa.numRegs;
-  }
-  if (static_cast<uint32_t>(regs) * kThreads < 256 * kSoftmaxRegs + 128 * kHelperRegs)
+  // softmax warps would wait for registers forever. The count is a property of the loaded
+  // module; it is queried per call (cheap, and right for every device and thread).
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, k_attention) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+  if (static_cast<uint32_t>(fa.numRegs) * kThreads < 256 * kSoftmaxRegs + 128 * kHelperRegs)
     return cudaErrorInvalidConfiguration;
   const size_t smem = 1024 + kOffCtl + sizeof(Ctl);
   cudaError_t e = cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize,

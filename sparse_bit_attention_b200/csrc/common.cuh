@@ -80,15 +80,17 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete. Gives up after kSpinLimitNs,
-// records SAGESLA_ERR_TIMEOUT and returns false; never spins without bound.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+// Waits for the phase with the given parity to complete. Gives up after limit_ns
+// (kSpinLimitNs unless a caller passes a shorter limit), records SAGESLA_ERR_TIMEOUT and
+// returns false; never spins without bound.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+                                          unsigned long long limit_ns = kSpinLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kSpinLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       record_error(status, SAGESLA_ERR_TIMEOUT);
       return false;
     }

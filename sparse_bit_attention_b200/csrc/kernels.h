@@ -85,9 +85,14 @@ sagesla_status require_b200();
 
 cudaError_t launch_fill_all_kept(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_complement_gemm(const ForwardPlan& p, char* ws, cudaStream_t stream);
+// Failure-path test hooks of the attention kernel (zero in normal use).
+struct AttnTestHooks {
+  uint32_t spin_limit_us;   // > 0: limit of every wait instead of kSpinLimitNs
+  int32_t skip_tile;        // 1: the first CTA never loads its first K tile pair
+};
 cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32_t out_dtype,
                              int64_t out_sb, int64_t out_sh, int64_t out_sn, float* sparse_out,
-                             char* ws, cudaStream_t stream);
+                             char* ws, const AttnTestHooks& hooks, cudaStream_t stream);
 cudaError_t launch_scale_scores(const ForwardPlan& p, const char* ws, float* scores_out,
                                 cudaStream_t stream);
 

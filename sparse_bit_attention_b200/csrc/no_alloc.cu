@@ -10,7 +10,9 @@
 // In host code the array's name only stands in for it; a kernel handed that name would fault
 // (or, where the GPU can reach host memory, quietly use the wrong memory). The device address
 // is therefore looked up with cudaGetSymbolAddress once per device, with that device current,
-// on the first call made on the device.
+// on the first call made on the device, and kept for the life of the process. A
+// cudaDeviceReset unloads the module and makes that address stale; the library does not see
+// the reset, so this entry point must not be used on a device after it was reset.
 #include <mutex>
 
 #include "common.cuh"
@@ -56,8 +58,12 @@ extern "C" sagesla_status sagesla_forward_no_alloc(const sagesla_tensor* q,
     return SAGESLA_ERR_INVALID_ARG;
   }
   if (need > SAGESLA_NO_ALLOC_SCRATCH_BYTES) return SAGESLA_ERR_WORKSPACE;
+  // Same device check, and so the same status, as sagesla_forward before the symbol lookup
+  // (on a device that is not sm_100 the module cannot load and the lookup would fail).
+  sagesla_status st = sagesla::require_b200();
+  if (st != SAGESLA_OK) return st;
   void* scratch = nullptr;
-  const sagesla_status st = sagesla::scratch_address(&scratch);
+  st = sagesla::scratch_address(&scratch);
   if (st != SAGESLA_OK) return st;
   // The forward clears the only scratch word it reads before writing (its status word) at the
   // start of every call; everything else it writes before reading.

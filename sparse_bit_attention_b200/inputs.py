@@ -117,8 +117,10 @@ def make_qkv(name: str, n_tokens: int | None = None, heads: int | None = None):
 
 
 def make_random(B: int, H: int, N: int, seed: int, k_offset_std: float = 0.0,
-                scale: float = 1.0):
-    """Q, K, V ~ N(0, scale^2) bf16 [B, H, N, 128]; optional per-(b,h,channel) K offset."""
+                scale: float = 1.0, qk_scale: float = 1.0, v_mean_std: float = 0.0):
+    """Q, K, V ~ N(0, scale^2) bf16 [B, H, N, 128]; optional per-(b,h,channel) K offset
+    ~ N(0, k_offset_std^2); Q and K further multiplied by ``qk_scale`` (large logits); optional
+    per-(b,h,channel) V mean ~ N(0, v_mean_std^2), drawn after the K offset."""
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     shape = (B, H, N, HEAD_DIM)
@@ -127,6 +129,10 @@ def make_random(B: int, H: int, N: int, seed: int, k_offset_std: float = 0.0,
     v = torch.randn(shape, generator=g, dtype=torch.float32) * scale
     if k_offset_std:
         k = k + torch.randn((B, H, 1, HEAD_DIM), generator=g, dtype=torch.float32) * k_offset_std
+    if v_mean_std:
+        v = v + torch.randn((B, H, 1, HEAD_DIM), generator=g, dtype=torch.float32) * v_mean_std
+    if qk_scale != 1.0:
+        q, k = q * qk_scale, k * qk_scale
     return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
 
 

@@ -14,6 +14,19 @@ from sparse_bit_attention_b200 import inputs
 OUT_TOL = 2e-3          # max |out_gpu - out_oracle|, fp32 output
 MARGIN = orc.AMBIGUOUS_MARGIN
 
+# Linear branch tolerance, per element: the GPU rounds four operands to bf16 on the way to
+# O_l (phi(k), H_j, G_i, phi(q); relative 2^-9 each), and every term of the numerator and of
+# the denominator is positive in phi, so to first order
+#   |O_l,gpu - O_l| <= 4 * 2^-9 * (A + |O_l|),  A = the linear branch of |V| (same weights),
+# plus the fp32 sums (about 2^-12 relative over a few thousand terms) and an absolute floor.
+# With V ~ N(0, 1) (the benchmark workloads) O_l is a few 1e-3 and the plain output gate
+# OUT_TOL covers it; inputs whose O_l is of order one add this bound to the output gate.
+LIN_REL = 4 * 2.0 ** -9 + 2.0 ** -12
+LIN_ABS = 1e-6
+
+# The two parts of the last compare_head result (output, sparse-branch output), for messages.
+LAST_ERRS = {}
+
 
 def _ws_slice(ws: torch.Tensor, off: int, count: int, dtype: torch.dtype) -> torch.Tensor:
     nbytes = count * torch.empty((), dtype=dtype).element_size()
@@ -98,9 +111,12 @@ def check_mask(prep, gpu_kept: list) -> int:
     return ambiguous
 
 
-def compare_head(q, k, v, ratio, res, b: int, h: int, rows=None, check_codes=True):
+def compare_head(q, k, v, ratio, res, b: int, h: int, rows=None, check_codes=True,
+                 linear_tol=False):
     """Oracle vs GPU for one head: codes (bit-exact), mask, and the output of the query blocks
-    in ``rows`` (default all). Returns (max abs error, ambiguous rows)."""
+    in ``rows`` (default all). Returns (max abs error, ambiguous rows): the largest amount by
+    which an element exceeds its allowance (ambiguous P codes and the row-sum window; with
+    ``linear_tol`` also the linear branch's bf16 bound) before the OUT_TOL gate."""
     B, H, N, D = q.shape
     bh = b * H + h
     qh, kh, vh = (inputs.as_float64(x[b, h]) for x in (q, k, v))
@@ -123,14 +139,24 @@ def compare_head(q, k, v, ratio, res, b: int, h: int, rows=None, check_codes=Tru
         assert not wc["q8"][N:].any() and not wc["k8"][N:].any() and not wc["v8"][N:].any()
     # err: max over elements of |gpu - oracle| minus the bound of what ambiguous P codes
     # (values within the exp2 approximation error of an e4m3 midpoint) could change
+    LAST_ERRS.clear()
+    h_abs = orc.key_block_states(kh, np.abs(vh)) if linear_tol else None
     err = 0.0
     for i, r in out.items():
         sl = orc.block_rows(i, N)
         g = res["out"][b, h, sl].double().numpy()
         assert np.isfinite(g).all(), f"non-finite output in block {i}"
-        err = max(err, float(np.max(np.abs(g - r["o"]) - r["o_s_ambig"])))
+        allow = r["o_s_ambig"]
+        if linear_tol:
+            mag = orc.linear_block_row(prep, i, qh, h_abs)
+            allow = allow + LIN_REL * (mag + np.abs(r["o_l"])) + LIN_ABS
+        e_out = float(np.max(np.abs(g - r["o"]) - allow))
+        LAST_ERRS["out"] = max(LAST_ERRS.get("out", -np.inf), e_out)
+        err = max(err, e_out)
         if "sparse" in res:
             gs = res["sparse"][b, h, sl].double().numpy()
             assert np.isfinite(gs).all(), f"non-finite sparse-branch output in block {i}"
-            err = max(err, float(np.max(np.abs(gs - r["o_s"]) - r["o_s_ambig"])))
+            e_sp = float(np.max(np.abs(gs - r["o_s"]) - r["o_s_ambig"]))
+            LAST_ERRS["sparse"] = max(LAST_ERRS.get("sparse", -np.inf), e_sp)
+            err = max(err, e_sp)
     return err, ambiguous

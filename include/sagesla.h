@@ -87,7 +87,24 @@ typedef struct {
    *   workspace starts clean. */
   uint32_t debug_spin_limit_us;
   int32_t debug_skip_tile;
+  /* Operand precision of the sparse branch (news.qq.com TurboDiffusion article, section
+   * 从训练到部署: SLA without the low-bit quantization is the attention that is fine-tuned;
+   * SageSLA, SLA plus SageAttention's 8-bit operands, replaces it at inference).
+   *   quant = 1, pv_fp8 = 1: INT8 Q.K^T (smoothed K, per-block scales), e4m3 P and V (the
+   *                          SageSLA forward);
+   *   quant = 1, pv_fp8 = 0: INT8 Q.K^T, P rounded to bf16 times the raw bf16 V;
+   *   quant = 0, pv_fp8 = 0: bf16 Q.K^T and bf16 P.V (the unquantized SLA forward, the one
+   *                          sagesla_sla_backward differentiates).
+   * quant = 0 with pv_fp8 = 1 is rejected (SAGESLA_ERR_UNSUPPORTED), other values
+   * (SAGESLA_ERR_INVALID_ARG). sagesla_options_init sets both to 1; a zero-filled struct
+   * selects the unquantized forward. The 16-bit modes need a larger workspace
+   * (sagesla_workspace_size_ex with the same options) and run one CTA per SM. */
+  int32_t quant;
+  int32_t pv_fp8;
 } sagesla_options;
+
+/* Fills *opt with the defaults: every pointer NULL, test hooks 0, quant = pv_fp8 = 1. */
+void sagesla_options_init(sagesla_options* opt);
 
 #define SAGESLA_N_STAGES 7
 
@@ -113,6 +130,9 @@ typedef struct {
   size_t amask;       /* bf16 [B*H][nb_m_pad][nb_k_pad] complement mask (1 = not kept) */
   size_t hflat;       /* bf16 [B*H][nb_k_pad][129*128] key-block states H_j as [n][c] */
   size_t gsum;        /* bf16 [B*H][nb_m_pad][129*128] complement sums G_i as [n][c] */
+  size_t qb, kb;      /* bf16 [B*H][n_pad][128] copies of Q and K (K rows key-interleaved
+                       * within each 64-key block) for quant = 0; 0 when absent */
+  size_t vb;          /* bf16 [B*H][n_pad][128] copy of V for pv_fp8 = 0; 0 when absent */
 } sagesla_workspace_layout;
 
 /* Human-readable name of a status code (static string). */
@@ -132,6 +152,16 @@ sagesla_status sagesla_get_workspace_layout(int64_t B, int64_t H, int64_t N, int
                                             double topk_ratio, int block,
                                             sagesla_workspace_layout* layout);
 
+/* As sagesla_workspace_size / sagesla_get_workspace_layout for the operand mode of *opt
+ * (quant, pv_fp8; opt NULL = the defaults): the 16-bit modes add bf16 copies of their
+ * operands. Errors as sagesla_forward_ex's mode checks; 0 bytes for invalid arguments. */
+size_t sagesla_workspace_size_ex(int64_t B, int64_t H, int64_t N, int64_t D, double topk_ratio,
+                                 int block, const sagesla_options* opt);
+sagesla_status sagesla_get_workspace_layout_ex(int64_t B, int64_t H, int64_t N, int64_t D,
+                                               double topk_ratio, int block,
+                                               const sagesla_options* opt,
+                                               sagesla_workspace_layout* layout);
+
 /* The SageSLA forward: out = sparse(Q,K,V) + linear(Q,K,V) as defined above.
  *   q, k, v   : bf16 [B,H,N,128] device tensors (read only)
  *   topk_ratio: r in (0, 1]
@@ -146,7 +176,9 @@ sagesla_status sagesla_forward(const sagesla_tensor* q, const sagesla_tensor* k,
                                sagesla_tensor* out, void* workspace, size_t workspace_bytes,
                                void* stream);
 
-/* As sagesla_forward, plus the optional outputs of *opt (opt may be NULL). */
+/* As sagesla_forward, plus the optional outputs and the operand mode of *opt (opt may be
+ * NULL: no extra outputs, quant = pv_fp8 = 1). The workspace must hold
+ * sagesla_workspace_size_ex(..., opt) bytes. */
 sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor* k,
                                   const sagesla_tensor* v, double topk_ratio, int block,
                                   sagesla_tensor* out, void* workspace, size_t workspace_bytes,

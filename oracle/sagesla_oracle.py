@@ -289,6 +289,35 @@ def online_softmax_p8(blocks, exp_rel_err: float = EXP2_REL_ERR):
     return o, l, amb, lw
 
 
+def online_softmax_real(blocks):
+    """The online loop with real P and V (SPEC sections 9 and 9.1): for each kept block in
+    ascending order, with logits s [nq, nk] and value rows v [nk, D]: m' = max(m, rowmax s),
+    alpha = e^{m - m'}, p = e^{s - m'}, l <- alpha l + sum p, o <- alpha o + p . v. Returns
+    (o, l, mag) with mag the same recurrence over p . |v| (so that mag / l is the output of
+    the same weights applied to |v|, the size of the terms each output element sums)."""
+    nq = blocks[0][0].shape[0]
+    d = blocks[0][1].shape[1]
+    m = np.full(nq, -np.inf)
+    l = np.zeros(nq)
+    o = np.zeros((nq, d))
+    mag = np.zeros((nq, d))
+    for s, v in blocks:
+        m_new = np.maximum(m, s.max(axis=1))
+        alpha = np.where(np.isneginf(m), 0.0, np.exp(m - m_new))
+        p = np.exp(s - m_new[:, None])
+        l = alpha * l + p.sum(axis=1)
+        o = alpha[:, None] * o + p @ v
+        mag = alpha[:, None] * mag + p @ np.abs(v)
+        m = m_new
+    return o, l, mag
+
+
+# Tolerance of the sparse branch when P (and V) enter the P.V product in bf16 (SPEC section
+# 10): P rounded to bf16 (relative 2^-9 per term), fp32 accumulation; twice the unit
+# roundoff times the size of the terms.
+BF16_PV_REL = 2.0 ** -8
+
+
 def sparse_output(o: np.ndarray, l: np.ndarray, s_v: np.ndarray) -> np.ndarray:
     """O_s = o s_v / (448 l): the P codes carry the scale 1/448, the V codes s_v per channel."""
     return o * (np.asarray(s_v, dtype=np.float64)[None, :] / (E4M3_MAX * l[:, None]))
@@ -369,48 +398,41 @@ def key_block_states(k: np.ndarray, v: np.ndarray) -> np.ndarray:
 
 
 def sparse_block_row(prep: HeadPrep, i: int, q, k, v, quant: bool = True,
-                     smooth_in_quant_off: bool = False, return_ambiguity: bool = False):
+                     smooth_in_quant_off: bool = False, return_ambiguity: bool = False,
+                     pv_fp8: bool = True):
     """Sparse branch for the real query tokens of block i: online softmax over kept(i) in
     ascending order, running max updated per key block (no lazy rescale).
 
-    With ``return_ambiguity`` also returns, per output element, the bound on what a kernel
-    may differ by through ambiguous P codes and the window of the row sum (zero with
-    quantization off)."""
+    ``quant``: logits from the INT8 codes (SPEC 4, 6) or from the real Q, K (SPEC 9).
+    ``pv_fp8`` (with ``quant``): P and V in e4m3 (SPEC 6), or real P and V (SPEC 9.1).
+    With ``return_ambiguity`` also returns, per output element, the allowance a kernel needs:
+    ambiguous P codes and the window of the row sum (e4m3 P.V), or the bf16 rounding of P
+    (real P.V: BF16_PV_REL times the output of the same weights applied to |v|)."""
     n = prep.n
     qrows = block_rows(i, n)
     inv_sqrt_d = 1.0 / math.sqrt(q.shape[1])
     if quant:
-        blocks = []
+        logits = []
         for j in prep.kept[i]:
             krows = block_rows(int(j), n)
             s_int = prep.q8[qrows].astype(np.float64) @ prep.k8[krows].astype(np.float64).T
-            blocks.append((s_int * (float(prep.sq[i]) * float(prep.sk[j])) * inv_sqrt_d,
-                           prep.v8[krows]))
-        o, l, amb, lw = online_softmax_p8(blocks)
-        o_s = sparse_output(o, l, prep.s_v)
-        if return_ambiguity:
-            return o_s, sparse_output(amb, l, prep.s_v) + np.abs(o_s) * (lw / l)[:, None]
-        return o_s
-    nq = qrows.stop - qrows.start
-    d = q.shape[1]
-    m = np.full(nq, -np.inf)
-    l = np.zeros(nq)
-    o = np.zeros((nq, d))
-    if smooth_in_quant_off:
-        k_used = k - smoothing_mean(k)[None, :]
+            logits.append((s_int * (float(prep.sq[i]) * float(prep.sk[j])) * inv_sqrt_d, krows))
+        if pv_fp8:
+            o, l, amb, lw = online_softmax_p8([(s_, prep.v8[kr]) for s_, kr in logits])
+            o_s = sparse_output(o, l, prep.s_v)
+            if return_ambiguity:
+                return o_s, sparse_output(amb, l, prep.s_v) + np.abs(o_s) * (lw / l)[:, None]
+            return o_s
+        o, l, mag = online_softmax_real([(s_, v[kr]) for s_, kr in logits])
     else:
-        k_used = k
-    for j in prep.kept[i]:
-        krows = block_rows(int(j), n)
-        s = (q[qrows] @ k_used[krows].T) * inv_sqrt_d
-        m_new = np.maximum(m, s.max(axis=1))
-        alpha = np.where(np.isneginf(m), 0.0, np.exp(m - m_new))
-        p = np.exp(s - m_new[:, None])
-        l = alpha * l + p.sum(axis=1)
-        o = alpha[:, None] * o + p @ v[krows]
-        m = m_new
+        k_used = k - smoothing_mean(k)[None, :] if smooth_in_quant_off else k
+        blocks = []
+        for j in prep.kept[i]:
+            krows = block_rows(int(j), n)
+            blocks.append(((q[qrows] @ k_used[krows].T) * inv_sqrt_d, v[krows]))
+        o, l, mag = online_softmax_real(blocks)
     if return_ambiguity:
-        return o / l[:, None], np.zeros_like(o)
+        return o / l[:, None], BF16_PV_REL * mag / l[:, None]
     return o / l[:, None]
 
 
@@ -456,7 +478,7 @@ def linear_block_row_bruteforce(prep: HeadPrep, i: int, q, k, v) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 
 def forward_head(q, k, v, topk_ratio: float, quant: bool = True, rows=None,
-                 kept_override=None, smooth_in_quant_off: bool = False):
+                 kept_override=None, smooth_in_quant_off: bool = False, pv_fp8: bool = True):
     """SageSLA forward for one (b,h). q, k, v: float64 [N, D] holding bf16 values.
 
     ``rows``: query blocks to evaluate (default all). Returns (prep, out) where out maps a
@@ -473,7 +495,7 @@ def forward_head(q, k, v, topk_ratio: float, quant: bool = True, rows=None,
     for i in rows:
         o_s, amb = sparse_block_row(prep, i, q, k, v, quant=quant,
                                     smooth_in_quant_off=smooth_in_quant_off,
-                                    return_ambiguity=True)
+                                    return_ambiguity=True, pv_fp8=pv_fp8)
         o_l = linear_block_row(prep, i, q, h_blocks)
         out[i] = {"o_s": o_s, "o_l": o_l, "o": o_s + o_l, "o_s_ambig": amb}
     return prep, out

@@ -48,18 +48,31 @@ class SageslaOptions(ctypes.Structure):
     _fields_ = [("kept_idx_out", ctypes.c_void_p), ("mask_out", ctypes.c_void_p),
                 ("scores_out", ctypes.c_void_p), ("sparse_out", ctypes.c_void_p),
                 ("stage_events", ctypes.POINTER(ctypes.c_void_p)),
-                ("debug_spin_limit_us", ctypes.c_uint32), ("debug_skip_tile", ctypes.c_int32)]
+                ("debug_spin_limit_us", ctypes.c_uint32), ("debug_skip_tile", ctypes.c_int32),
+                ("quant", ctypes.c_int32), ("pv_fp8", ctypes.c_int32)]
+
+
+def _options(quant: bool = True, pv_fp8: bool = True) -> SageslaOptions:
+    opt = SageslaOptions()
+    load_library().sagesla_options_init(ctypes.byref(opt))
+    opt.quant = 1 if quant else 0
+    opt.pv_fp8 = 1 if pv_fp8 else 0
+    return opt
 
 
 _LAYOUT_FIELDS = ["status", "q8", "k8", "v8", "sq", "sk", "s_v", "inv_v", "mu", "qbar", "kbar",
                   "ksum_part", "vmax_part", "scores", "kept", "mask", "amask", "hflat", "gsum"]
 
 
+# bf16 operand copies of the 16-bit modes (offset 0 when absent)
+_MODE_LAYOUT_FIELDS = ["qb", "kb", "vb"]
+
+
 class SageslaWorkspaceLayout(ctypes.Structure):
     _fields_ = ([("total_bytes", ctypes.c_size_t)] +
                 [(n, ctypes.c_int64) for n in
                  ("nb", "k", "n_pad", "mask_words", "nb_k_pad", "nb_m_pad")] +
-                [(n, ctypes.c_size_t) for n in _LAYOUT_FIELDS])
+                [(n, ctypes.c_size_t) for n in _LAYOUT_FIELDS + _MODE_LAYOUT_FIELDS])
 
 
 SAGESLA_LAYER_NORM = 0
@@ -84,6 +97,11 @@ _SIGNATURES = {
     "sagesla_workspace_size": (ctypes.c_size_t, [ctypes.c_int64] * 4 + [ctypes.c_double, ctypes.c_int]),
     "sagesla_get_workspace_layout": (ctypes.c_int, [ctypes.c_int64] * 4 + [
         ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaWorkspaceLayout)]),
+    "sagesla_options_init": (None, [ctypes.c_void_p]),
+    "sagesla_workspace_size_ex": (ctypes.c_size_t, [ctypes.c_int64] * 4 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p]),
+    "sagesla_get_workspace_layout_ex": (ctypes.c_int, [ctypes.c_int64] * 4 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.POINTER(SageslaWorkspaceLayout)]),
     "sagesla_forward": (ctypes.c_int, [ctypes.POINTER(SageslaTensor)] * 3 + [
         ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaTensor), ctypes.c_void_p,
         ctypes.c_size_t, ctypes.c_void_p]),
@@ -172,16 +190,22 @@ def sagesla_topk_count(N: int, topk_ratio: float, block: int = BLOCK) -> int:
 
 
 def sagesla_workspace_size(B: int, H: int, N: int, D: int = HEAD_DIM, topk_ratio: float = 0.1,
-                           block: int = BLOCK) -> int:
-    return int(load_library().sagesla_workspace_size(B, H, N, D, float(topk_ratio), block))
+                           block: int = BLOCK, quant: bool = True, pv_fp8: bool = True) -> int:
+    if quant and pv_fp8:
+        return int(load_library().sagesla_workspace_size(B, H, N, D, float(topk_ratio), block))
+    opt = _options(quant, pv_fp8)
+    return int(load_library().sagesla_workspace_size_ex(B, H, N, D, float(topk_ratio), block,
+                                                        ctypes.byref(opt)))
 
 
 def sagesla_get_workspace_layout(B: int, H: int, N: int, D: int = HEAD_DIM,
-                                 topk_ratio: float = 0.1, block: int = BLOCK) -> dict:
+                                 topk_ratio: float = 0.1, block: int = BLOCK,
+                                 quant: bool = True, pv_fp8: bool = True) -> dict:
     lay = SageslaWorkspaceLayout()
-    _check(load_library().sagesla_get_workspace_layout(B, H, N, D, float(topk_ratio), block,
-                                                       ctypes.byref(lay)),
-           "sagesla_get_workspace_layout")
+    opt = _options(quant, pv_fp8)
+    _check(load_library().sagesla_get_workspace_layout_ex(B, H, N, D, float(topk_ratio), block,
+                                                          ctypes.byref(opt), ctypes.byref(lay)),
+           "sagesla_get_workspace_layout_ex")
     return {name: getattr(lay, name) for name, _ in SageslaWorkspaceLayout._fields_}
 
 
@@ -198,18 +222,20 @@ def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_rati
                     workspace: torch.Tensor | None = None, stream=None,
                     out_dtype: torch.dtype = torch.float32, kept_idx_out=None, mask_out=None,
                     scores_out=None, sparse_out=None, stage_events=None,
-                    debug_spin_limit_us: int = 0, debug_skip_tile: bool = False) -> torch.Tensor:
+                    debug_spin_limit_us: int = 0, debug_skip_tile: bool = False,
+                    quant: bool = True, pv_fp8: bool = True) -> torch.Tensor:
     """SageSLA forward on device tensors q, k, v (bf16 [B, H, N, 128]); returns ``out``.
 
     ``stage_events``: optional list of N_STAGES + 1 torch.cuda.Event(enable_timing=True)
     recorded around each kernel of the forward on the launching stream.
     ``debug_spin_limit_us`` / ``debug_skip_tile``: the failure-path test hooks of
-    sagesla_options (0 / False in normal use)."""
+    sagesla_options (0 / False in normal use). ``quant`` / ``pv_fp8``: the operand mode
+    (INT8 Q.K^T / e4m3 P.V by default; False selects bf16)."""
     lib = load_library()
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
     B, H, N, D = q.shape
-    need = sagesla_workspace_size(B, H, N, D, topk_ratio, block)
+    need = sagesla_workspace_size(B, H, N, D, topk_ratio, block, quant, pv_fp8)
     if workspace is None:
         workspace = alloc_workspace(need, q.device)
     vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
@@ -218,8 +244,11 @@ def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_rati
             ctypes.byref(vo), ctypes.c_void_p(workspace.data_ptr()),
             workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_ptr(stream)))
     if (any(x is not None for x in extra) or stage_events is not None or debug_spin_limit_us
-            or debug_skip_tile):
-        opt = SageslaOptions(*[None if x is None else x.data_ptr() for x in extra])
+            or debug_skip_tile or not quant or not pv_fp8):
+        opt = _options(quant, pv_fp8)
+        for name, x in zip(("kept_idx_out", "mask_out", "scores_out", "sparse_out"), extra):
+            if x is not None:
+                setattr(opt, name, x.data_ptr())
         opt.debug_spin_limit_us = int(debug_spin_limit_us)
         opt.debug_skip_tile = 1 if debug_skip_tile else 0
         if stage_events is not None:

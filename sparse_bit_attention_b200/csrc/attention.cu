@@ -52,27 +52,43 @@ constexpr int kThreads = 384;
 // setmaxnreg split: 256 x 88 + 128 x 56 = 29696 registers, within the 384 x 80 a CTA is
 // launched with (checked on the host before the launch).
 constexpr uint32_t kSoftmaxRegs = 88, kHelperRegs = 56;
-constexpr uint32_t kKVBytes = 64 * 128;      // one K8 or V8 tile
-// e4m3 P tile of one half (64 rows), K-major without swizzle: core matrices of 8 rows x 16
-// keys (128 B); K-chunks 160 B apart and 8-row groups 672 B apart. The padding makes the
-// 16-byte stores of the softmax threads (one store phase holds rows r, r+8, r+1, r+9 and key
-// halves 0, 1) fall on eight distinct bank groups.
-constexpr uint32_t kPChunk = 160, kPGroup = 672;
-constexpr uint32_t kPBytes = 8 * kPGroup;
-// Per-half private region.
-constexpr uint32_t kHQ = 0;                  // the half's 64 Q8 rows (SW128), 8 KB
-constexpr uint32_t kHK = 8192;               // K8 tiles of a pair of kept blocks, 16 KB
-constexpr uint32_t kHV = kHK + 2 * kKVBytes; // V8 ring, kNV x 8 KB
-constexpr uint32_t kHalfBytes = kHV + kNV * kKVBytes;
+constexpr uint32_t kChunk = 8192;            // 64 rows x 128 bytes: one SW128 tile chunk
 constexpr uint32_t kHLinA = 0;               // epilogue: phi(Q) bf16, 2 x [64][128 B]
 constexpr uint32_t kHLinG = 16384;           // epilogue: G_i bf16, 2 x [128][128 B]
-static_assert(kHLinG + 32768 <= kHalfBytes, "linear operands fit in the half region");
-static_assert(kHalfBytes % 1024 == 0, "half regions keep the 1024-byte swizzle atoms aligned");
-constexpr uint32_t kOffP = 2 * kHalfBytes;   // the two halves' P tiles
-constexpr uint32_t kOffCtl = kOffP + 2 * kPBytes;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemS = 128;              // first S buffer column
-constexpr uint32_t kIdescPV = make_idesc(kFmtF32, kFmtE4M3, kFmtE4M3, 0, 1, 64, 128);
+
+// Shared-memory layout of one operand mode. kQK8: Q.K^T on INT8 codes (else bf16 Q and K);
+// kPV8: P.V on e4m3 P and V codes (else bf16 P and raw bf16 V).
+//   per half: Q rows (64 x 128 channels), K tiles of a pair of kept blocks, a kNV-stage V ring;
+//   after both halves: one P tile per half; then the control block.
+// A 16-bit tile of 128 channels is two 64-channel chunks (each 64 rows x 128 B, SW128); the
+// K pair of bf16 keys is chunk 0 of both blocks (16 KB) then chunk 1 of both blocks, so that
+// each chunk holds the 128 key rows an N=128 MMA reads.
+template <bool kQK8, bool kPV8>
+struct Lay {
+  static constexpr uint32_t kQBytes = kQK8 ? kChunk : 2 * kChunk;
+  static constexpr uint32_t kKBlock = kQK8 ? kChunk : 2 * kChunk;   // K tile of one key block
+  static constexpr uint32_t kVBlock = kPV8 ? kChunk : 2 * kChunk;   // V tile of one key block
+  static constexpr uint32_t kHQ = 0;
+  static constexpr uint32_t kHK = kQBytes;
+  static constexpr uint32_t kHV = kHK + 2 * kKBlock;
+  static constexpr uint32_t kHalfBytes = kHV + kNV * kVBlock;
+  // e4m3 P tile (64 rows), K-major without swizzle: core matrices of 8 rows x 16 keys
+  // (128 B); K-chunks 160 B apart and 8-row groups 672 B apart. The padding makes the 16-byte
+  // stores of the softmax threads (one store phase holds rows r, r+8, r+1, r+9 and key halves
+  // 0, 1) fall on eight distinct bank groups. bf16 P tile: 64 rows x 128 B, SW128.
+  static constexpr uint32_t kPChunk = 160, kPGroup = 672;
+  static constexpr uint32_t kPBytes = kPV8 ? 8 * kPGroup : kChunk;
+  static constexpr uint32_t kOffP = 2 * kHalfBytes;
+  static constexpr uint32_t kOffCtl = kOffP + 2 * kPBytes;
+  static_assert(kHLinG + 32768 <= kHalfBytes, "linear operands fit in the half region");
+  static_assert(kHalfBytes % 1024 == 0 && kOffP % 1024 == 0 && kPBytes % 32 == 0,
+                "swizzle atoms stay 1024-byte aligned");
+  static_assert(kPV8 || kPBytes % 1024 == 0, "bf16 P tiles are SW128 atoms");
+};
+constexpr uint32_t kIdescPV8 = make_idesc(kFmtF32, kFmtE4M3, kFmtE4M3, 0, 1, 64, 128);
+constexpr uint32_t kIdescPV16 = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 1, 64, 128);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kInvSqrtD = 0.08838834764831845f;
 constexpr float kLog2_448 = 8.807354922057604f;
@@ -99,9 +115,14 @@ struct Ctl {
   uint16_t klist[2][kListCap];
 };
 
-// Two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA, and 1 KB of
-// alignment slack in each CTA's request.
-static_assert(2 * (1024 + kOffCtl + sizeof(Ctl) + 1024) <= 228 * 1024, "two CTAs fit on an SM");
+// Dynamic shared memory of a mode: the layout, the control block and 1 KB of alignment slack.
+template <bool kQK8, bool kPV8>
+constexpr size_t attn_smem_bytes() { return 1024 + Lay<kQK8, kPV8>::kOffCtl + sizeof(Ctl); }
+// The 8-bit mode runs two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA.
+// The 16-bit modes run one (227 KB at most per CTA).
+static_assert(2 * (attn_smem_bytes<true, true>() + 1024) <= 228 * 1024, "two CTAs fit on an SM");
+static_assert(attn_smem_bytes<true, false>() <= 227 * 1024, "fits one CTA");
+static_assert(attn_smem_bytes<false, false>() <= 227 * 1024, "fits one CTA");
 
 // n-th kept key block of half h's query block: its kept list (shared-memory copy first), or
 // block n itself when every block is kept (no list).
@@ -184,12 +205,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// Converts the row's int32 scores to floats in place (exact: |S| < 2^21) and returns the
-// largest of the first `valid` of them, by three-input maxima in four chains.
-template <bool kFull>
+// With kInt, converts the row's int32 scores to floats in place (exact: |S| < 2^21); returns
+// the largest of the first `valid` scores, by three-input maxima in four chains.
+template <bool kFull, bool kInt>
 __device__ __forceinline__ float row_block_fmax(uint32_t (&a)[32], int valid) {
+  if (kInt) {
 #pragma unroll
-  for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__int2float_rn(static_cast<int>(a[q])));
+    for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__int2float_rn(static_cast<int>(a[q])));
+  }
   float m[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -203,9 +226,11 @@ __device__ __forceinline__ float row_block_fmax(uint32_t (&a)[32], int valid) {
   }
   return fmaxf(fmax3(m[0], m[1], m[2]), m[3]);
 }
-template <bool kFull>
+// 448 p = 2^(S c + neg) for the thread's 32 scores: returns their sum and packs them into
+// the P operand, as e4m3 codes (kP8: pk[0..7]) or as bf16 values (pk[0..15]).
+template <bool kFull, bool kP8>
 __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int valid, float c,
-                                              float neg, uint32_t (&pk)[8]) {
+                                              float neg, uint32_t (&pk)[16]) {
   const unsigned long long c2 = pk2(c, c), neg2 = pk2(neg, neg);
   unsigned long long acc0 = pk2(0.f, 0.f), acc1 = pk2(0.f, 0.f);
 #pragma unroll
@@ -225,22 +250,34 @@ __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int vali
     }
     acc0 = add2(acc0, pk2(y[0], y[1]));
     acc1 = add2(acc1, pk2(y[2], y[3]));
-    pk[q >> 2] = static_cast<uint32_t>(f32x2_to_e4m3x2(y[0], y[1])) |
-                 (static_cast<uint32_t>(f32x2_to_e4m3x2(y[2], y[3])) << 16);
+    if (kP8) {
+      pk[q >> 2] = static_cast<uint32_t>(f32x2_to_e4m3x2(y[0], y[1])) |
+                   (static_cast<uint32_t>(f32x2_to_e4m3x2(y[2], y[3])) << 16);
+    } else {
+      __nv_bfloat162 b0 = __floats2bfloat162_rn(y[0], y[1]);
+      __nv_bfloat162 b1 = __floats2bfloat162_rn(y[2], y[3]);
+      pk[q >> 1] = *reinterpret_cast<uint32_t*>(&b0);
+      pk[(q >> 1) + 1] = *reinterpret_cast<uint32_t*>(&b1);
+    }
   }
   float a, b;
   up2(add2(acc0, acc1), a, b);
   return a + b;
 }
 
+template <bool kQK8, bool kPV8>
 __global__ void __launch_bounds__(kThreads, 2)
 k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
             AttnParams prm) {
+  using L = Lay<kQK8, kPV8>;
+  constexpr uint32_t kHalfBytes = L::kHalfBytes, kHQ = L::kHQ, kHK = L::kHK, kHV = L::kHV;
+  constexpr uint32_t kOffP = L::kOffP, kPBytes = L::kPBytes;
+  constexpr uint32_t kPChunk = L::kPChunk, kPGroup = L::kPGroup;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + kOffCtl);
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + L::kOffCtl);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x;
@@ -297,11 +334,13 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int row_base = static_cast<int>(bh * prm.n_pad);
+      // A 16-bit tile of 128 channels arrives as two boxes of 64 channels (x = 0, 64).
       for (int h = 0; h < 2; ++h) {
         if (U[h] == 0) continue;
-        mbar_arrive_expect_tx(&ctl->hc[h].q_full, 8192u);
-        tma_load_2d(smem + h * kHalfBytes + kHQ, &tm_q, &ctl->hc[h].q_full, 0,
-                    row_base + 128 * pair + 64 * h);
+        mbar_arrive_expect_tx(&ctl->hc[h].q_full, L::kQBytes);
+        uint8_t* qst = smem + h * kHalfBytes + kHQ;
+        tma_load_2d(qst, &tm_q, &ctl->hc[h].q_full, 0, row_base + 128 * pair + 64 * h);
+        if (!kQK8) tma_load_2d(qst + kChunk, &tm_q, &ctl->hc[h].q_full, 64, row_base + 128 * pair + 64 * h);
       }
       bool ok = true;
       const int Umax = max(U[0], U[1]);
@@ -316,10 +355,13 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           // Failure-path test: the first pair of CTA (0, 0) is never loaded, so the waits for
           // it run out (nothing is left in flight: neither its bytes nor its copies exist).
           if (prm.skip_tile && n0 == 0 && h == 0 && pair == 0 && bh == 0) continue;
-          mbar_arrive_expect_tx(&c.k_full, two * kKVBytes);
+          mbar_arrive_expect_tx(&c.k_full, two * L::kKBlock);
           uint8_t* kst = smem + h * kHalfBytes + kHK;
-          tma_load_2d(kst, &tm_k, &c.k_full, 0, row_base + 64 * kept_at(ctl, h, klist, n0));
-          if (two == 2) tma_load_2d(kst + kKVBytes, &tm_k, &c.k_full, 0, row_base + 64 * kept_at(ctl, h, klist, n0 + 1));
+          for (int b = 0; b < two; ++b) {
+            const int y = row_base + 64 * kept_at(ctl, h, klist, n0 + b);
+            tma_load_2d(kst + b * kChunk, &tm_k, &c.k_full, 0, y);
+            if (!kQK8) tma_load_2d(kst + 2 * kChunk + b * kChunk, &tm_k, &c.k_full, 64, y);
+          }
         }
         // V8 of blocks n0 and n0 + 1: stage n % kNV is free once P.V(n - kNV) is done
         for (int n = n0; n < n0 + 2 && ok; ++n)
@@ -329,9 +371,11 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int s = n % kNV;
             if (n >= kNV && !(ok = wait_or_abort(&c.v_empty[s], ((n / kNV) - 1) & 1, ctl, status, prm.spin_ns))) break;
             const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) : nullptr;
-            mbar_arrive_expect_tx(&c.v_full[s], kKVBytes);
-            tma_load_2d(smem + h * kHalfBytes + kHV + s * kKVBytes, &tm_v, &c.v_full[s], 0,
-                        row_base + 64 * kept_at(ctl, h, klist, n));
+            mbar_arrive_expect_tx(&c.v_full[s], L::kVBlock);
+            uint8_t* vst = smem + h * kHalfBytes + kHV + s * L::kVBlock;
+            const int y = row_base + 64 * kept_at(ctl, h, klist, n);
+            tma_load_2d(vst, &tm_v, &c.v_full[s], 0, y);
+            if (!kPV8) tma_load_2d(vst + kChunk, &tm_v, &c.v_full[s], 64, y);
           }
       }
       // G_i once the half's loop MMAs are done (its tile overlaps the K and V stages)
@@ -351,6 +395,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // halves, one M=64 N=128 group per pair of kept blocks) and the linear-branch MMA
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc(kFmtS32, kFmtS8, kFmtS8, 0, 0, 64, 128);
+      constexpr uint32_t idesc_s16 = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 64, 128);
       constexpr uint32_t idesc_l = make_idesc(kFmtF32, kFmtBF16, kFmtBF16, 0, 0, 64, 128);
       bool ok = true;
       for (int h = 0; h < 2 && ok; ++h)
@@ -373,10 +418,20 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           if (p > 0 && !(ok = wait_or_abort(&c.s_free, (p - 1) & 1, ctl, status, prm.spin_ns))) break;
           tc_fence_after();
           const uint32_t d = tmem + (static_cast<uint32_t>(16 * h) << 16) + kTmemS;
-          mma_i8(d, dq[h], dk[h], idesc_s, 0u);
-          mma_i8(d, dq[h] + 2, dk[h] + 2, idesc_s, 1u);
-          mma_i8(d, dq[h] + 4, dk[h] + 4, idesc_s, 1u);
-          mma_i8(d, dq[h] + 6, dk[h] + 6, idesc_s, 1u);
+          if (kQK8) {
+            mma_i8(d, dq[h], dk[h], idesc_s, 0u);
+            mma_i8(d, dq[h] + 2, dk[h] + 2, idesc_s, 1u);
+            mma_i8(d, dq[h] + 4, dk[h] + 4, idesc_s, 1u);
+            mma_i8(d, dq[h] + 6, dk[h] + 6, idesc_s, 1u);
+          } else {
+            // bf16: eight K-steps of 16 channels (32 bytes), four per 64-channel chunk; the
+            // address field counts 16-byte units.
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16(d, dq[h] + (kk >> 2) * (kChunk >> 4) + (kk & 3) * 2,
+                       dk[h] + (kk >> 2) * (2 * kChunk >> 4) + (kk & 3) * 2, idesc_s16,
+                       kk ? 1u : 0u);
+          }
           mma_commit(&c.s_full);
         }
       }
@@ -408,6 +463,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       const uint32_t p_addr = smem_u32(smem) + kOffP + h * kPBytes;
       const uint64_t dp0 = make_sdesc(p_addr, kPChunk, kPGroup, kLayoutNone);
       const uint64_t dp1 = make_sdesc(p_addr + 2 * kPChunk, kPChunk, kPGroup, kLayoutNone);
+      const uint64_t dp16 = make_sdesc(p_addr, 16, 1024, kLayoutSW128);   // bf16 P, SW128
       const uint32_t vb = smem_u32(smem + h * kHalfBytes) + kHV;
       const uint32_t d = tmem + (static_cast<uint32_t>(16 * h) << 16);
       for (int n = 0; n < U[h]; ++n) {
@@ -415,11 +471,19 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (!wait_or_abort(&c.p_full, n & 1, ctl, status, prm.spin_ns)) break;
         if (!wait_or_abort(&c.v_full[s], (n / kNV) & 1, ctl, status, prm.spin_ns)) break;
         tc_fence_after();
-        // P: K-major, no swizzle (layout above). V: MN-major (d contiguous), 128-byte
-        // swizzle, 8-key groups 1024 B apart.
-        const uint32_t v_addr = vb + s * kKVBytes;
-        mma_f8(d, dp0, make_sdesc(v_addr, 8192, 1024, kLayoutSW128), kIdescPV, n > 0 ? 1u : 0u);
-        mma_f8(d, dp1, make_sdesc(v_addr + 4096, 8192, 1024, kLayoutSW128), kIdescPV, 1u);
+        // P: K-major (e4m3: no swizzle, layout above; bf16: SW128). V: MN-major (d
+        // contiguous), 128-byte swizzle, 8-key groups 1024 B apart, bf16 channel chunks
+        // 8 KB apart.
+        const uint32_t v_addr = vb + s * L::kVBlock;
+        if (kPV8) {
+          mma_f8(d, dp0, make_sdesc(v_addr, 8192, 1024, kLayoutSW128), kIdescPV8, n > 0 ? 1u : 0u);
+          mma_f8(d, dp1, make_sdesc(v_addr + 4096, 8192, 1024, kLayoutSW128), kIdescPV8, 1u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // K-steps of 16 keys: 32 B of P, 2 KB of V
+            mma_bf16(d, dp16 + kk * 2, make_sdesc(v_addr + kk * 2048, 8192, 1024, kLayoutSW128),
+                     kIdescPV16, (n > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(&c.pv_done[n & 1]);
         mma_commit(&c.v_empty[s]);
         if (n == U[h] - 1) mma_commit(&c.mma_done);
@@ -446,20 +510,23 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     bool ok = Uh > 0;
     float m_run = -INFINITY, l_part = 0.f;
     if (ok) {
-      const float cs = prm.sq[bh * prm.nbq + qblock] * (kLog2e * kInvSqrtD);
+      // base-2 exponent per unit of S: sq sk log2(e) / sqrt(128) for INT8 scores, log2(e) /
+      // sqrt(128) for bf16 scores
+      const float cs = kQK8 ? prm.sq[bh * prm.nbq + qblock] * (kLog2e * kInvSqrtD)
+                            : kLog2e * kInvSqrtD;
       const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + qblock) * static_cast<int64_t>(prm.k) : nullptr;
       const float* skh = prm.sk + bh * prm.nbq;
       // kept indices are read two blocks ahead and scales one block ahead, so that no load
       // of the loop waits for another one
       int j_cur = kept_block(klist, 0);
       int j_ahead = Uh > 1 ? kept_block(klist, 1) : 0;
-      float sk_next = __ldg(skh + j_cur);
+      float sk_next = kQK8 ? __ldg(skh + j_cur) : 1.f;
       for (int n = 0; n < Uh; ++n) {
         const int b = n & 1;
         const int j = j_cur;
         const float skj = sk_next;
         if (n + 1 < Uh) {
-          sk_next = __ldg(skh + j_ahead);
+          if (kQK8) sk_next = __ldg(skh + j_ahead);
           j_cur = j_ahead;
           if (n + 2 < Uh) j_ahead = kept_block(klist, n + 2);
         }
@@ -474,24 +541,33 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           if (lane == 0) mbar_arrive(&c.s_free);
         }
         const bool full = j != prm.nb - 1 || prm.n_last == 64;   // no padded keys
-        float mx = full ? row_block_fmax<true>(sr, 32) : row_block_fmax<false>(sr, valid);
+        float mx = full ? row_block_fmax<true, kQK8>(sr, 32) : row_block_fmax<false, kQK8>(sr, valid);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float cst = cs * skj;
+        const float cst = kQK8 ? cs * skj : cs;
         const float m_new = fmaxf(m_run, mx * cst);
         const float alpha = ex2_mufu(m_run - m_new);
         const float neg = kLog2_448 - m_new;    // 2^(S c + neg) = 448 p
-        uint32_t pk[8];
-        const float rs = full ? row_exp_pack<true>(sr, 32, cst, neg, pk)
-                              : row_exp_pack<false>(sr, valid, cst, neg, pk);
+        uint32_t pk[16];
+        const float rs = full ? row_exp_pack<true, kPV8>(sr, 32, cst, neg, pk)
+                              : row_exp_pack<false, kPV8>(sr, valid, cst, neg, pk);
         l_part = alpha * l_part + rs;
         m_run = m_new;
         // P.V(n-1) must be done: it frees P buffer b (read by P.V(n-2) before it), makes O
         // stable for the rescale, and orders the P.V MMAs issued from different warps.
         if (n >= 1 && !wait_or_abort(&c.pv_done[b ^ 1], ((n - 1) >> 1) & 1, ctl, status, prm.spin_ns)) { ok = false; break; }
         tc_fence_after();
-        uint8_t* pb = smem + kOffP + h * kPBytes + (r >> 3) * kPGroup + (r & 7) * 16 + 2 * kh * kPChunk;
-        *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(pb + kPChunk) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        if (kPV8) {
+          uint8_t* pb = smem + kOffP + h * kPBytes + (r >> 3) * kPGroup + (r & 7) * 16 + 2 * kh * kPChunk;
+          *reinterpret_cast<uint4*>(pb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(pb + kPChunk) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+          // bf16 P row r: this thread's 32 keys are the 16-byte chunks 4kh .. 4kh+3 (SW128)
+          uint8_t* pt = smem + kOffP + h * kPBytes;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            *reinterpret_cast<uint4*>(pt + sw128_offset(r, 4 * kh + e)) =
+                make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
         fence_proxy_async_smem();
         // rescale this row's O (skipped when no row of the warp moved its max); the two
         // threads of a row each take 64 of the 128 columns
@@ -604,7 +680,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float os = __uint_as_float(o[e]) * ctl->s_v[64 * cb + 2 * e + kh] * inv_l;
+          const float os = kPV8 ? __uint_as_float(o[e]) * ctl->s_v[64 * cb + 2 * e + kh] * inv_l
+                                : __uint_as_float(o[e]) * inv_l;
           o[e] = __float_as_uint(os);
           lin[e] = __float_as_uint(prm.linear ? os + __uint_as_float(lin[e]) * inv_den : os);
         }
@@ -647,22 +724,54 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
 }  // namespace
 
-cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32_t out_dtype,
-                             int64_t out_sb, int64_t out_sh, int64_t out_sn, float* sparse_out,
-                             char* ws, const AttnTestHooks& hooks, cudaStream_t stream) {
+namespace {
+
+// Tensor map of a per-head operand buffer [BH * n_pad rows][128 channels]: 8-bit codes in one
+// 128-byte box per row, or bf16 values in boxes of 64 channels (128 B), 64 rows, SW128.
+bool operand_map(CUtensorMap* m, bool eight_bit, const void* base, uint64_t rows) {
+  return eight_bit ? encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, base, 128,
+                                    64, CU_TENSOR_MAP_SWIZZLE_128B)
+                   : encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128, rows, 256, base, 64,
+                                    64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <bool kQK8, bool kPV8>
+cudaError_t launch_mode(const ForwardPlan& p, const AttnParams& prm, const char* ws,
+                        cudaStream_t stream) {
   const auto& L = p.lay;
   CUtensorMap tq, tk, tv, tg;
   const uint64_t rows = static_cast<uint64_t>(p.BH * p.n_pad);
-  if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, ws + L.q8, 128, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, ws + L.k8, 128, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, ws + L.v8, 128, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!operand_map(&tq, kQK8, ws + (kQK8 ? L.q8 : L.qb), rows) ||
+      !operand_map(&tk, kQK8, ws + (kQK8 ? L.k8 : L.kb), rows) ||
+      !operand_map(&tv, kPV8, ws + (kPV8 ? L.v8 : L.vb), rows) ||
       !encode_tmap_2d(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128,
                       static_cast<uint64_t>(p.BH * p.nb_m_pad * 129), 256, ws + L.gsum, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  // The register split (setmaxnreg) must fit the registers the CTA is launched with, or the
+  // softmax warps would wait for registers forever. The count is a property of the loaded
+  // module; it is queried per call (cheap, and right for every device and thread).
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, k_attention<kQK8, kPV8>) != cudaSuccess)
+    return cudaErrorInvalidDeviceFunction;
+  if (static_cast<uint32_t>(fa.numRegs) * kThreads < 256 * kSoftmaxRegs + 128 * kHelperRegs)
+    return cudaErrorInvalidConfiguration;
+  const size_t smem = attn_smem_bytes<kQK8, kPV8>();
+  cudaError_t e = cudaFuncSetAttribute(k_attention<kQK8, kPV8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(static_cast<unsigned>(p.n_pairs), static_cast<unsigned>(p.BH));
+  k_attention<kQK8, kPV8><<<grid, kThreads, smem, stream>>>(tq, tk, tv, tg, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32_t out_dtype,
+                             int64_t out_sb, int64_t out_sh, int64_t out_sn, float* sparse_out,
+                             char* ws, const AttnTestHooks& hooks, cudaStream_t stream) {
+  const auto& L = p.lay;
   AttnParams prm;
   prm.sq = reinterpret_cast<const float*>(ws + L.sq);
   prm.sk = reinterpret_cast<const float*>(ws + L.sk);
@@ -687,20 +796,10 @@ cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32
   prm.linear = p.linear_empty ? 0 : 1;
   prm.spin_ns = hooks.spin_limit_us ? 1000ull * hooks.spin_limit_us : kSpinLimitNs;
   prm.skip_tile = hooks.skip_tile;
-  // The register split (setmaxnreg) must fit the registers the CTA is launched with, or the
-  // softmax warps would wait for registers forever. The count is a property of the loaded
-  // module; it is queried per call (cheap, and right for every device and thread).
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, k_attention) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
-  if (static_cast<uint32_t>(fa.numRegs) * kThreads < 256 * kSoftmaxRegs + 128 * kHelperRegs)
-    return cudaErrorInvalidConfiguration;
-  const size_t smem = 1024 + kOffCtl + sizeof(Ctl);
-  cudaError_t e = cudaFuncSetAttribute(k_attention, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(p.n_pairs), static_cast<unsigned>(p.BH));
-  k_attention<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tg, prm);
-  return cudaGetLastError();
+  if (p.quant && p.pv_fp8) return launch_mode<true, true>(p, prm, ws, stream);
+  if (p.quant) return launch_mode<true, false>(p, prm, ws, stream);
+  if (!p.pv_fp8) return launch_mode<false, false>(p, prm, ws, stream);
+  return cudaErrorInvalidValue;     // bf16 Q.K^T with e4m3 P.V is not a mode
 }
 
 }  // namespace sagesla

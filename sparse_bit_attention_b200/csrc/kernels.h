@@ -29,11 +29,14 @@ struct ForwardPlan {
   int64_t nb_m_pad;    // nb rounded up to 128 (M extent of the complement-sum GEMM)
   int32_t n_last;      // tokens in the last block
   bool linear_empty;   // k == nb: every block kept, the linear branch is zero
+  bool quant;          // INT8 Q.K^T (else bf16 Q.K^T from packed bf16 copies)
+  bool pv_fp8;         // e4m3 P.V (else bf16 P and raw bf16 V)
   sagesla_workspace_layout lay;
 };
 
-// Fills plan from the problem size; returns false for invalid arguments.
-bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* plan);
+// Fills plan from the problem size and operand mode; returns false for invalid arguments.
+bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* plan,
+               bool quant = true, bool pv_fp8 = true);
 
 // Resolves cuTensorMapEncodeTiled through the runtime (no link-time libcuda dependency).
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint64_t inner, uint64_t outer,
@@ -77,6 +80,9 @@ cudaError_t launch_stats(const ForwardPlan& p, TensorArg k, TensorArg v, char* w
 cudaError_t launch_finalize(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_quant(const ForwardPlan& p, TensorArg q, TensorArg k, TensorArg v, char* ws,
                          cudaStream_t stream);
+// bf16 copies of Q and K (quant off) and V (pv_fp8 off) into the workspace.
+cudaError_t launch_pack_bf16(const ForwardPlan& p, TensorArg q, TensorArg k, TensorArg v,
+                             char* ws, cudaStream_t stream);
 cudaError_t launch_scores(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_topk(const ForwardPlan& p, char* ws, cudaStream_t stream);
 // SAGESLA_OK when the current device is a compute-capability-10.0 part (B200), else

@@ -434,6 +434,46 @@ cudaError_t launch_finalize(const ForwardPlan& p, char* ws, cudaStream_t stream)
   return cudaGetLastError();
 }
 
+// bf16 operand copies for the 16-bit modes of the attention: rows [head][n_pad][128] with
+// zero rows past N, 16 bytes per thread. Q and V keep the token order; K rows are stored
+// key-interleaved inside each 64-key block like the INT8 codes (row 2(r mod 32) + r div 32
+// holds key r), so that every softmax thread's TMEM fragment holds 32 consecutive keys.
+__global__ void k_pack_bf16(TensorArg src, int N, int n_pad, int64_t total, int interleave,
+                            uint4* __restrict__ dst) {
+  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (idx >= total) return;
+  const int chunk = static_cast<int>(idx & 15);
+  const int64_t row = idx >> 4;
+  const int64_t bh = row / n_pad;
+  const int pos = static_cast<int>(row - bh * n_pad);
+  // token held by stored row `pos`: the inverse of the interleaving within its block
+  const int in_block = pos & 63;
+  const int n = interleave ? (pos - in_block) + (in_block >> 1) + 32 * (in_block & 1) : pos;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (n < N) {
+    const int64_t b = bh / src.H, h = bh % src.H;
+    const uint16_t* base = static_cast<const uint16_t*>(src.data) + b * src.stride_b +
+                           h * src.stride_h + static_cast<int64_t>(n) * src.stride_n;
+    v = __ldg(reinterpret_cast<const uint4*>(base) + chunk);
+  }
+  dst[idx] = v;
+}
+
+cudaError_t launch_pack_bf16(const ForwardPlan& p, TensorArg q, TensorArg k, TensorArg v,
+                             char* ws, cudaStream_t stream) {
+  const auto& L = p.lay;
+  const int64_t total = p.BH * p.n_pad * 16;
+  const unsigned grid = static_cast<unsigned>((total + 255) / 256);
+  const int N = static_cast<int>(p.N), n_pad = static_cast<int>(p.n_pad);
+  if (!p.quant) {
+    k_pack_bf16<<<grid, 256, 0, stream>>>(q, N, n_pad, total, 0, reinterpret_cast<uint4*>(ws + L.qb));
+    k_pack_bf16<<<grid, 256, 0, stream>>>(k, N, n_pad, total, 1, reinterpret_cast<uint4*>(ws + L.kb));
+  }
+  if (!p.pv_fp8)
+    k_pack_bf16<<<grid, 256, 0, stream>>>(v, N, n_pad, total, 0, reinterpret_cast<uint4*>(ws + L.vb));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quant(const ForwardPlan& p, TensorArg q, TensorArg k, TensorArg v, char* ws,
                          cudaStream_t stream) {
   const auto& L = p.lay;

@@ -39,9 +39,13 @@ std::once_flag g_encode_once;
 
 }  // namespace
 
-bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* p) {
+bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* p, bool quant,
+               bool pv_fp8) {
   if (B < 1 || H < 1 || N < 1 || !valid_ratio(topk_ratio)) return false;
+  if (!quant && pv_fp8) return false;          // bf16 Q.K^T with e4m3 P.V is not a mode
   std::memset(p, 0, sizeof(*p));
+  p->quant = quant;
+  p->pv_fp8 = pv_fp8;
   p->B = B;
   p->H = H;
   p->N = N;
@@ -94,6 +98,12 @@ bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* 
   L.amask = take(static_cast<size_t>(BH * p->nb_m_pad * p->nb_k_pad) * 2);
   L.hflat = take(static_cast<size_t>(BH * p->nb_k_pad) * kHFlat * 2);
   L.gsum = take(static_cast<size_t>(BH * p->nb_m_pad) * kHFlat * 2);
+  // bf16 operand copies of the 16-bit modes (offset 0 = absent: the status word is there)
+  if (!quant) {
+    L.qb = take(static_cast<size_t>(BH * p->n_pad) * 256);
+    L.kb = take(static_cast<size_t>(BH * p->n_pad) * 256);
+  }
+  if (!pv_fp8) L.vb = take(static_cast<size_t>(BH * p->n_pad) * 256);
   L.total_bytes = off;
   return true;
 }
@@ -231,22 +241,64 @@ int64_t sagesla_topk_count(int64_t N, double topk_ratio, int block) {
   return topk_count(ceil_div(N, kBlock), topk_ratio);
 }
 
-sagesla_status sagesla_get_workspace_layout(int64_t B, int64_t H, int64_t N, int64_t D,
-                                            double topk_ratio, int block,
-                                            sagesla_workspace_layout* layout) {
+void sagesla_options_init(sagesla_options* opt) {
+  if (!opt) return;
+  std::memset(opt, 0, sizeof(*opt));
+  opt->quant = 1;
+  opt->pv_fp8 = 1;
+}
+
+}  // extern "C"
+
+namespace {
+// Operand mode of a call: the options' quant / pv_fp8 (defaults without options).
+sagesla_status read_mode(const sagesla_options* opt, bool* quant, bool* pv_fp8) {
+  *quant = true;
+  *pv_fp8 = true;
+  if (!opt) return SAGESLA_OK;
+  if ((opt->quant != 0 && opt->quant != 1) || (opt->pv_fp8 != 0 && opt->pv_fp8 != 1))
+    return SAGESLA_ERR_INVALID_ARG;
+  if (opt->quant == 0 && opt->pv_fp8 == 1) return SAGESLA_ERR_UNSUPPORTED;
+  *quant = opt->quant != 0;
+  *pv_fp8 = opt->pv_fp8 != 0;
+  return SAGESLA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+sagesla_status sagesla_get_workspace_layout_ex(int64_t B, int64_t H, int64_t N, int64_t D,
+                                               double topk_ratio, int block,
+                                               const sagesla_options* opt,
+                                               sagesla_workspace_layout* layout) {
   if (!layout) return SAGESLA_ERR_INVALID_ARG;
   if (D != kHeadDim || block != kBlock) return SAGESLA_ERR_UNSUPPORTED;
+  bool quant, pv_fp8;
+  const sagesla_status st = read_mode(opt, &quant, &pv_fp8);
+  if (st != SAGESLA_OK) return st;
   ForwardPlan p;
-  if (!make_plan(B, H, N, topk_ratio, &p)) return SAGESLA_ERR_INVALID_ARG;
+  if (!make_plan(B, H, N, topk_ratio, &p, quant, pv_fp8)) return SAGESLA_ERR_INVALID_ARG;
   *layout = p.lay;
   return SAGESLA_OK;
 }
 
+sagesla_status sagesla_get_workspace_layout(int64_t B, int64_t H, int64_t N, int64_t D,
+                                            double topk_ratio, int block,
+                                            sagesla_workspace_layout* layout) {
+  return sagesla_get_workspace_layout_ex(B, H, N, D, topk_ratio, block, nullptr, layout);
+}
+
+size_t sagesla_workspace_size_ex(int64_t B, int64_t H, int64_t N, int64_t D, double topk_ratio,
+                                 int block, const sagesla_options* opt) {
+  sagesla_workspace_layout L;
+  if (sagesla_get_workspace_layout_ex(B, H, N, D, topk_ratio, block, opt, &L) != SAGESLA_OK)
+    return 0;
+  return L.total_bytes;
+}
+
 size_t sagesla_workspace_size(int64_t B, int64_t H, int64_t N, int64_t D, double topk_ratio,
                               int block) {
-  sagesla_workspace_layout L;
-  if (sagesla_get_workspace_layout(B, H, N, D, topk_ratio, block, &L) != SAGESLA_OK) return 0;
-  return L.total_bytes;
+  return sagesla_workspace_size_ex(B, H, N, D, topk_ratio, block, nullptr);
 }
 
 sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor* k,
@@ -260,8 +312,10 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
   if ((st = check_view(out, q, true)) != SAGESLA_OK) return st;
   if (block != kBlock) return SAGESLA_ERR_UNSUPPORTED;
   if (!valid_ratio(topk_ratio)) return SAGESLA_ERR_INVALID_ARG;
+  bool quant, pv_fp8;
+  if ((st = read_mode(opt, &quant, &pv_fp8)) != SAGESLA_OK) return st;
   ForwardPlan p;
-  if (!make_plan(q->B, q->H, q->N, topk_ratio, &p)) return SAGESLA_ERR_INVALID_ARG;
+  if (!make_plan(q->B, q->H, q->N, topk_ratio, &p, quant, pv_fp8)) return SAGESLA_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
       workspace_bytes < p.lay.total_bytes)
     return SAGESLA_ERR_WORKSPACE;
@@ -289,6 +343,7 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
   SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
   SAGESLA_LAUNCH(mark(2));
   SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
+  if (!p.quant || !p.pv_fp8) SAGESLA_LAUNCH(launch_pack_bf16(p, qa, ka, va, ws, stream));
   SAGESLA_LAUNCH(mark(3));
   // With every key block kept (k == nb) the selection is the identity: the scores are only
   // computed when asked for, and the kept lists and masks only written when asked for.
@@ -388,6 +443,7 @@ sagesla_status sagesla_sla_backward(const sagesla_tensor* q, const sagesla_tenso
   SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
   SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
   SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
+  if (!p.quant || !p.pv_fp8) SAGESLA_LAUNCH(launch_pack_bf16(p, qa, ka, va, ws, stream));
   if (!p.linear_empty) {
     SAGESLA_LAUNCH(launch_scores(p, ws, stream));
     SAGESLA_LAUNCH(launch_topk(p, ws, stream));

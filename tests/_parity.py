@@ -33,13 +33,14 @@ def _ws_slice(ws: torch.Tensor, off: int, count: int, dtype: torch.dtype) -> tor
     return ws[off: off + nbytes].view(dtype)
 
 
-def gpu_run(q, k, v, ratio, out_dtype=torch.float32, extras=True, device="cuda:0"):
+def gpu_run(q, k, v, ratio, out_dtype=torch.float32, extras=True, device="cuda:0",
+            quant=True, pv_fp8=True):
     """Forward on the GPU. Returns a dict of CPU tensors: out, kept [BH,nb,k], mask words,
     scores, sparse (sparse-branch output) and the raw workspace tensor (on the device)."""
     dev = torch.device(device)
     qd, kd, vd = (x.to(dev) for x in (q, k, v))
     B, H, N, D = q.shape
-    lay = sba.sagesla_get_workspace_layout(B, H, N, D, ratio)
+    lay = sba.sagesla_get_workspace_layout(B, H, N, D, ratio, quant=quant, pv_fp8=pv_fp8)
     ws = sba.alloc_workspace(lay["total_bytes"], dev)
     nb, kk, W = lay["nb"], lay["k"], lay["mask_words"]
     res = {"layout": lay, "ws": ws}
@@ -49,7 +50,8 @@ def gpu_run(q, k, v, ratio, out_dtype=torch.float32, extras=True, device="cuda:0
                   mask_out=torch.empty(B * H * nb * W, dtype=torch.int32, device=dev),
                   scores_out=torch.empty(B * H * nb * nb, dtype=torch.float32, device=dev),
                   sparse_out=torch.empty(B * H * N * D, dtype=torch.float32, device=dev))
-    out = sba.sagesla_forward(qd, kd, vd, ratio, out_dtype=out_dtype, workspace=ws, **kw)
+    out = sba.sagesla_forward(qd, kd, vd, ratio, out_dtype=out_dtype, workspace=ws,
+                              quant=quant, pv_fp8=pv_fp8, **kw)
     status = sba.sagesla_stream_status(None, ws)
     assert status == 0, sba.sagesla_status_string(status)
     res["out"] = out.float().cpu()
@@ -112,7 +114,7 @@ def check_mask(prep, gpu_kept: list) -> int:
 
 
 def compare_head(q, k, v, ratio, res, b: int, h: int, rows=None, check_codes=True,
-                 linear_tol=False):
+                 linear_tol=False, quant=True, pv_fp8=True):
     """Oracle vs GPU for one head: codes (bit-exact), mask, and the output of the query blocks
     in ``rows`` (default all). Returns (max abs error, ambiguous rows): the largest amount by
     which an element exceeds its allowance (ambiguous P codes and the row-sum window; with
@@ -122,7 +124,9 @@ def compare_head(q, k, v, ratio, res, b: int, h: int, rows=None, check_codes=Tru
     qh, kh, vh = (inputs.as_float64(x[b, h]) for x in (q, k, v))
     nb = res["layout"]["nb"]
     gpu_kept = [res["kept"][bh, i] for i in range(nb)]
-    prep, out = orc.forward_head(qh, kh, vh, ratio, rows=rows, kept_override=gpu_kept)
+    prep, out = orc.forward_head(qh, kh, vh, ratio, rows=rows, kept_override=gpu_kept,
+                                 quant=quant, pv_fp8=pv_fp8)
+    check_codes = check_codes and quant      # quant off: the oracle forms no codes
     ambiguous = check_mask(prep, gpu_kept)
     # the mask words and the kept lists agree
     assert all(np.array_equal(a, bb) for a, bb in

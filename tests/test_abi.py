@@ -131,3 +131,38 @@ def test_host_entry_rejects_bad_arguments():
                                     1, None, 0, None) == 2
     assert lib.sagesla_forward_host(p, p, p, 1, 1, 64, 128, 0.1, 64, ctypes.c_void_p(o.data_ptr()),
                                     1, None, 0, None) == 3
+
+
+def test_operand_modes_workspace_and_validation():
+    """The 16-bit modes add bf16 copies of their operands to the workspace (Q and K for
+    quant = 0, V for pv_fp8 = 0); bf16 Q.K^T with e4m3 P.V is not a mode."""
+    B, H, N = 1, 3, 1000
+    base = sba.sagesla_workspace_size(B, H, N, 128, 0.2)
+    n_pad = sba.sagesla_get_workspace_layout(B, H, N, 128, 0.2)["n_pad"]
+    copy = B * H * n_pad * 256
+    lay_v = sba.sagesla_get_workspace_layout(B, H, N, 128, 0.2, pv_fp8=False)
+    lay_qkv = sba.sagesla_get_workspace_layout(B, H, N, 128, 0.2, quant=False, pv_fp8=False)
+    assert lay_v["qb"] == 0 and lay_v["kb"] == 0 and lay_v["vb"] >= base
+    assert lay_v["total_bytes"] >= base + copy
+    assert min(lay_qkv["qb"], lay_qkv["kb"], lay_qkv["vb"]) >= base
+    assert lay_qkv["total_bytes"] >= base + 3 * copy
+    assert all(lay_qkv[f] % 256 == 0 for f in ("qb", "kb", "vb"))
+    assert sba.sagesla_workspace_size(B, H, N, 128, 0.2, quant=False, pv_fp8=False) == lay_qkv["total_bytes"]
+    lib = binding.load_library()
+    opt = binding._options(quant=False, pv_fp8=True)
+    assert lib.sagesla_workspace_size_ex(B, H, N, 128, 0.2, 64, ctypes.byref(opt)) == 0
+    lay = binding.SageslaWorkspaceLayout()
+    assert lib.sagesla_get_workspace_layout_ex(B, H, N, 128, 0.2, 64, ctypes.byref(opt),
+                                               ctypes.byref(lay)) == 2     # UNSUPPORTED
+    opt = binding._options()
+    opt.quant = 3
+    assert lib.sagesla_get_workspace_layout_ex(B, H, N, 128, 0.2, 64, ctypes.byref(opt),
+                                               ctypes.byref(lay)) == 1     # INVALID_ARG
+
+
+def test_options_init_defaults():
+    opt = binding.SageslaOptions()
+    opt.debug_skip_tile = 7
+    binding.load_library().sagesla_options_init(ctypes.byref(opt))
+    assert opt.quant == 1 and opt.pv_fp8 == 1 and opt.debug_skip_tile == 0
+    assert not opt.kept_idx_out and not opt.stage_events

@@ -359,3 +359,36 @@ def test_e4m3_ambiguity_bound():
     np.testing.assert_allclose(amb, np.diff(grid))
     off = orc.e4m3_ambiguity(grid[1:], 1e-6)     # on the grid: unambiguous
     assert not off.any()
+
+
+def test_int8_logits_with_real_pv_equal_block_masked_attention_of_dequantized_q_k():
+    """SPEC 9.1 (INT8 Q.K^T, real P and V): the sparse branch equals softmax attention over
+    the kept blocks with the dequantized Q8 * sq and K8 * sk (the logits are the same numbers)
+    and the raw V, through the library routine."""
+    n = 300
+    q, k, v = _rand_head(n, 17, k_offset=1.0)
+    prep, out = orc.forward_head(q, k, v, 0.4, quant=True, pv_fp8=False)
+    qd = np.zeros_like(q)
+    kd = np.zeros_like(k)
+    for j in range(prep.nb):
+        r = orc.block_rows(j, n)
+        qd[r] = prep.q8[r] * float(prep.sq[j])
+        kd[r] = prep.k8[r] * float(prep.sk[j])
+    mask = np.zeros((n, n), dtype=bool)
+    for i in range(prep.nb):
+        for j in prep.kept[i]:
+            mask[orc.block_rows(i, n), orc.block_rows(int(j), n)] = True
+    ref = _sdpa64(qd, kd, v, mask)
+    o_s = np.concatenate([out[i]["o_s"] for i in range(prep.nb)])
+    np.testing.assert_allclose(o_s, ref, rtol=0, atol=1e-10)
+
+
+def test_real_pv_allowance_is_the_branch_of_abs_v():
+    """The bf16-P allowance of the real-P.V modes is BF16_PV_REL times the same weights applied
+    to |v|: with V >= 0 it equals BF16_PV_REL times the output itself."""
+    q, k, v = _rand_head(200, 18)
+    v = np.abs(v)
+    for quant in (False, True):
+        _, out = orc.forward_head(q, k, v, 0.5, quant=quant, pv_fp8=False)
+        for r in out.values():
+            np.testing.assert_allclose(r["o_s_ambig"], orc.BF16_PV_REL * r["o_s"], rtol=1e-12)

@@ -17,7 +17,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsagesla.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
-SOURCES = ["sagesla_api.cu", "prologue.cu", "topk.cu", "linear.cu", "attention.cu", "no_alloc.cu",
+SOURCES = ["sagesla_api.cu", "prologue.cu", "topk.cu", "linear.cu", "attention.cu",
+           "attention_dense.cu", "no_alloc.cu",
            "norm.cu", "w8a8.cu", "backward.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",

@@ -99,6 +99,11 @@ struct AttnTestHooks {
 cudaError_t launch_attention(const ForwardPlan& p, TensorArg q, void* out, int32_t out_dtype,
                              int64_t out_sb, int64_t out_sh, int64_t out_sn, float* sparse_out,
                              char* ws, const AttnTestHooks& hooks, cudaStream_t stream);
+// Dense mode (every key block kept, INT8 / e4m3 operands): M=128 tiles over all key blocks.
+cudaError_t launch_attention_dense(const ForwardPlan& p, TensorArg q, void* out, int32_t out_dtype,
+                                   int64_t out_sb, int64_t out_sh, int64_t out_sn,
+                                   float* sparse_out, char* ws, const AttnTestHooks& hooks,
+                                   cudaStream_t stream);
 cudaError_t launch_scale_scores(const ForwardPlan& p, const char* ws, float* scores_out,
                                 cudaStream_t stream);
 

@@ -360,9 +360,14 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
     hooks.spin_limit_us = opt->debug_spin_limit_us;
     hooks.skip_tile = opt->debug_skip_tile != 0;
   }
-  SAGESLA_LAUNCH(launch_attention(p, qa, out->data, out->dtype, out->stride_b, out->stride_h,
-                                  out->stride_n, opt ? opt->sparse_out : nullptr, ws, hooks,
-                                  stream));
+  if (p.linear_empty && p.quant && p.pv_fp8)
+    SAGESLA_LAUNCH(launch_attention_dense(p, qa, out->data, out->dtype, out->stride_b,
+                                          out->stride_h, out->stride_n,
+                                          opt ? opt->sparse_out : nullptr, ws, hooks, stream));
+  else
+    SAGESLA_LAUNCH(launch_attention(p, qa, out->data, out->dtype, out->stride_b, out->stride_h,
+                                    out->stride_n, opt ? opt->sparse_out : nullptr, ws, hooks,
+                                    stream));
   SAGESLA_LAUNCH(mark(SAGESLA_N_STAGES));
   if (opt) {
     if (opt->kept_idx_out)

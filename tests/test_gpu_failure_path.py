@@ -21,14 +21,16 @@ pytestmark = pytest.mark.gpu
 TIMEOUT = 5   # SAGESLA_ERR_TIMEOUT
 
 
-def test_skipped_tile_times_out_and_the_next_call_is_clean():
+@pytest.mark.parametrize("ratio", [0.1, 1.0])
+def test_skipped_tile_times_out_and_the_next_call_is_clean(ratio):
+    """Ratio 0.1 runs the sparse attention kernel, ratio 1 the dense-mode kernel."""
     q, k, v = (x.cuda() for x in inputs.make_random(1, 2, 2048, 61, k_offset_std=1.0))
     B, H, N, D = q.shape
-    ws = sba.alloc_workspace(sba.sagesla_workspace_size(B, H, N, D, 0.1))
+    ws = sba.alloc_workspace(sba.sagesla_workspace_size(B, H, N, D, ratio))
     out = torch.zeros(q.shape, dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    sba.sagesla_forward(q, k, v, 0.1, out=out, workspace=ws, debug_spin_limit_us=10000,
+    sba.sagesla_forward(q, k, v, ratio, out=out, workspace=ws, debug_spin_limit_us=10000,
                         debug_skip_tile=True)
     status = sba.sagesla_stream_status(None, ws)
     elapsed = time.perf_counter() - t0
@@ -36,12 +38,12 @@ def test_skipped_tile_times_out_and_the_next_call_is_clean():
     assert elapsed < 5.0, elapsed               # bounded: a few 10 ms limits, not the 2 s one
     # the CTAs that were not starved wrote their rows: all but the first two query blocks of
     # head 0 (the starved CTA's), whose rows may be left unwritten
-    ref = gpu_run(q.cpu(), k.cpu(), v.cpu(), 0.1, extras=False)["out"]
+    ref = gpu_run(q.cpu(), k.cpu(), v.cpu(), ratio, extras=False)["out"]
     got = out.cpu()
     assert torch.equal(got[:, 0, 128:], ref[:, 0, 128:])
     assert torch.equal(got[:, 1], ref[:, 1])
     # the same workspace, normal call: status clean, output equal to a fresh workspace's
-    out2 = sba.sagesla_forward(q, k, v, 0.1, workspace=ws)
+    out2 = sba.sagesla_forward(q, k, v, ratio, workspace=ws)
     assert sba.sagesla_stream_status(None, ws) == 0
     assert torch.equal(out2.cpu(), ref)
 

@@ -30,14 +30,16 @@
 // Each half owns 48 KB of shared memory (its Q rows, the K8 pair, a 3-stage V8 ring), reused
 // for the linear-branch operands once its main loop is done; its P tile sits after both halves.
 //
-// Softmax arithmetic per score: the int32 score becomes a float exactly (|S| < 2^21) by one
-// conversion each (measured ~2.5% faster for the whole kernel than forming it through the
-// 1.5*2^23 bias with an integer add and a packed f32x2 subtract), and the block's row maximum
-// is taken on those floats with three-input maxima (about 1% faster than 32 integer maxima);
+// Softmax arithmetic per score: the block's row maximum is taken on the int32 scores (integer
+// maxima), and each score becomes a float exactly (|S| < 2^21) by one conversion inside the
+// exponential loop, where it overlaps the MUFU work (measured ~1% faster than converting all
+// scores first and taking three-input float maxima, and ~2.5% faster than forming the floats
+// through the 1.5*2^23 bias with an integer add and a packed f32x2 subtract);
 // one packed FFMA forms the base-2 exponent with the factor 448 of the P quantization folded in; 2^x
 // comes from the MUFU ex2 unit (measured faster here than moving part of the exponentials to
 // a polynomial on the FMA pipe: the loop is bound by latency, not by MUFU throughput).
 #include <cuda_bf16.h>
+#include <climits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -205,13 +207,24 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// With kInt, converts the row's int32 scores to floats in place (exact: |S| < 2^21); returns
-// the largest of the first `valid` scores, by three-input maxima in four chains.
+// Largest of the first `valid` scores as a float: for int32 scores integer maxima in four
+// chains (the conversion to float happens in the exponential loop), for float scores
+// three-input float maxima.
 template <bool kFull, bool kInt>
 __device__ __forceinline__ float row_block_fmax(uint32_t (&a)[32], int valid) {
   if (kInt) {
+    int m[4];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__int2float_rn(static_cast<int>(a[q])));
+    for (int c = 0; c < 4; ++c) {
+      int x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int q = 8 * c + u;
+        x[u] = (kFull || q < valid) ? static_cast<int>(a[q]) : INT_MIN;
+      }
+      m[c] = max(max(max(x[0], x[1]), max(x[2], x[3])), max(max(x[4], x[5]), max(x[6], x[7])));
+    }
+    return __int2float_rn(max(max(m[0], m[1]), max(m[2], m[3])));
   }
   float m[4];
 #pragma unroll
@@ -228,7 +241,7 @@ __device__ __forceinline__ float row_block_fmax(uint32_t (&a)[32], int valid) {
 }
 // 448 p = 2^(S c + neg) for the thread's 32 scores: returns their sum and packs them into
 // the P operand, as e4m3 codes (kP8: pk[0..7]) or as bf16 values (pk[0..15]).
-template <bool kFull, bool kP8>
+template <bool kFull, bool kP8, bool kInt>
 __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int valid, float c,
                                               float neg, uint32_t (&pk)[16]) {
   const unsigned long long c2 = pk2(c, c), neg2 = pk2(neg, neg);
@@ -238,7 +251,9 @@ __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int vali
     float y[4];
 #pragma unroll
     for (int t = 0; t < 4; t += 2) {
-      const unsigned long long f2 = pk2(__uint_as_float(sr[q + t]), __uint_as_float(sr[q + t + 1]));
+      const unsigned long long f2 =
+          kInt ? pk2(__int2float_rn(static_cast<int>(sr[q + t])), __int2float_rn(static_cast<int>(sr[q + t + 1])))
+               : pk2(__uint_as_float(sr[q + t]), __uint_as_float(sr[q + t + 1]));
       float x0, x1;
       up2(fma2(f2, c2, neg2), x0, x1);
       y[t] = ex2_mufu(x0);
@@ -548,8 +563,8 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float alpha = ex2_mufu(m_run - m_new);
         const float neg = kLog2_448 - m_new;    // 2^(S c + neg) = 448 p
         uint32_t pk[16];
-        const float rs = full ? row_exp_pack<true, kPV8>(sr, 32, cst, neg, pk)
-                              : row_exp_pack<false, kPV8>(sr, valid, cst, neg, pk);
+        const float rs = full ? row_exp_pack<true, kPV8, kQK8>(sr, 32, cst, neg, pk)
+                              : row_exp_pack<false, kPV8, kQK8>(sr, valid, cst, neg, pk);
         l_part = alpha * l_part + rs;
         m_run = m_new;
         // P.V(n-1) must be done: it frees P buffer b (read by P.V(n-2) before it), makes O

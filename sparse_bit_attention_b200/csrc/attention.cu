@@ -159,6 +159,9 @@ struct AttnParams {
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ctl* ctl,
                                               int* status, unsigned long long limit_ns) {
+  // A completed phase is safe to pass; the CTA's abort flag (a shared-memory load) is read only
+  // when the wait would block (measured: 6% of the sparse kernel's time at 14B-720P).
+  if (mbar_try_wait(bar, parity)) return true;
   if (ctl->abort) return false;
   if (!mbar_wait(bar, parity, status, limit_ns)) {
     ctl->abort = 1;

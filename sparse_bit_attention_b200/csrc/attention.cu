@@ -215,7 +215,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // three-input float maxima.
 template <bool kFull, bool kInt>
 __device__ __forceinline__ float row_block_fmax(uint32_t (&a)[32], int valid) {
-  if (kInt) {
+  if constexpr (kInt) {
     int m[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {

@@ -46,7 +46,10 @@ typedef enum {
   SAGESLA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
   SAGESLA_ERR_TIMEOUT = 5,      /* a device-side wait exceeded its limit (see stream_status) */
   SAGESLA_ERR_DEVICE_CHECK = 6, /* a device-side consistency check failed */
-  SAGESLA_ERR_NO_DEVICE = 7     /* no sm_100 device is current */
+  SAGESLA_ERR_NO_DEVICE = 7,    /* no sm_100 device is current */
+  SAGESLA_ERR_BOUNDS = 8,       /* bounds-checking build: an index or TMA coordinate was out of
+                                 * range; the access was skipped (see sagesla_build_checks) */
+  SAGESLA_ERR_CANARY = 9        /* debug_checks: a workspace canary was overwritten */
 } sagesla_status;
 
 typedef enum { SAGESLA_BF16 = 0, SAGESLA_F32 = 1 } sagesla_dtype;
@@ -101,16 +104,39 @@ typedef struct {
    * (sagesla_workspace_size_ex with the same options) and run one CTA per SM. */
   int32_t quant;
   int32_t pv_fp8;
+  /* debug_checks = 1: the call writes a 16-byte canary after every workspace region before
+   * its first kernel and verifies them all after its last one, on the stream; a damaged
+   * canary leaves SAGESLA_ERR_CANARY in the status word (read it with sagesla_stream_status).
+   * Two extra kernels, nothing else changes.
+   * debug_plant (failure-path tests, host-side fault injection; 0 in normal use):
+   *   1 = after the canaries are written, overwrite one of them (needs debug_checks = 1): the
+   *       call ends with SAGESLA_ERR_CANARY;
+   *   2 = after the Top-K selection, overwrite the first kept-list entry with -1: the
+   *       bounds-checking build (sagesla_build_checks() == 1) skips the access and ends with
+   *       SAGESLA_ERR_BOUNDS; the normal build rejects this value (SAGESLA_ERR_UNSUPPORTED).
+   * Other values: SAGESLA_ERR_INVALID_ARG. */
+  int32_t debug_checks;
+  int32_t debug_plant;
 } sagesla_options;
 
 /* Fills *opt with the defaults: every pointer NULL, test hooks 0, quant = pv_fp8 = 1. */
 void sagesla_options_init(sagesla_options* opt);
 
+/* 1 for the bounds-checking build of this library (compiled with SAGESLA_CHECKS=1:
+ * libsagesla_checks.so), 0 for the normal build. In the checking build every kept-list entry
+ * a kernel reads, every Top-K output position and every TMA row coordinate of the attention
+ * kernels is checked before use; a failed check records SAGESLA_ERR_BOUNDS in the status
+ * word, the access is skipped, and the CTA stops (no trap, no assert: the context stays
+ * usable). */
+int sagesla_build_checks(void);
+
 #define SAGESLA_N_STAGES 7
 
 /* Offsets (bytes, from the workspace start) of the intermediates a forward call leaves in
  * its workspace, for inspection after the stream has completed. Per-head arrays are
- * contiguous over B*H; n_pad = 128*ceil(nb/2) token rows per head. */
+ * contiguous over B*H; n_pad = 128*ceil(nb/2) token rows per head. Regions start on 256-byte
+ * boundaries, and at least 16 bytes separate the end of each region from the next one: the
+ * 16 bytes at the end rounded up to 16 hold the region's canary when debug_checks is set. */
 typedef struct {
   size_t total_bytes;
   int64_t nb, k, n_pad, mask_words, nb_k_pad, nb_m_pad;

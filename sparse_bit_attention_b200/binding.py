@@ -6,6 +6,7 @@ or fails to load, every call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -13,6 +14,8 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsagesla.so")
+# the bounds-checking build of the same sources (SAGESLA_CHECKS=1)
+LIB_CHECKS_PATH = os.path.join(_PKG, "libsagesla_checks.so")
 
 SAGESLA_BF16 = 0
 SAGESLA_F32 = 1
@@ -22,7 +25,8 @@ HEAD_DIM = 128
 STATUS_NAMES = {
     0: "SAGESLA_OK", 1: "SAGESLA_ERR_INVALID_ARG", 2: "SAGESLA_ERR_UNSUPPORTED",
     3: "SAGESLA_ERR_WORKSPACE", 4: "SAGESLA_ERR_CUDA", 5: "SAGESLA_ERR_TIMEOUT",
-    6: "SAGESLA_ERR_DEVICE_CHECK", 7: "SAGESLA_ERR_NO_DEVICE",
+    6: "SAGESLA_ERR_DEVICE_CHECK", 7: "SAGESLA_ERR_NO_DEVICE", 8: "SAGESLA_ERR_BOUNDS",
+    9: "SAGESLA_ERR_CANARY",
 }
 
 
@@ -49,7 +53,8 @@ class SageslaOptions(ctypes.Structure):
                 ("scores_out", ctypes.c_void_p), ("sparse_out", ctypes.c_void_p),
                 ("stage_events", ctypes.POINTER(ctypes.c_void_p)),
                 ("debug_spin_limit_us", ctypes.c_uint32), ("debug_skip_tile", ctypes.c_int32),
-                ("quant", ctypes.c_int32), ("pv_fp8", ctypes.c_int32)]
+                ("quant", ctypes.c_int32), ("pv_fp8", ctypes.c_int32),
+                ("debug_checks", ctypes.c_int32), ("debug_plant", ctypes.c_int32)]
 
 
 def _options(quant: bool = True, pv_fp8: bool = True) -> SageslaOptions:
@@ -98,6 +103,7 @@ _SIGNATURES = {
     "sagesla_get_workspace_layout": (ctypes.c_int, [ctypes.c_int64] * 4 + [
         ctypes.c_double, ctypes.c_int, ctypes.POINTER(SageslaWorkspaceLayout)]),
     "sagesla_options_init": (None, [ctypes.c_void_p]),
+    "sagesla_build_checks": (ctypes.c_int, []),
     "sagesla_workspace_size_ex": (ctypes.c_size_t, [ctypes.c_int64] * 4 + [
         ctypes.c_double, ctypes.c_int, ctypes.c_void_p]),
     "sagesla_get_workspace_layout_ex": (ctypes.c_int, [ctypes.c_int64] * 4 + [
@@ -137,11 +143,7 @@ NO_ALLOC_SCRATCH_BYTES = 64 << 20
 _lib = None
 
 
-def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Loads libsagesla.so (built by ``python -m sparse_bit_attention_b200.build``)."""
-    global _lib
-    if _lib is not None:
-        return _lib
+def _open(path: str) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m sparse_bit_attention_b200.build` (there is no fallback)")
@@ -150,8 +152,40 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
-    _lib = lib
     return lib
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libsagesla.so (built by ``python -m sparse_bit_attention_b200.build``); every
+    call of this module goes to it (see ``using_library`` for another build)."""
+    global _lib
+    if _lib is None:
+        _lib = _open(path)
+    return _lib
+
+
+_checks_lib = None
+
+
+def load_checks_library() -> ctypes.CDLL:
+    """Loads the bounds-checking build libsagesla_checks.so (``python -m
+    sparse_bit_attention_b200.build --checks``) beside the normal one."""
+    global _checks_lib
+    if _checks_lib is None:
+        _checks_lib = _open(LIB_CHECKS_PATH)
+    return _checks_lib
+
+
+@contextlib.contextmanager
+def using_library(lib: ctypes.CDLL):
+    """Routes this module's calls to ``lib`` (e.g. the checking build) inside the block."""
+    global _lib
+    prev = load_library()
+    _lib = lib
+    try:
+        yield lib
+    finally:
+        _lib = prev
 
 
 def exported_symbols() -> list[str]:
@@ -223,14 +257,18 @@ def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_rati
                     out_dtype: torch.dtype = torch.float32, kept_idx_out=None, mask_out=None,
                     scores_out=None, sparse_out=None, stage_events=None,
                     debug_spin_limit_us: int = 0, debug_skip_tile: bool = False,
-                    quant: bool = True, pv_fp8: bool = True) -> torch.Tensor:
+                    quant: bool = True, pv_fp8: bool = True, debug_checks: bool = False,
+                    debug_plant: int = 0) -> torch.Tensor:
     """SageSLA forward on device tensors q, k, v (bf16 [B, H, N, 128]); returns ``out``.
 
     ``stage_events``: optional list of N_STAGES + 1 torch.cuda.Event(enable_timing=True)
     recorded around each kernel of the forward on the launching stream.
     ``debug_spin_limit_us`` / ``debug_skip_tile``: the failure-path test hooks of
     sagesla_options (0 / False in normal use). ``quant`` / ``pv_fp8``: the operand mode
-    (INT8 Q.K^T / e4m3 P.V by default; False selects bf16)."""
+    (INT8 Q.K^T / e4m3 P.V by default; False selects bf16). ``debug_checks``: workspace
+    canaries written before and verified after the call (the result lands in the status word:
+    ``sagesla_stream_status``); ``debug_plant``: host-side fault injection of the failure-path
+    tests (1: a damaged canary, 2: an out-of-range kept index, checking build only)."""
     lib = load_library()
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
@@ -244,8 +282,10 @@ def sagesla_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_rati
             ctypes.byref(vo), ctypes.c_void_p(workspace.data_ptr()),
             workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_ptr(stream)))
     if (any(x is not None for x in extra) or stage_events is not None or debug_spin_limit_us
-            or debug_skip_tile or not quant or not pv_fp8):
+            or debug_skip_tile or not quant or not pv_fp8 or debug_checks or debug_plant):
         opt = _options(quant, pv_fp8)
+        opt.debug_checks = 1 if debug_checks else 0
+        opt.debug_plant = int(debug_plant)
         for name, x in zip(("kept_idx_out", "mask_out", "scores_out", "sparse_out"), extra):
             if x is not None:
                 setattr(opt, name, x.data_ptr())

@@ -134,6 +134,12 @@ __device__ __forceinline__ int kept_at(const Ctl* ctl, int h, const int32_t* kli
   return n < kListCap ? static_cast<int>(ctl->klist[h][n]) : __ldg(klist + n);
 }
 
+// A block index as used for a load that runs ahead of its bounds check: unchanged in the
+// normal build, clamped into [0, nb) in the checking build.
+__device__ __forceinline__ int clamp_block(int j, int nb) {
+  return kChecks ? min(max(j, 0), nb - 1) : j;
+}
+
 // n-th kept key block of a query block: its kept list, or block n itself when every block is
 // kept (no list).
 __device__ __forceinline__ int kept_block(const int32_t* klist, int n) {
@@ -356,6 +362,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // A 16-bit tile of 128 channels arrives as two boxes of 64 channels (x = 0, 64).
       for (int h = 0; h < 2; ++h) {
         if (U[h] == 0) continue;
+        if (!in_range(128 * pair + 64 * h, prm.n_pad, status)) { ctl->abort = 1; break; }
         mbar_arrive_expect_tx(&ctl->hc[h].q_full, L::kQBytes);
         uint8_t* qst = smem + h * kHalfBytes + kHQ;
         tma_load_2d(qst, &tm_q, &ctl->hc[h].q_full, 0, row_base + 128 * pair + 64 * h);
@@ -374,10 +381,16 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           // Failure-path test: the first pair of CTA (0, 0) is never loaded, so the waits for
           // it run out (nothing is left in flight: neither its bytes nor its copies exist).
           if (prm.skip_tile && n0 == 0 && h == 0 && pair == 0 && bh == 0) continue;
+          int jk[2] = {kept_at(ctl, h, klist, n0), two > 1 ? kept_at(ctl, h, klist, n0 + 1) : 0};
+          if (kChecks && !(in_range(jk[0], prm.nb, status) && in_range(jk[1], prm.nb, status))) {
+            ctl->abort = 1;     // checking build: the out-of-range tile is not loaded
+            ok = false;
+            break;
+          }
           mbar_arrive_expect_tx(&c.k_full, two * L::kKBlock);
           uint8_t* kst = smem + h * kHalfBytes + kHK;
           for (int b = 0; b < two; ++b) {
-            const int y = row_base + 64 * kept_at(ctl, h, klist, n0 + b);
+            const int y = row_base + 64 * jk[b];
             tma_load_2d(kst + b * kChunk, &tm_k, &c.k_full, 0, y);
             if (!kQK8) tma_load_2d(kst + 2 * kChunk + b * kChunk, &tm_k, &c.k_full, 64, y);
           }
@@ -390,9 +403,11 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int s = n % kNV;
             if (n >= kNV && !(ok = wait_or_abort(&c.v_empty[s], ((n / kNV) - 1) & 1, ctl, status, prm.spin_ns))) break;
             const int32_t* klist = prm.kept ? prm.kept + (bh * prm.nb + ia + h) * static_cast<int64_t>(prm.k) : nullptr;
+            const int jv = kept_at(ctl, h, klist, n);
+            if (!in_range(jv, prm.nb, status)) { ctl->abort = 1; ok = false; break; }
             mbar_arrive_expect_tx(&c.v_full[s], L::kVBlock);
             uint8_t* vst = smem + h * kHalfBytes + kHV + s * L::kVBlock;
-            const int y = row_base + 64 * kept_at(ctl, h, klist, n);
+            const int y = row_base + 64 * jv;
             tma_load_2d(vst, &tm_v, &c.v_full[s], 0, y);
             if (!kPV8) tma_load_2d(vst + kChunk, &tm_v, &c.v_full[s], 64, y);
           }
@@ -402,6 +417,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (U[h] == 0) continue;
         HalfCtl& c = ctl->hc[h];
         if (!(ok = wait_or_abort(&c.mma_done, 0, ctl, status, prm.spin_ns))) break;
+        if (!(ok = in_range(ia + h, prm.nb_m_pad, status))) { ctl->abort = 1; break; }
         const int gy = static_cast<int>((bh * prm.nb_m_pad + ia + h) * 129);
         uint8_t* hb = smem + h * kHalfBytes;
         mbar_arrive_expect_tx(&c.g_full, 32768u);
@@ -539,13 +555,20 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // of the loop waits for another one
       int j_cur = kept_block(klist, 0);
       int j_ahead = Uh > 1 ? kept_block(klist, 1) : 0;
-      float sk_next = kQK8 ? __ldg(skh + j_cur) : 1.f;
+      // (the scale loads run ahead of the checks: the checking build clamps their index)
+      float sk_next = kQK8 ? __ldg(skh + clamp_block(j_cur, prm.nb)) : 1.f;
       for (int n = 0; n < Uh; ++n) {
         const int b = n & 1;
         const int j = j_cur;
         const float skj = sk_next;
+        // checking build: an out-of-range kept entry stops the CTA before it is used
+        if (kChecks && !__all_sync(0xffffffffu, in_range(j, prm.nb, status))) {
+          ctl->abort = 1;
+          ok = false;
+          break;
+        }
         if (n + 1 < Uh) {
-          if (kQK8) sk_next = __ldg(skh + j_ahead);
+          if (kQK8) sk_next = __ldg(skh + clamp_block(j_ahead, prm.nb));
           j_cur = j_ahead;
           if (n + 2 < Uh) j_ahead = kept_block(klist, n + 2);
         }

@@ -256,7 +256,8 @@ k_attention_dense(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   if (warp == kDProducer) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (lane == 0 && !in_range(128 * pair + 64, prm.n_pad, status)) ctl->abort = 1;
+    else if (lane == 0) {
       mbar_arrive_expect_tx(&ctl->q_full, 2 * kTile);
       tma_load_2d(smem + kOffQ, &tm_q, &ctl->q_full, 0, row_base + 128 * pair);
       tma_load_2d(smem + kOffQ + kTile, &tm_q, &ctl->q_full, 0, row_base + 128 * pair + 64);
@@ -264,6 +265,7 @@ k_attention_dense(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int s = n % kStages;
         const uint32_t par = ((n / kStages) - 1) & 1;
         if (n >= kStages && !dwait(&ctl->k_empty[s], par, ctl, status, prm.spin_ns)) break;
+        if (!in_range(64 * n, prm.n_pad, status)) { ctl->abort = 1; break; }
         // failure-path test: the first K tile of CTA (0, 0) is never loaded
         if (!(prm.skip_tile && n == 0 && pair == 0 && bh == 0)) {
           mbar_arrive_expect_tx(&ctl->k_full[s], kTile);

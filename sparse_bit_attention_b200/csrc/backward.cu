@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(1024) k_bwd_list_scan(int nb, const int32_t* _
 
 __global__ void k_bwd_list_fill(int nb, int k, int mask_words, int64_t BH,
                                 const uint32_t* __restrict__ mask, const int32_t* __restrict__ toff,
-                                int32_t* __restrict__ tlist) {
+                                int32_t* __restrict__ tlist, int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
   if (w >= BH * nb) return;
@@ -208,7 +208,9 @@ __global__ void k_bwd_list_fill(int nb, int k, int mask_words, int64_t BH,
     const int i = i0 + lane;
     const bool kept = i < nb && ((__ldg(mcol + static_cast<int64_t>(i) * mask_words) >> (j & 31)) & 1u);
     const uint32_t bits = __ballot_sync(0xffffffffu, kept);
-    if (kept) out[count + __popc(bits & ((1u << lane) - 1u))] = i;
+    const int pos = count + __popc(bits & ((1u << lane) - 1u));
+    if (kept && in_range(toff[bh * (nb + 1) + j] + pos, static_cast<long long>(nb) * k, status))
+      out[pos] = i;
     count += __popc(bits);
   }
 }
@@ -355,7 +357,12 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           ok = false;
           break;
         }
-        const int jm = blk0 + __ldg(klist + m);
+        const int jk = __ldg(klist + m);
+        if (!in_range(jk, prm.nb, prm.status)) {   // checking build: the tile is not loaded
+          ok = false;
+          break;
+        }
+        const int jm = blk0 + jk;
         mbar_arrive_expect_tx(&k_full[b], kTile);
         load_tile(k_t + b * kTile, &tm_k, &k_full[b], jm);
         mbar_arrive_expect_tx(&v_full[b], kTile);
@@ -551,7 +558,12 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
           ok = false;
           break;
         }
-        const int jm = blk0 + __ldg(klist + m);
+        const int jk = __ldg(klist + m);
+        if (!in_range(jk, prm.nb, prm.status)) {   // checking build: the tile is not loaded
+          ok = false;
+          break;
+        }
+        const int jm = blk0 + jk;
         mbar_arrive_expect_tx(&kv_full[b], 2 * kTile);
         load_tile(k_t + b * kTile, &tm_k, &kv_full[b], jm);
         load_tile(v_t + b * kTile, &tm_v, &kv_full[b], jm);
@@ -748,7 +760,12 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             ok = false;
             break;
           }
-          const int im = blk0 + __ldg(ilist + m);
+          const int ik = __ldg(ilist + m);
+          if (!in_range(ik, prm.nb, prm.status)) {   // checking build: the tile is not loaded
+            ok = false;
+            break;
+          }
+          const int im = blk0 + ik;
           mbar_arrive_expect_tx(&qo_full[b], 2 * kTile);
           load_tile(q_t + b * kTile, &tm_q, &qo_full[b], im);
           load_tile(o_t + b * kTile, &tm_do, &qo_full[b], im);
@@ -1323,7 +1340,8 @@ cudaError_t launch_sla_backward(const ForwardPlan& p, const BackwardLayout& bl, 
     k_bwd_list_fill<<<lgrid, 256, 0, stream>>>(static_cast<int>(p.nb), static_cast<int>(p.k),
                                                static_cast<int>(p.mask_words), p.BH, mask,
                                                reinterpret_cast<const int32_t*>(ws + bl.toff),
-                                               reinterpret_cast<int32_t*>(ws + bl.tlist));
+                                               reinterpret_cast<int32_t*>(ws + bl.tlist),
+                                               reinterpret_cast<int*>(ws + p.lay.status));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   CUtensorMap tq, tk, tv, td;

@@ -35,6 +35,20 @@ __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Bounds checks of the checking build (compiled with -DSAGESLA_CHECKS=1): in_range records
+// SAGESLA_ERR_BOUNDS and returns false when i is outside [0, n), and the caller skips the
+// access. In the normal build it is the constant true and the checks compile away.
+#ifndef SAGESLA_CHECKS
+#define SAGESLA_CHECKS 0
+#endif
+constexpr bool kChecks = SAGESLA_CHECKS != 0;
+__device__ __forceinline__ bool in_range(long long i, long long n, int* status) {
+  if (!kChecks) return true;
+  if (i >= 0 && i < n) return true;
+  record_error(status, SAGESLA_ERR_BOUNDS);
+  return false;
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -17,6 +17,8 @@ struct TensorArg {
   int32_t H;
 };
 
+constexpr int kMaxCanaries = 32;
+
 struct ForwardPlan {
   int64_t B, H, N, BH;
   int64_t nb;          // key/query blocks per head
@@ -32,6 +34,9 @@ struct ForwardPlan {
   bool quant;          // INT8 Q.K^T (else bf16 Q.K^T from packed bf16 copies)
   bool pv_fp8;         // e4m3 P.V (else bf16 P and raw bf16 V)
   sagesla_workspace_layout lay;
+  // canary of each workspace region: 16 bytes at the region's end rounded up to 16
+  int32_t n_canary;
+  uint64_t canary[kMaxCanaries];
 };
 
 // Fills plan from the problem size and operand mode; returns false for invalid arguments.
@@ -104,6 +109,10 @@ cudaError_t launch_attention_dense(const ForwardPlan& p, TensorArg q, void* out,
                                    int64_t out_sb, int64_t out_sh, int64_t out_sn,
                                    float* sparse_out, char* ws, const AttnTestHooks& hooks,
                                    cudaStream_t stream);
+// debug_checks: write the canary pattern after every workspace region / verify it (a damaged
+// canary records SAGESLA_ERR_CANARY in the status word).
+cudaError_t launch_canary_fill(const ForwardPlan& p, char* ws, cudaStream_t stream);
+cudaError_t launch_canary_verify(const ForwardPlan& p, char* ws, cudaStream_t stream);
 cudaError_t launch_scale_scores(const ForwardPlan& p, const char* ws, float* scores_out,
                                 cudaStream_t stream);
 

@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -68,9 +69,13 @@ bool make_plan(int64_t B, int64_t H, int64_t N, double topk_ratio, ForwardPlan* 
   sagesla_workspace_layout& L = p->lay;
   const int64_t BH = p->BH, nb = p->nb, nbq = 2 * p->n_pairs;
   size_t off = 0;
+  // Each region starts on a kAlign boundary and is followed by its 16-byte canary (used by
+  // debug_checks) at its end rounded up to 16.
   auto take = [&](size_t bytes) {
     const size_t at = off;
-    off = align_up(off + bytes, kAlign);
+    const size_t canary = align_up(at + bytes, 16);
+    if (p->n_canary < kMaxCanaries) p->canary[p->n_canary++] = canary;
+    off = align_up(canary + 16, kAlign);
     return at;
   };
   L.nb = nb;
@@ -202,6 +207,15 @@ sagesla_status check_device() { return require_b200(); }
     if ((call) != cudaSuccess) return SAGESLA_ERR_CUDA; \
   } while (0)
 
+// NVTX range around the launches of one stage (named "sagesla/<stage>"), so that a timeline
+// or an ncu --nvtx filter can find each kernel of a call; a no-op without a tool attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 }  // namespace
 
 // The current device must be a compute-capability-10.0 part (B200).
@@ -232,6 +246,8 @@ const char* sagesla_status_string(sagesla_status s) {
     case SAGESLA_ERR_TIMEOUT: return "device-side wait timed out";
     case SAGESLA_ERR_DEVICE_CHECK: return "device-side check failed";
     case SAGESLA_ERR_NO_DEVICE: return "no sm_100 device current";
+    case SAGESLA_ERR_BOUNDS: return "index or coordinate out of range (access skipped)";
+    case SAGESLA_ERR_CANARY: return "workspace canary overwritten";
   }
   return "unknown status";
 }
@@ -240,6 +256,8 @@ int64_t sagesla_topk_count(int64_t N, double topk_ratio, int block) {
   if (N < 1 || block != kBlock || !valid_ratio(topk_ratio)) return -1;
   return topk_count(ceil_div(N, kBlock), topk_ratio);
 }
+
+int sagesla_build_checks(void) { return kChecks ? 1 : 0; }
 
 void sagesla_options_init(sagesla_options* opt) {
   if (!opt) return;
@@ -261,6 +279,11 @@ sagesla_status read_mode(const sagesla_options* opt, bool* quant, bool* pv_fp8) 
   if (opt->quant == 0 && opt->pv_fp8 == 1) return SAGESLA_ERR_UNSUPPORTED;
   *quant = opt->quant != 0;
   *pv_fp8 = opt->pv_fp8 != 0;
+  if (opt->debug_checks != 0 && opt->debug_checks != 1) return SAGESLA_ERR_INVALID_ARG;
+  if (opt->debug_plant < 0 || opt->debug_plant > 2) return SAGESLA_ERR_INVALID_ARG;
+  if (opt->debug_plant == 1 && !opt->debug_checks) return SAGESLA_ERR_INVALID_ARG;
+  // an out-of-range kept index is only safe where the kernels check it
+  if (opt->debug_plant == 2 && !kChecks) return SAGESLA_ERR_UNSUPPORTED;
   return SAGESLA_OK;
 }
 }  // namespace
@@ -336,39 +359,69 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
   auto mark = [&](int i) -> cudaError_t {
     return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), stream) : cudaSuccess;
   };
+  const bool checks = opt && opt->debug_checks;
+  const int plant = opt ? opt->debug_plant : 0;
   SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.lay.status, 0, sizeof(int32_t), stream));
+  if (checks) SAGESLA_LAUNCH(launch_canary_fill(p, ws, stream));
+  // failure-path test: damage the canary after the scores region (host-side injection)
+  if (plant == 1) SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.canary[13], 0, 4, stream));
+  NvtxRange call_range("sagesla/forward");
   SAGESLA_LAUNCH(mark(0));
-  SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
+  {
+    NvtxRange r("sagesla/stats");
+    SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
+  }
   SAGESLA_LAUNCH(mark(1));
-  SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
+  {
+    NvtxRange r("sagesla/finalize");
+    SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
+  }
   SAGESLA_LAUNCH(mark(2));
-  SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
-  if (!p.quant || !p.pv_fp8) SAGESLA_LAUNCH(launch_pack_bf16(p, qa, ka, va, ws, stream));
+  {
+    NvtxRange r("sagesla/quant");
+    SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
+    if (!p.quant || !p.pv_fp8) SAGESLA_LAUNCH(launch_pack_bf16(p, qa, ka, va, ws, stream));
+  }
   SAGESLA_LAUNCH(mark(3));
   // With every key block kept (k == nb) the selection is the identity: the scores are only
   // computed when asked for, and the kept lists and masks only written when asked for.
   const bool want_lists = opt && (opt->kept_idx_out || opt->mask_out);
-  if (!p.linear_empty || (opt && opt->scores_out)) SAGESLA_LAUNCH(launch_scores(p, ws, stream));
+  if (!p.linear_empty || (opt && opt->scores_out)) {
+    NvtxRange r("sagesla/scores");
+    SAGESLA_LAUNCH(launch_scores(p, ws, stream));
+  }
   SAGESLA_LAUNCH(mark(4));
-  if (!p.linear_empty) SAGESLA_LAUNCH(launch_topk(p, ws, stream));
-  else if (want_lists) SAGESLA_LAUNCH(launch_fill_all_kept(p, ws, stream));
+  {
+    NvtxRange r("sagesla/topk");
+    if (!p.linear_empty) SAGESLA_LAUNCH(launch_topk(p, ws, stream));
+    else if (want_lists) SAGESLA_LAUNCH(launch_fill_all_kept(p, ws, stream));
+  }
+  // failure-path test of the checking build: an out-of-range first kept index (-1)
+  if (plant == 2) SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.lay.kept, 0xFF, 4, stream));
   SAGESLA_LAUNCH(mark(5));
-  if (!p.linear_empty) SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
+  if (!p.linear_empty) {
+    NvtxRange r("sagesla/complement_gemm");
+    SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
+  }
   SAGESLA_LAUNCH(mark(6));
   AttnTestHooks hooks{};
   if (opt) {
     hooks.spin_limit_us = opt->debug_spin_limit_us;
     hooks.skip_tile = opt->debug_skip_tile != 0;
   }
-  if (p.linear_empty && p.quant && p.pv_fp8)
-    SAGESLA_LAUNCH(launch_attention_dense(p, qa, out->data, out->dtype, out->stride_b,
-                                          out->stride_h, out->stride_n,
-                                          opt ? opt->sparse_out : nullptr, ws, hooks, stream));
-  else
-    SAGESLA_LAUNCH(launch_attention(p, qa, out->data, out->dtype, out->stride_b, out->stride_h,
-                                    out->stride_n, opt ? opt->sparse_out : nullptr, ws, hooks,
-                                    stream));
+  {
+    NvtxRange r("sagesla/attention");
+    if (p.linear_empty && p.quant && p.pv_fp8)
+      SAGESLA_LAUNCH(launch_attention_dense(p, qa, out->data, out->dtype, out->stride_b,
+                                            out->stride_h, out->stride_n,
+                                            opt ? opt->sparse_out : nullptr, ws, hooks, stream));
+    else
+      SAGESLA_LAUNCH(launch_attention(p, qa, out->data, out->dtype, out->stride_b,
+                                      out->stride_h, out->stride_n,
+                                      opt ? opt->sparse_out : nullptr, ws, hooks, stream));
+  }
   SAGESLA_LAUNCH(mark(SAGESLA_N_STAGES));
+  if (checks) SAGESLA_LAUNCH(launch_canary_verify(p, ws, stream));
   if (opt) {
     if (opt->kept_idx_out)
       SAGESLA_LAUNCH(cudaMemcpyAsync(opt->kept_idx_out, ws + p.lay.kept,
@@ -443,18 +496,22 @@ sagesla_status sagesla_sla_backward(const sagesla_tensor* q, const sagesla_tenso
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   char* ws = static_cast<char*>(workspace);
   const TensorArg qa = to_arg(q), ka = to_arg(k), va = to_arg(v), da = to_arg(d_out);
+  NvtxRange call_range("sagesla/sla_backward");
   SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.lay.status, 0, sizeof(int32_t), stream));
   // the forward's selection and complement sums (same kernels, so the same block mask)
-  SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
-  SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
-  SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
-  if (!p.quant || !p.pv_fp8) SAGESLA_LAUNCH(launch_pack_bf16(p, qa, ka, va, ws, stream));
-  if (!p.linear_empty) {
-    SAGESLA_LAUNCH(launch_scores(p, ws, stream));
-    SAGESLA_LAUNCH(launch_topk(p, ws, stream));
-    SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
-  } else {
-    SAGESLA_LAUNCH(launch_fill_all_kept(p, ws, stream));
+  {
+    NvtxRange r("sagesla/backward_prologue");
+    SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
+    SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
+    SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
+    if (!p.quant || !p.pv_fp8) SAGESLA_LAUNCH(launch_pack_bf16(p, qa, ka, va, ws, stream));
+    if (!p.linear_empty) {
+      SAGESLA_LAUNCH(launch_scores(p, ws, stream));
+      SAGESLA_LAUNCH(launch_topk(p, ws, stream));
+      SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
+    } else {
+      SAGESLA_LAUNCH(launch_fill_all_kept(p, ws, stream));
+    }
   }
   GradOut g;
   g.dq = dq->data; g.dk = dk->data; g.dv = dv->data;
@@ -466,6 +523,7 @@ sagesla_status sagesla_sla_backward(const sagesla_tensor* q, const sagesla_tenso
     dst[a][2] = gs[a]->stride_n;
   }
   g.dtype = dq->dtype;
+  NvtxRange r("sagesla/backward_gradients");
   SAGESLA_LAUNCH(launch_sla_backward(p, bl, qa, ka, va, da, g, ws, stream));
   return SAGESLA_OK;
 }

@@ -214,7 +214,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& excl) 
 __global__ void __launch_bounds__(kTopkThreads)
 k_topk(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __restrict__ scores,
        int32_t* __restrict__ kept, uint32_t* __restrict__ mask, __nv_bfloat16* __restrict__ amask,
-       int nb_m_pad) {
+       int nb_m_pad, int* status) {
   extern __shared__ uint32_t keys[];          // [nb]
   __shared__ int hist[256];
   __shared__ int warp_tot[8];
@@ -281,6 +281,7 @@ k_topk(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __restr
     int k_excl;
     const int k_tot = block_excl_scan(sel ? 1 : 0, warp_tot, k_excl);
     if (sel && kept_base + k_excl < k) krow[kept_base + k_excl] = j;
+    else if (kChecks && sel) record_error(status, SAGESLA_ERR_BOUNDS);
     if (j < nb_k_pad) arow[j] = (j < nb && !sel) ? one : zero;
     equal_base += eq_tot;
     kept_base += k_tot;
@@ -309,7 +310,7 @@ __device__ __forceinline__ uint32_t warp_sort_desc(uint32_t v, int lane) {
 template <int M>
 __device__ __forceinline__ void topk_row(const uint32_t (&key)[M], int lane, uint32_t* cw, int nb,
                                          int k, int mask_words, int nb_k_pad, int32_t* krow,
-                                         uint32_t* mrow, __nv_bfloat16* arow) {
+                                         uint32_t* mrow, __nv_bfloat16* arow, int* status) {
   const __nv_bfloat16 one = __float2bfloat16_rn(1.f), zero = __float2bfloat16_rn(0.f);
   // Invariants: count(key >= lo) = cnt_lo >= k, count(key > hi) = cnt_above < k. The bracket
   // starts at the row's smallest and largest keys and is split at the midpoint of the two
@@ -360,7 +361,8 @@ __device__ __forceinline__ void topk_row(const uint32_t (&key)[M], int lane, uin
       const int j = 32 * m + lane;
       const bool sel = key[m] >= T;
       const uint32_t sel_bits = __ballot_sync(0xffffffffu, sel);
-      if (sel) krow[kept_base + __popc(sel_bits & below)] = j;
+      if (sel && in_range(kept_base + __popc(sel_bits & below), k, status))
+        krow[kept_base + __popc(sel_bits & below)] = j;
       if (lane == 0 && m < mask_words) mrow[m] = sel_bits;
       if (j < nb_k_pad) arow[j] = (j < nb && !sel) ? one : zero;
       kept_base += __popc(sel_bits);
@@ -376,7 +378,8 @@ __device__ __forceinline__ void topk_row(const uint32_t (&key)[M], int lane, uin
       const uint32_t eq_bits = __ballot_sync(0xffffffffu, eq);
       const bool sel = j < nb && (key[m] > T || (eq && eq_base + __popc(eq_bits & below) < take_equal));
       const uint32_t sel_bits = __ballot_sync(0xffffffffu, sel);
-      if (sel) krow[kept_base + __popc(sel_bits & below)] = j;
+      if (sel && in_range(kept_base + __popc(sel_bits & below), k, status))
+        krow[kept_base + __popc(sel_bits & below)] = j;
       if (lane == 0 && m < mask_words) mrow[m] = sel_bits;
       if (j < nb_k_pad) arow[j] = (j < nb && !sel) ? one : zero;
       eq_base += __popc(eq_bits);
@@ -401,7 +404,7 @@ template <int M>
 __global__ void __launch_bounds__(128, M <= 8 ? 8 : (M <= 16 ? 6 : (M <= 48 ? 4 : 3)))
 k_topk_warp(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __restrict__ scores,
             int32_t* __restrict__ kept, uint32_t* __restrict__ mask,
-            __nv_bfloat16* __restrict__ amask, int nb_m_pad, int64_t n_rows) {
+            __nv_bfloat16* __restrict__ amask, int nb_m_pad, int64_t n_rows, int* status) {
   __shared__ uint32_t cand[4][32];
   __shared__ __align__(16) float rowbuf[4][32 * M];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -442,7 +445,7 @@ k_topk_warp(int nb, int ld, int k, int mask_words, int nb_k_pad, const float* __
     if (row + stride < n_rows) prefetch_row(row + stride);
     topk_row<M>(key, lane, cw, nb, k, mask_words, nb_k_pad,
                 kept + (bh * nb + i) * static_cast<int64_t>(k),
-                mask + (bh * nb + i) * static_cast<int64_t>(mask_words), arow);
+                mask + (bh * nb + i) * static_cast<int64_t>(mask_words), arow, status);
   }
   cp_async_wait_all();
 }
@@ -500,7 +503,8 @@ static cudaError_t launch_topk_warp(const ForwardPlan& p, char* ws, cudaStream_t
       static_cast<int>(p.nb), static_cast<int>(p.scores_ld), static_cast<int>(p.k), static_cast<int>(p.mask_words),
       static_cast<int>(p.nb_k_pad), reinterpret_cast<const float*>(ws + L.scores),
       reinterpret_cast<int32_t*>(ws + L.kept), reinterpret_cast<uint32_t*>(ws + L.mask),
-      reinterpret_cast<__nv_bfloat16*>(ws + L.amask), static_cast<int>(p.nb_m_pad), n_rows);
+      reinterpret_cast<__nv_bfloat16*>(ws + L.amask), static_cast<int>(p.nb_m_pad), n_rows,
+      reinterpret_cast<int*>(ws + L.status));
   return cudaGetLastError();
 }
 
@@ -526,7 +530,8 @@ cudaError_t launch_topk(const ForwardPlan& p, char* ws, cudaStream_t stream) {
       static_cast<int>(p.nb), static_cast<int>(p.scores_ld), static_cast<int>(p.k), static_cast<int>(p.mask_words),
       static_cast<int>(p.nb_k_pad), reinterpret_cast<const float*>(ws + L.scores),
       reinterpret_cast<int32_t*>(ws + L.kept), reinterpret_cast<uint32_t*>(ws + L.mask),
-      reinterpret_cast<__nv_bfloat16*>(ws + L.amask), static_cast<int>(p.nb_m_pad));
+      reinterpret_cast<__nv_bfloat16*>(ws + L.amask), static_cast<int>(p.nb_m_pad),
+      reinterpret_cast<int*>(ws + L.status));
   return cudaGetLastError();
 }
 

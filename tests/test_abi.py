@@ -115,8 +115,9 @@ def test_validation_rejects_bad_arguments_before_launch():
 
 
 def test_status_strings():
-    for s in range(8):
-        assert sba.sagesla_status_string(s)
+    for s in range(10):
+        assert sba.sagesla_status_string(s) != "unknown status"
+        assert s in binding.STATUS_NAMES
     assert sba.sagesla_status_string(99) == "unknown status"
 
 

@@ -207,7 +207,7 @@ sagesla_status check_device() { return require_b200(); }
     if ((call) != cudaSuccess) return SAGESLA_ERR_CUDA; \
   } while (0)
 
-// NVTX range around the launches of one stage (named "sagesla/<stage>"), so that a timeline
+// NVTX range around the launches of one stage (named "sagesla.<stage>"), so that a timeline
 // or an ncu --nvtx filter can find each kernel of a call; a no-op without a tool attached.
 struct NvtxRange {
   explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
@@ -365,20 +365,20 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
   if (checks) SAGESLA_LAUNCH(launch_canary_fill(p, ws, stream));
   // failure-path test: damage the canary after the scores region (host-side injection)
   if (plant == 1) SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.canary[13], 0, 4, stream));
-  NvtxRange call_range("sagesla/forward");
+  NvtxRange call_range("sagesla.forward");
   SAGESLA_LAUNCH(mark(0));
   {
-    NvtxRange r("sagesla/stats");
+    NvtxRange r("sagesla.stats");
     SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
   }
   SAGESLA_LAUNCH(mark(1));
   {
-    NvtxRange r("sagesla/finalize");
+    NvtxRange r("sagesla.finalize");
     SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
   }
   SAGESLA_LAUNCH(mark(2));
   {
-    NvtxRange r("sagesla/quant");
+    NvtxRange r("sagesla.quant");
     SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
     if (!p.quant || !p.pv_fp8) SAGESLA_LAUNCH(launch_pack_bf16(p, qa, ka, va, ws, stream));
   }
@@ -387,12 +387,12 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
   // computed when asked for, and the kept lists and masks only written when asked for.
   const bool want_lists = opt && (opt->kept_idx_out || opt->mask_out);
   if (!p.linear_empty || (opt && opt->scores_out)) {
-    NvtxRange r("sagesla/scores");
+    NvtxRange r("sagesla.scores");
     SAGESLA_LAUNCH(launch_scores(p, ws, stream));
   }
   SAGESLA_LAUNCH(mark(4));
   {
-    NvtxRange r("sagesla/topk");
+    NvtxRange r("sagesla.topk");
     if (!p.linear_empty) SAGESLA_LAUNCH(launch_topk(p, ws, stream));
     else if (want_lists) SAGESLA_LAUNCH(launch_fill_all_kept(p, ws, stream));
   }
@@ -400,7 +400,7 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
   if (plant == 2) SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.lay.kept, 0xFF, 4, stream));
   SAGESLA_LAUNCH(mark(5));
   if (!p.linear_empty) {
-    NvtxRange r("sagesla/complement_gemm");
+    NvtxRange r("sagesla.complement_gemm");
     SAGESLA_LAUNCH(launch_complement_gemm(p, ws, stream));
   }
   SAGESLA_LAUNCH(mark(6));
@@ -410,7 +410,7 @@ sagesla_status sagesla_forward_ex(const sagesla_tensor* q, const sagesla_tensor*
     hooks.skip_tile = opt->debug_skip_tile != 0;
   }
   {
-    NvtxRange r("sagesla/attention");
+    NvtxRange r("sagesla.attention");
     if (p.linear_empty && p.quant && p.pv_fp8)
       SAGESLA_LAUNCH(launch_attention_dense(p, qa, out->data, out->dtype, out->stride_b,
                                             out->stride_h, out->stride_n,
@@ -496,11 +496,11 @@ sagesla_status sagesla_sla_backward(const sagesla_tensor* q, const sagesla_tenso
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   char* ws = static_cast<char*>(workspace);
   const TensorArg qa = to_arg(q), ka = to_arg(k), va = to_arg(v), da = to_arg(d_out);
-  NvtxRange call_range("sagesla/sla_backward");
+  NvtxRange call_range("sagesla.sla_backward");
   SAGESLA_LAUNCH(cudaMemsetAsync(ws + p.lay.status, 0, sizeof(int32_t), stream));
   // the forward's selection and complement sums (same kernels, so the same block mask)
   {
-    NvtxRange r("sagesla/backward_prologue");
+    NvtxRange r("sagesla.backward_prologue");
     SAGESLA_LAUNCH(launch_stats(p, ka, va, ws, stream));
     SAGESLA_LAUNCH(launch_finalize(p, ws, stream));
     SAGESLA_LAUNCH(launch_quant(p, qa, ka, va, ws, stream));
@@ -523,7 +523,7 @@ sagesla_status sagesla_sla_backward(const sagesla_tensor* q, const sagesla_tenso
     dst[a][2] = gs[a]->stride_n;
   }
   g.dtype = dq->dtype;
-  NvtxRange r("sagesla/backward_gradients");
+  NvtxRange r("sagesla.backward_gradients");
   SAGESLA_LAUNCH(launch_sla_backward(p, bl, qa, ka, va, da, g, ws, stream));
   return SAGESLA_OK;
 }

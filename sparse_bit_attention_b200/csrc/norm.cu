@@ -6,12 +6,14 @@
 // fly. Here one pass over a token row reads the bf16 row once and writes the normalized,
 // modulated row (bf16) and/or its INT8 codes with one scale per row.
 //
-// B200 mapping: one 128-thread CTA per row. Each thread holds its chunks of 8 channels
-// (16-byte loads; up to 16 chunks, K <= 16384; the count is a template parameter so that the
-// registers, and with them the occupancy, follow K) in registers, so the row is read from HBM exactly once; the
-// mean / variance (or mean square) and the row's absolute maximum are block reductions
-// (warp shuffles, then 4 warp partials in shared memory). The kernel is bound by HBM
-// bandwidth: per row 2K bytes in, 2K bytes of bf16 and K bytes of codes out.
+// B200 mapping (K <= 8192): one warp per row, four rows per CTA. The warp copies its row into
+// shared memory with cp.async (lane l copies, reads and overwrites only the 16-byte chunks
+// l + 32 i, so no barrier is needed), and every reduction (mean, variance or mean square, the
+// row's absolute maximum) is a warp shuffle: a row never waits for the rest of its CTA. The
+// arithmetic runs on packed f32x2 pairs (each lane rounds like the scalar operation), and
+// each INT8 code is one round-to-nearest-even conversion of the fp32 product. Rows of more
+// than 8192 channels use one 128-thread CTA per row with the row in registers. The kernels
+// are bound by HBM bandwidth: per row 2K bytes in, 2K bytes of bf16 and K bytes of codes out.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -29,6 +31,7 @@ constexpr int kMaxChunks = 16;              // 16 x 8 x 128 = 16384 channels
 struct NormParams {
   const uint16_t* x;
   int64_t x_stride;
+  int64_t M;
   int K, kind;
   float eps;
   const uint16_t *gamma, *beta, *scale, *shift;
@@ -68,6 +71,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
 }
 
+// Rows of more than kWarpRowMaxK channels: one 128-thread CTA per row.
 // kCh = chunks of 8 channels per thread (K <= 8 * 128 * kCh): the row stays in registers.
 template <int kCh>
 __global__ void __launch_bounds__(kNormThreads)
@@ -185,6 +189,179 @@ k_norm_quant(NormParams p) {
   if (t == 0) p.code_scale[row] = a > 0.f ? a / 127.0f : 1.0f;
 }
 
+// One warp per row (K <= 8192), the row staged in shared memory.
+constexpr int kRowsPerCta = 4;
+constexpr int64_t kWarpRowMaxK = 8192;
+__device__ __forceinline__ void cp_async16w(void* smem_dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// packed f32x2 arithmetic (each lane rounds exactly like the scalar operation)
+__device__ __forceinline__ unsigned long long p2(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void u2(unsigned long long v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// the two bf16 values of a word as a packed pair (exact)
+__device__ __forceinline__ unsigned long long bf2(uint32_t w) {
+  return p2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+__global__ void __launch_bounds__(32 * kRowsPerCta)
+k_norm_quant_warp(NormParams p) {
+  extern __shared__ uint4 rows_s[];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + w;
+  if (row >= p.M) return;
+  const int nch = p.K >> 3;
+  uint4* rs = rows_s + static_cast<int64_t>(w) * nch;
+  const uint4* xr = reinterpret_cast<const uint4*>(p.x + row * p.x_stride);
+  for (int c = lane; c < nch; c += 32) cp_async16w(rs + c, xr + c);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  const float inv_k = 1.0f / static_cast<float>(p.K);
+  float mu = 0.f, rstd;
+  if (p.kind == SAGESLA_NO_NORM) {
+    rstd = 1.0f;
+  } else if (p.kind == SAGESLA_LAYER_NORM) {
+    unsigned long long s2 = 0ull;
+    for (int c = lane; c < nch; c += 32) {
+      const uint4 v = rs[c];
+      s2 = add2(add2(s2, bf2(v.x)), add2(bf2(v.y), add2(bf2(v.z), bf2(v.w))));
+    }
+    float sa, sb;
+    u2(s2, sa, sb);
+    mu = warp_sum(sa + sb) * inv_k;
+    const unsigned long long nmu2 = p2(-mu, -mu);
+    unsigned long long q2 = 0ull;
+    for (int c = lane; c < nch; c += 32) {
+      const uint4 v = rs[c];
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const unsigned long long d2 = add2(bf2(wv[e]), nmu2);
+        q2 = fma2(d2, d2, q2);
+      }
+    }
+    float qa, qb;
+    u2(q2, qa, qb);
+    rstd = 1.0f / sqrtf(warp_sum(qa + qb) * inv_k + p.eps);
+  } else {
+    unsigned long long q2 = 0ull;
+    for (int c = lane; c < nch; c += 32) {
+      const uint4 v = rs[c];
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const unsigned long long x2 = bf2(wv[e]);
+        q2 = fma2(x2, x2, q2);
+      }
+    }
+    float qa, qb;
+    u2(q2, qa, qb);
+    rstd = 1.0f / sqrtf(warp_sum(qa + qb) * inv_k + p.eps);
+  }
+  const int64_t b = p.rows_per_sample > 0 ? row / p.rows_per_sample : 0;
+  const uint4* g4 = reinterpret_cast<const uint4*>(p.gamma);
+  const uint4* be4 = reinterpret_cast<const uint4*>(p.beta);
+  const uint4* sc4 = p.scale ? reinterpret_cast<const uint4*>(p.scale + b * p.K) : nullptr;
+  const uint4* sh4 = p.shift ? reinterpret_cast<const uint4*>(p.shift + b * p.K) : nullptr;
+  uint4* yr = p.y ? reinterpret_cast<uint4*>(p.y + row * p.y_stride) : nullptr;
+  float amax = 0.f;
+  for (int c = lane; c < nch; c += 32) {
+    const uint4 xv = rs[c];
+    const uint4 zero4 = make_uint4(0, 0, 0, 0);
+    const uint4 gv = g4 ? __ldg(g4 + c) : zero4, bv = be4 ? __ldg(be4 + c) : zero4;
+    const uint4 sv = sc4 ? __ldg(sc4 + c) : zero4, hv = sh4 ? __ldg(sh4 + c) : zero4;
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w}, sw[4] = {sv.x, sv.y, sv.z, sv.w};
+    const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+    uint32_t packed[4];
+    const unsigned long long nmu2 = p2(-mu, -mu), rstd2 = p2(rstd, rstd), one2 = p2(1.f, 1.f);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      unsigned long long y2 = mul2(add2(bf2(xw[e]), nmu2), rstd2);
+      if (g4) y2 = mul2(y2, bf2(gw[e]));
+      if (be4) y2 = add2(y2, bf2(bw[e]));
+      if (sc4) y2 = mul2(y2, add2(one2, bf2(sw[e])));
+      if (sh4) y2 = add2(y2, bf2(hw[e]));
+      float v[2];
+      u2(y2, v[0], v[1]);
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[0], v[1]);
+      packed[e] = *reinterpret_cast<uint32_t*>(&h2);
+      amax = fmaxf(amax, fmaxf(fabsf(__low2float(h2)), fabsf(__high2float(h2))));
+    }
+    rs[c] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    if (yr) yr[c] = rs[c];
+  }
+  if (!p.codes) return;
+  const float a = warp_max(amax);
+  const float inv = a > 0.f ? 127.0f / a : 0.f;
+  uint2* cr = reinterpret_cast<uint2*>(p.codes + row * p.codes_stride);
+  if (a < INFINITY) {
+    // rne(fl32(y * inv)) by one rounding conversion of the fp32 product; |y * inv| <= 127.5,
+    // so the code needs no clamp
+    const unsigned long long inv2 = p2(inv, inv);
+    for (int c = lane; c < nch; c += 32) {
+      const uint4 v = rs[c];
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t b[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float t0, t1;
+        u2(mul2(bf2(wv[e]), inv2), t0, t1);
+        b[2 * e] = static_cast<uint32_t>(__float2int_rn(t0));
+        b[2 * e + 1] = static_cast<uint32_t>(__float2int_rn(t1));
+      }
+      cr[c] = make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
+                         __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
+    }
+  } else {
+    for (int c = lane; c < nch; c += 32) {
+      float f[8];
+      unpack8(rs[c], f);
+      uint32_t wd[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float q = fminf(fmaxf(rintf(f[e] * inv), -127.f), 127.f);
+        wd[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(q)) & 0xFFu) << (8 * (e & 3));
+      }
+      cr[c] = make_uint2(wd[0], wd[1]);
+    }
+  }
+  if (lane == 0) p.code_scale[row] = a > 0.f ? a / 127.0f : 1.0f;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 bool overlaps(const void* a0, size_t na, const void* b0, size_t nb) {
@@ -245,17 +422,21 @@ extern "C" sagesla_status sagesla_norm_quant(const sagesla_norm_args* a, void* s
   p.codes = a->codes;
   p.codes_stride = a->codes_stride;
   p.code_scale = a->code_scale;
+  p.M = a->M;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->K <= kWarpRowMaxK) {   // one warp per row, rows staged in shared memory
+    const int smem = kRowsPerCta * static_cast<int>(a->K) * 2;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(k_norm_quant_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return SAGESLA_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>((a->M + kRowsPerCta - 1) / kRowsPerCta);
+    k_norm_quant_warp<<<grid, 32 * kRowsPerCta, smem, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SAGESLA_OK : SAGESLA_ERR_CUDA;
+  }
   const int ch = static_cast<int>((a->K / 8 + kNormThreads - 1) / kNormThreads);
   const dim3 grid(static_cast<unsigned>(a->M));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (ch <= 1) k_norm_quant<1><<<grid, kNormThreads, 0, s>>>(p);
-  else if (ch <= 2) k_norm_quant<2><<<grid, kNormThreads, 0, s>>>(p);
-  else if (ch <= 3) k_norm_quant<3><<<grid, kNormThreads, 0, s>>>(p);
-  else if (ch <= 4) k_norm_quant<4><<<grid, kNormThreads, 0, s>>>(p);
-  else if (ch <= 5) k_norm_quant<5><<<grid, kNormThreads, 0, s>>>(p);
-  else if (ch <= 6) k_norm_quant<6><<<grid, kNormThreads, 0, s>>>(p);
-  else if (ch <= 8) k_norm_quant<8><<<grid, kNormThreads, 0, s>>>(p);
-  else if (ch <= 12) k_norm_quant<12><<<grid, kNormThreads, 0, s>>>(p);
+  if (ch <= 12) k_norm_quant<12><<<grid, kNormThreads, 0, s>>>(p);   // K in (8192, 12288]
   else k_norm_quant<kMaxChunks><<<grid, kNormThreads, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? SAGESLA_OK : SAGESLA_ERR_CUDA;
 }

@@ -177,46 +177,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ct
   return true;
 }
 
-// ---------------------------------------------------------------- packed f32x2 arithmetic
-__device__ __forceinline__ unsigned long long pk2(float a, float b) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void up2(unsigned long long v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
-                                                   unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-
-__device__ __forceinline__ float ex2_mufu(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Maximum of this thread's valid scores (eight independent chains).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // Largest of the first `valid` scores as a float: for int32 scores integer maxima in four
 // chains (the conversion to float happens in the exponential loop), for float scores
 // three-input float maxima.
@@ -254,18 +214,18 @@ __device__ __forceinline__ float row_block_fmax(uint32_t (&a)[32], int valid) {
 template <bool kFull, bool kP8, bool kInt>
 __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int valid, float c,
                                               float neg, uint32_t (&pk)[16]) {
-  const unsigned long long c2 = pk2(c, c), neg2 = pk2(neg, neg);
-  unsigned long long acc0 = pk2(0.f, 0.f), acc1 = pk2(0.f, 0.f);
+  const unsigned long long c2 = f2_pack(c, c), neg2 = f2_pack(neg, neg);
+  unsigned long long acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
 #pragma unroll
   for (int q = 0; q < 32; q += 4) {
     float y[4];
 #pragma unroll
     for (int t = 0; t < 4; t += 2) {
       const unsigned long long f2 =
-          kInt ? pk2(__int2float_rn(static_cast<int>(sr[q + t])), __int2float_rn(static_cast<int>(sr[q + t + 1])))
-               : pk2(__uint_as_float(sr[q + t]), __uint_as_float(sr[q + t + 1]));
+          kInt ? f2_pack(__int2float_rn(static_cast<int>(sr[q + t])), __int2float_rn(static_cast<int>(sr[q + t + 1])))
+               : f2_pack(__uint_as_float(sr[q + t]), __uint_as_float(sr[q + t + 1]));
       float x0, x1;
-      up2(fma2(f2, c2, neg2), x0, x1);
+      f2_unpack(f2_fma(f2, c2, neg2), x0, x1);
       y[t] = ex2_mufu(x0);
       y[t + 1] = ex2_mufu(x1);
       if (!kFull) {
@@ -273,8 +233,8 @@ __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int vali
         if (q + t + 1 >= valid) y[t + 1] = 0.f;
       }
     }
-    acc0 = add2(acc0, pk2(y[0], y[1]));
-    acc1 = add2(acc1, pk2(y[2], y[3]));
+    acc0 = f2_add(acc0, f2_pack(y[0], y[1]));
+    acc1 = f2_add(acc1, f2_pack(y[2], y[3]));
     if (kP8) {
       pk[q >> 2] = static_cast<uint32_t>(f32x2_to_e4m3x2(y[0], y[1])) |
                    (static_cast<uint32_t>(f32x2_to_e4m3x2(y[2], y[3])) << 16);
@@ -286,7 +246,7 @@ __device__ __forceinline__ float row_exp_pack(const uint32_t (&sr)[32], int vali
     }
   }
   float a, b;
-  up2(add2(acc0, acc1), a, b);
+  f2_unpack(f2_add(acc0, acc1), a, b);
   return a + b;
 }
 
@@ -614,7 +574,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // rescale this row's O (skipped when no row of the warp moved its max); the two
         // threads of a row each take 64 of the 128 columns
         if (n >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          const unsigned long long a2 = pk2(alpha, alpha);
+          const unsigned long long a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
           for (int cc = 0; cc < 2; ++cc) {
             uint32_t o[32];
@@ -623,7 +583,7 @@ k_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int q = 0; q < 32; q += 2) {
               float x0, x1;
-              up2(mul2(pk2(__uint_as_float(o[q]), __uint_as_float(o[q + 1])), a2), x0, x1);
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[q]), __uint_as_float(o[q + 1])), a2), x0, x1);
               o[q] = __float_as_uint(x0);
               o[q + 1] = __float_as_uint(x1);
             }

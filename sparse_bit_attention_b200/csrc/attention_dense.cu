@@ -117,41 +117,6 @@ __device__ __forceinline__ void tmem_ld32x64(uint32_t taddr, uint32_t (&r)[64]) 
       : "r"(taddr));
 }
 
-__device__ __forceinline__ unsigned long long dpk2(float a, float b) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void dup2(unsigned long long v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long dfma2(unsigned long long a, unsigned long long b,
-                                                    unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ unsigned long long dadd2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ unsigned long long dmul2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ float dex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float dmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // Score column holding natural key u of the block (the K8 rows are key-interleaved).
 __host__ __device__ constexpr int key_column(int u) { return 2 * (u & 31) + (u >> 5); }
 
@@ -178,26 +143,26 @@ __device__ __forceinline__ float dense_row_max(uint32_t (&a)[64], int valid) {
 template <bool kFull>
 __device__ __forceinline__ float dense_row_exp(const uint32_t (&s)[64], int valid, float c,
                                                float neg, uint32_t (&pk)[16], uint8_t* prow) {
-  const unsigned long long c2 = dpk2(c, c), neg2 = dpk2(neg, neg);
-  unsigned long long acc0 = dpk2(0.f, 0.f), acc1 = dpk2(0.f, 0.f);
+  const unsigned long long c2 = f2_pack(c, c), neg2 = f2_pack(neg, neg);
+  unsigned long long acc0 = f2_pack(0.f, 0.f), acc1 = f2_pack(0.f, 0.f);
 #pragma unroll
   for (int u = 0; u < 64; u += 4) {
     float y[4];
 #pragma unroll
     for (int t = 0; t < 4; t += 2) {
-      const unsigned long long f2 = dpk2(__int2float_rn(static_cast<int>(s[key_column(u + t)])),
+      const unsigned long long f2 = f2_pack(__int2float_rn(static_cast<int>(s[key_column(u + t)])),
                                          __int2float_rn(static_cast<int>(s[key_column(u + t + 1)])));
       float x0, x1;
-      dup2(dfma2(f2, c2, neg2), x0, x1);
-      y[t] = dex2(x0);
-      y[t + 1] = dex2(x1);
+      f2_unpack(f2_fma(f2, c2, neg2), x0, x1);
+      y[t] = ex2_mufu(x0);
+      y[t + 1] = ex2_mufu(x1);
       if (!kFull) {
         if (u + t >= valid) y[t] = 0.f;
         if (u + t + 1 >= valid) y[t + 1] = 0.f;
       }
     }
-    acc0 = dadd2(acc0, dpk2(y[0], y[1]));
-    acc1 = dadd2(acc1, dpk2(y[2], y[3]));
+    acc0 = f2_add(acc0, f2_pack(y[0], y[1]));
+    acc1 = f2_add(acc1, f2_pack(y[2], y[3]));
     pk[u >> 2] = static_cast<uint32_t>(f32x2_to_e4m3x2(y[0], y[1])) |
                  (static_cast<uint32_t>(f32x2_to_e4m3x2(y[2], y[3])) << 16);
     if ((u & 15) == 12) {   // keys u - 12 .. u + 3: one 16-key K-chunk of the P row
@@ -207,7 +172,7 @@ __device__ __forceinline__ float dense_row_exp(const uint32_t (&s)[64], int vali
     }
   }
   float a, b;
-  dup2(dadd2(acc0, acc1), a, b);
+  f2_unpack(f2_add(acc0, acc1), a, b);
   return a + b;
 }
 
@@ -347,7 +312,7 @@ k_attention_dense(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float mx = full ? dense_row_max<true>(sr, 64) : dense_row_max<false>(sr, prm.n_last);
       const float cst = cs * skj;
       const float m_new = fmaxf(m_run, mx * cst);
-      const float alpha = dex2(m_run - m_new);               // 0 on the first block
+      const float alpha = ex2_mufu(m_run - m_new);               // 0 on the first block
       const float neg = kLog2_448D - m_new;                  // 2^(S c + neg) = 448 p
       // P tile b is free once P.V(n - 2) has read it (long done by now, as a rule); the P row
       // is stored chunk by chunk inside the exponential loop
@@ -364,7 +329,7 @@ k_attention_dense(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (n >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (!wwait(&ctl->pv_done[b ^ 1], ((n - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const unsigned long long a2 = dpk2(alpha, alpha);
+        const unsigned long long a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
@@ -373,7 +338,7 @@ k_attention_dense(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             float x0, x1;
-            dup2(dmul2(dpk2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), x0, x1);
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), x0, x1);
             o[e] = __float_as_uint(x0);
             o[e + 1] = __float_as_uint(x1);
           }

@@ -207,34 +207,9 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// packed f32x2 arithmetic (each lane rounds exactly like the scalar operation)
-__device__ __forceinline__ unsigned long long p2(float a, float b) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void u2(unsigned long long v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
-                                                   unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-// the two bf16 values of a word as a packed pair (exact)
+// The two bf16 values of a word as a packed pair (exact).
 __device__ __forceinline__ unsigned long long bf2(uint32_t w) {
-  return p2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
 __global__ void __launch_bounds__(32 * kRowsPerCta)
@@ -257,24 +232,24 @@ k_norm_quant_warp(NormParams p) {
     unsigned long long s2 = 0ull;
     for (int c = lane; c < nch; c += 32) {
       const uint4 v = rs[c];
-      s2 = add2(add2(s2, bf2(v.x)), add2(bf2(v.y), add2(bf2(v.z), bf2(v.w))));
+      s2 = f2_add(f2_add(s2, bf2(v.x)), f2_add(bf2(v.y), f2_add(bf2(v.z), bf2(v.w))));
     }
     float sa, sb;
-    u2(s2, sa, sb);
+    f2_unpack(s2, sa, sb);
     mu = warp_sum(sa + sb) * inv_k;
-    const unsigned long long nmu2 = p2(-mu, -mu);
+    const unsigned long long nmu2 = f2_pack(-mu, -mu);
     unsigned long long q2 = 0ull;
     for (int c = lane; c < nch; c += 32) {
       const uint4 v = rs[c];
       const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const unsigned long long d2 = add2(bf2(wv[e]), nmu2);
-        q2 = fma2(d2, d2, q2);
+        const unsigned long long d2 = f2_add(bf2(wv[e]), nmu2);
+        q2 = f2_fma(d2, d2, q2);
       }
     }
     float qa, qb;
-    u2(q2, qa, qb);
+    f2_unpack(q2, qa, qb);
     rstd = 1.0f / sqrtf(warp_sum(qa + qb) * inv_k + p.eps);
   } else {
     unsigned long long q2 = 0ull;
@@ -284,11 +259,11 @@ k_norm_quant_warp(NormParams p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const unsigned long long x2 = bf2(wv[e]);
-        q2 = fma2(x2, x2, q2);
+        q2 = f2_fma(x2, x2, q2);
       }
     }
     float qa, qb;
-    u2(q2, qa, qb);
+    f2_unpack(q2, qa, qb);
     rstd = 1.0f / sqrtf(warp_sum(qa + qb) * inv_k + p.eps);
   }
   const int64_t b = p.rows_per_sample > 0 ? row / p.rows_per_sample : 0;
@@ -307,16 +282,16 @@ k_norm_quant_warp(NormParams p) {
     const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w}, sw[4] = {sv.x, sv.y, sv.z, sv.w};
     const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
     uint32_t packed[4];
-    const unsigned long long nmu2 = p2(-mu, -mu), rstd2 = p2(rstd, rstd), one2 = p2(1.f, 1.f);
+    const unsigned long long nmu2 = f2_pack(-mu, -mu), rstd2 = f2_pack(rstd, rstd), one2 = f2_pack(1.f, 1.f);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      unsigned long long y2 = mul2(add2(bf2(xw[e]), nmu2), rstd2);
-      if (g4) y2 = mul2(y2, bf2(gw[e]));
-      if (be4) y2 = add2(y2, bf2(bw[e]));
-      if (sc4) y2 = mul2(y2, add2(one2, bf2(sw[e])));
-      if (sh4) y2 = add2(y2, bf2(hw[e]));
+      unsigned long long y2 = f2_mul(f2_add(bf2(xw[e]), nmu2), rstd2);
+      if (g4) y2 = f2_mul(y2, bf2(gw[e]));
+      if (be4) y2 = f2_add(y2, bf2(bw[e]));
+      if (sc4) y2 = f2_mul(y2, f2_add(one2, bf2(sw[e])));
+      if (sh4) y2 = f2_add(y2, bf2(hw[e]));
       float v[2];
-      u2(y2, v[0], v[1]);
+      f2_unpack(y2, v[0], v[1]);
       __nv_bfloat162 h2 = __floats2bfloat162_rn(v[0], v[1]);
       packed[e] = *reinterpret_cast<uint32_t*>(&h2);
       amax = fmaxf(amax, fmaxf(fabsf(__low2float(h2)), fabsf(__high2float(h2))));
@@ -331,7 +306,7 @@ k_norm_quant_warp(NormParams p) {
   if (a < INFINITY) {
     // rne(fl32(y * inv)) by one rounding conversion of the fp32 product; |y * inv| <= 127.5,
     // so the code needs no clamp
-    const unsigned long long inv2 = p2(inv, inv);
+    const unsigned long long inv2 = f2_pack(inv, inv);
     for (int c = lane; c < nch; c += 32) {
       const uint4 v = rs[c];
       const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -339,7 +314,7 @@ k_norm_quant_warp(NormParams p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float t0, t1;
-        u2(mul2(bf2(wv[e]), inv2), t0, t1);
+        f2_unpack(f2_mul(bf2(wv[e]), inv2), t0, t1);
         b[2 * e] = static_cast<uint32_t>(__float2int_rn(t0));
         b[2 * e + 1] = static_cast<uint32_t>(__float2int_rn(t1));
       }

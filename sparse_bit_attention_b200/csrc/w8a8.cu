@@ -98,21 +98,6 @@ struct GemmParams {
   int* status;
 };
 
-__device__ __forceinline__ unsigned long long pk2g(float a, float b) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void up2g(unsigned long long v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long fma2g(unsigned long long a, unsigned long long b,
-                                                    unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
 __device__ __forceinline__ void tma_store_2d_g(const CUtensorMap* map, const void* smem_src,
                                                int x, int y) {
   asm volatile(
@@ -196,7 +181,7 @@ k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     for (int kb = 0; kb < nkb; ++kb) {
       const int b = kb & 1;
       const float c = __ldg(wsc + kb);
-      const unsigned long long c2 = pk2g(c, c);
+      const unsigned long long c2 = f2_pack(c, c);
       if (!mbar_wait(&acc_full[b], (kb >> 1) & 1, p.status)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
@@ -206,9 +191,9 @@ k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const unsigned long long f2 = pk2g(__int2float_rn(static_cast<int>(r[e])),
+          const unsigned long long f2 = f2_pack(__int2float_rn(static_cast<int>(r[e])),
                                              __int2float_rn(static_cast<int>(r[e + 1])));
-          acc[16 * cc + (e >> 1)] = fma2g(c2, f2, acc[16 * cc + (e >> 1)]);
+          acc[16 * cc + (e >> 1)] = f2_fma(c2, f2, acc[16 * cc + (e >> 1)]);
         }
       }
       tc_fence_before();
@@ -228,7 +213,7 @@ k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           float v0, v1;
-          up2g(acc[i], v0, v1);
+          f2_unpack(acc[i], v0, v1);
           const int col = 2 * i;
           if (p.bias) {
             const int n = ncol0 + col;
@@ -248,7 +233,7 @@ k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           float v0, v1;
-          up2g(acc[i], v0, v1);
+          f2_unpack(acc[i], v0, v1);
           const int col = 2 * i;
           if (p.bias) {
             const int n = ncol0 + col;

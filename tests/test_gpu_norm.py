@@ -79,8 +79,11 @@ def _x(M, K, seed, spread=1.0, offset=0.0):
     return x.to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("M,K", [(300, 5120), (257, 1536), (64, 8), (33, 16384), (100, 1032)])
+@pytest.mark.parametrize("M,K", [(300, 5120), (257, 1536), (64, 8), (33, 16384), (100, 1032),
+                                 (37, 8192), (29, 8200), (5, 16)])
 def test_layer_norm_with_modulation_and_codes(M, K):
+    """K <= 8192 runs the one-warp-per-row kernel (8192: its largest shared-memory footprint),
+    larger K the one-CTA-per-row kernel (8200: the first width past the boundary)."""
     g = torch.Generator().manual_seed(K)
     x = _x(M, K, M + K, spread=2.0, offset=0.3)
     R = max(1, M // 3)

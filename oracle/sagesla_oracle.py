@@ -258,7 +258,7 @@ def e4m3_ambiguity(y: np.ndarray, rel) -> np.ndarray:
 
 
 def online_softmax_p8(blocks, exp_rel_err: float = EXP2_REL_ERR):
-    """The online loop of the sparse branch with the P tile in e4m3 (SPEC section 6).
+    """The online loop of the sparse branch with the P tile in e4m3.
 
     ``blocks``: the kept key blocks in ascending order, each a pair (s, v8) of the logits
     s [nq, nk] (float64, natural-log units) and the decoded V codes v8 [nk, D] of its keys.
@@ -290,7 +290,7 @@ def online_softmax_p8(blocks, exp_rel_err: float = EXP2_REL_ERR):
 
 
 def online_softmax_real(blocks):
-    """The online loop with real P and V (SPEC sections 9 and 9.1): for each kept block in
+    """The online loop with real P and V (the 16-bit operand modes): for each kept block in
     ascending order, with logits s [nq, nk] and value rows v [nk, D]: m' = max(m, rowmax s),
     alpha = e^{m - m'}, p = e^{s - m'}, l <- alpha l + sum p, o <- alpha o + p . v. Returns
     (o, l, mag) with mag the same recurrence over p . |v| (so that mag / l is the output of
@@ -312,9 +312,9 @@ def online_softmax_real(blocks):
     return o, l, mag
 
 
-# Tolerance of the sparse branch when P (and V) enter the P.V product in bf16 (SPEC section
-# 10): P rounded to bf16 (relative 2^-9 per term), fp32 accumulation; twice the unit
-# roundoff times the size of the terms.
+# Tolerance of the sparse branch when P (and V) enter the P.V product in bf16: P rounded to
+# bf16 (relative 2^-9 per term), fp32 accumulation; twice the unit roundoff times the size of
+# the terms.
 BF16_PV_REL = 2.0 ** -8
 
 
@@ -403,8 +403,8 @@ def sparse_block_row(prep: HeadPrep, i: int, q, k, v, quant: bool = True,
     """Sparse branch for the real query tokens of block i: online softmax over kept(i) in
     ascending order, running max updated per key block (no lazy rescale).
 
-    ``quant``: logits from the INT8 codes (SPEC 4, 6) or from the real Q, K (SPEC 9).
-    ``pv_fp8`` (with ``quant``): P and V in e4m3 (SPEC 6), or real P and V (SPEC 9.1).
+    ``quant``: logits from the INT8 codes of the smoothed, block-scaled Q and K, or from the
+    real Q and K. ``pv_fp8`` (with ``quant``): P and V as e4m3 codes, or real P and V.
     With ``return_ambiguity`` also returns, per output element, the allowance a kernel needs:
     ambiguous P codes and the window of the row sum (e4m3 P.V), or the bf16 rounding of P
     (real P.V: BF16_PV_REL times the output of the same weights applied to |v|)."""

@@ -3,7 +3,7 @@
 TEST INFRASTRUCTURE ONLY. Only the tests and the CPU legs of ``bench.py`` may import this
 module; the product path never calls it, and it shares no code with the CUDA path.
 
-What it computes (float64, plain numpy; SPEC §13): the layer fine-tuned is SLA without the
+What it computes (float64, plain numpy): the layer fine-tuned is SLA without the
 8-bit quantization (news.qq.com TurboDiffusion article, section 从训练到部署: full attention
 is replaced by SLA and fine-tuned; SageSLA, SLA plus low-bit quantization, replaces it only
 at inference). The block selection of the forward is held fixed. For one (b, h) with kept
@@ -21,7 +21,8 @@ lists ``kept[i]`` and the output gradient dO:
   db = dH_j[:, :d] v_u + dH_j[:, d], dk_u += b * (db - b . db), dv_u += dH_j[:, :d]^T b.
 
 Each gradient comes with its magnitude: the same sums with every term taken in absolute
-value, which scales the tolerance of the GPU comparison (SPEC §13).
+value, which scales the tolerance of the GPU comparison (2^-5 of it, plus 1e-6 of the
+largest gradient).
 
 Pins: ``tests/test_sla_backward_oracle_pins.py`` (central finite differences of the forward,
 float64 autograd of an independent torch forward, dense attention gradients from torch's

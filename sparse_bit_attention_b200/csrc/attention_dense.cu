@@ -1,4 +1,4 @@
-// Dense mode of the SageSLA forward (every key block kept): the sparse branch of SPEC section 6
+// Dense mode of the SageSLA forward (every key block kept): the sparse branch's online softmax
 // over all key blocks in ascending order, INT8 Q.K^T and FP8 P.V on tcgen05 at M=128.
 //
 // Method: news.qq.com TurboDiffusion article, section 第一把钥匙 — SageAttention's 8-bit

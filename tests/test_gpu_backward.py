@@ -1,7 +1,7 @@
 """GPU parity of the SLA backward (through the C ABI) against the float64 CPU oracle
 (oracle/sla_backward_oracle.py), element by element, on the GPU's own block selection (read
 back from the workspace; the selection itself is checked against the oracle's Top-K by the
-forward's parity tests). Tolerance (SPEC §13): |g - ref| <= 2^-5 * magnitude + 1e-6 *
+forward's parity tests). Tolerance: |g - ref| <= 2^-5 * magnitude + 1e-6 *
 max|ref|, the magnitude being the oracle's sum of absolute terms of the element."""
 import numpy as np
 import pytest

@@ -362,7 +362,7 @@ def test_e4m3_ambiguity_bound():
 
 
 def test_int8_logits_with_real_pv_equal_block_masked_attention_of_dequantized_q_k():
-    """SPEC 9.1 (INT8 Q.K^T, real P and V): the sparse branch equals softmax attention over
+    """INT8 Q.K^T with real P and V: the sparse branch equals softmax attention over
     the kept blocks with the dequantized Q8 * sq and K8 * sk (the logits are the same numbers)
     and the raw V, through the library routine."""
     n = 300

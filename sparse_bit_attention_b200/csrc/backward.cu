@@ -302,6 +302,16 @@ struct BwdParams {
 // a two-stage ring, refilling a stage as soon as the MMAs of the block in it have completed.
 // Everything is ordered by mbarriers (no block-wide barrier in the loop); every wait is
 // bounded, and a timed-out wait ends every role's loop through abort_flag.
+// Wait of the role-warp kernels: a completed phase passes at once; otherwise the CTA's abort
+// flag is read (set: give up at once), then the bounded wait. Trying the barrier first keeps
+// the shared-memory read of the flag off the path of waits that need not block.
+__device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatile int& abort_flag,
+                                         int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  if (abort_flag) return false;
+  return mbar_wait(bar, parity, status);
+}
+
 constexpr int kLseThreads = 224;
 
 __global__ void __launch_bounds__(kLseThreads, 2)
@@ -353,7 +363,7 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       for (int m = 0; m < U; ++m) {
         const int b = m & 1;
         // stage b held block m - 2: its S and dP MMAs must have completed
-        if (m >= 2 && (abort_flag || !mbar_wait(&s_done[b], ((m - 2) >> 1) & 1, prm.status))) {
+        if (m >= 2 && !bwd_wait(&s_done[b], ((m - 2) >> 1) & 1, abort_flag, prm.status)) {
           ok = false;
           break;
         }
@@ -382,8 +392,8 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       for (int n = 0; n < U && ok; ++n) {
         const int b = n & 1;
         // buffer b held block n - 2: the softmax warps must have read it
-        if (n >= 2) ok = !abort_flag && mbar_wait(&s_free[b], ((n - 2) >> 1) & 1, prm.status);
-        ok = ok && !abort_flag && mbar_wait(&full[b], (n >> 1) & 1, prm.status);
+        if (n >= 2) ok = bwd_wait(&s_free[b], ((n - 2) >> 1) & 1, abort_flag, prm.status);
+        ok = ok && bwd_wait(&full[b], (n >> 1) & 1, abort_flag, prm.status);
         if (!ok) break;
         tc_fence_after();
         const uint32_t bsm = stage + b * kTile;
@@ -404,7 +414,7 @@ k_bwd_lse(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     float m_run = -INFINITY, l_part = 0.f, d_part = 0.f;
     for (int n = 0; n < U; ++n) {
       const int st = n & 1;
-      ok = !abort_flag && mbar_wait(&s_done[st], (n >> 1) & 1, prm.status);
+      ok = bwd_wait(&s_done[st], (n >> 1) & 1, abort_flag, prm.status);
       ok = __all_sync(0xffffffffu, ok) != 0;      // the warp leaves together
       if (!ok) break;
       tc_fence_after();
@@ -554,7 +564,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       for (int m = 0; m < U; ++m) {
         const int b = m & 1;
         // stage b held block m - 2: its dQ (after its S and dP) must have completed
-        if (m >= 2 && (abort_flag || !mbar_wait(&dq_done[b], ((m - 2) >> 1) & 1, prm.status))) {
+        if (m >= 2 && !bwd_wait(&dq_done[b], ((m - 2) >> 1) & 1, abort_flag, prm.status)) {
           ok = false;
           break;
         }
@@ -574,7 +584,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     // ------------------------------------------------ dQ issuer
     if (lane == 0) {
       for (int n = 0; n < U; ++n) {
-        ok = !abort_flag && mbar_wait(&ds_full[n & 1], (n >> 1) & 1, prm.status);
+        ok = bwd_wait(&ds_full[n & 1], (n >> 1) & 1, abort_flag, prm.status);
         if (!ok) break;
         tc_fence_after();
         const uint32_t sa = smem_u32(s_t + (n & 1) * kPTile);
@@ -598,8 +608,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       for (int n = 0; n < U && ok; ++n) {
         const int b = n & 1;
         // buffer b held block n - 2: the softmax warps must have read it
-        if (n >= 2) ok = !abort_flag && mbar_wait(&s_free[b], ((n - 2) >> 1) & 1, prm.status);
-        ok = ok && !abort_flag && mbar_wait(&kv_full[b], (n >> 1) & 1, prm.status);
+        if (n >= 2) ok = bwd_wait(&s_free[b], ((n - 2) >> 1) & 1, abort_flag, prm.status);
+        ok = ok && bwd_wait(&kv_full[b], (n >> 1) & 1, abort_flag, prm.status);
         if (!ok) break;
         tc_fence_after();
         const uint32_t bsm = stage + b * kTile;
@@ -623,7 +633,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     const float c2 = kScale * kLog2e;
     for (int n = 0; n < U; ++n) {
       const int b = n & 1;
-      ok = !abort_flag && mbar_wait(&s_done[b], (n >> 1) & 1, prm.status);
+      ok = bwd_wait(&s_done[b], (n >> 1) & 1, abort_flag, prm.status);
       ok = __all_sync(0xffffffffu, ok) != 0;      // the warp leaves together
       if (!ok) break;
       tc_fence_after();
@@ -642,7 +652,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       }
       // dQ of block n - 2 has read dS tile b
       if (n >= 2) {
-        ok = !abort_flag && mbar_wait(&dq_done[b], ((n - 2) >> 1) & 1, prm.status);
+        ok = bwd_wait(&dq_done[b], ((n - 2) >> 1) & 1, abort_flag, prm.status);
         ok = __all_sync(0xffffffffu, ok) != 0;
         if (!ok) break;
       }
@@ -756,7 +766,7 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         for (int m = 0; m < T; ++m) {
           const int b = m & 1;
           // stage b held query block m - 2: its dV / dK MMAs must have completed
-          if (m >= 2 && (abort_flag || !mbar_wait(&acc_done[b], ((m - 2) >> 1) & 1, prm.status))) {
+          if (m >= 2 && !bwd_wait(&acc_done[b], ((m - 2) >> 1) & 1, abort_flag, prm.status)) {
             ok = false;
             break;
           }
@@ -777,7 +787,7 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       if (lane == 0) {
         const uint32_t pa = smem_u32(p_t), sa = smem_u32(s_t);
         for (int n = 0; n < T; ++n) {
-          ok = !abort_flag && mbar_wait(&p_full, n & 1, prm.status);
+          ok = bwd_wait(&p_full, n & 1, abort_flag, prm.status);
           if (!ok) break;
           tc_fence_after();
           const int b = n & 1;
@@ -805,8 +815,8 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         for (int n = 0; n < T && ok; ++n) {
           const int b = n & 1;
           // buffer b held query block n - 2: the softmax warps must have read it
-          if (n >= 2) ok = !abort_flag && mbar_wait(&s_free[b], ((n - 2) >> 1) & 1, prm.status);
-          ok = ok && !abort_flag && mbar_wait(&qo_full[b], (n >> 1) & 1, prm.status);
+          if (n >= 2) ok = bwd_wait(&s_free[b], ((n - 2) >> 1) & 1, abort_flag, prm.status);
+          ok = ok && bwd_wait(&qo_full[b], (n >> 1) & 1, abort_flag, prm.status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t bsm = stage + b * kTile;
@@ -840,7 +850,7 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         lq[4 * u] = a.x; lq[4 * u + 1] = a.y; lq[4 * u + 2] = a.z; lq[4 * u + 3] = a.w;
         dq_[4 * u] = c.x; dq_[4 * u + 1] = c.y; dq_[4 * u + 2] = c.z; dq_[4 * u + 3] = c.w;
       }
-      ok = !abort_flag && mbar_wait(&s_done[b], (n >> 1) & 1, prm.status);
+      ok = bwd_wait(&s_done[b], (n >> 1) & 1, abort_flag, prm.status);
       ok = __all_sync(0xffffffffu, ok) != 0;      // the warp leaves together
       if (!ok) break;
       tc_fence_after();
@@ -859,7 +869,7 @@ k_bwd_dkv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
       }
       // dV / dK of query block n - 1 have read the P^T and dS^T tiles
       if (n >= 1) {
-        ok = !abort_flag && mbar_wait(&acc_done[(n - 1) & 1], ((n - 1) >> 1) & 1, prm.status);
+        ok = bwd_wait(&acc_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, prm.status);
         ok = __all_sync(0xffffffffu, ok) != 0;
         if (!ok) break;
       }

@@ -70,7 +70,7 @@ def parse_args():
                          "14B-720P, locality at three ratios)")
     ap.add_argument("--sweep", action="store_true",
                     help="Top-K ratio sweep and dense BF16 comparison, one JSON line per point")
-    ap.add_argument("--kernel-case", choices=["norm", "w8a8", "bwd"], default=None,
+    ap.add_argument("--kernel-case", choices=["norm", "w8a8", "bwd", "dense"], default=None,
                     help="run a small case of one next-row kernel a few times (for ncu captures)")
     args = ap.parse_args()
     globals()["WORKLOAD"] = args.workload
@@ -735,6 +735,17 @@ def run_kernel_case(args):
         for _ in range(3):
             sba.sagesla_norm_quant(x, sba.SAGESLA_LAYER_NORM, 1e-6, None, None, scale, shift,
                                    rows_per_sample=M, want_codes=True)
+    elif args.kernel_case == "dense":
+        # dense mode (Top-K ratio 1: the M=128 dense kernel) on the Wan2.1-1.3B-480P shape
+        from sparse_bit_attention_b200 import inputs
+        q, k, v = (x.cuda() for x in inputs.make_qkv("wan21_1p3b_480p"))
+        B, H, N, D = q.shape
+        ws = sba.alloc_workspace(sba.sagesla_workspace_size(B, H, N, D, 1.0))
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+        for _ in range(2):
+            sba.sagesla_forward(q, k, v, 1.0, out=out, workspace=ws)
+        if sba.sagesla_stream_status(None, ws) != 0:
+            raise RuntimeError("device status after the dense-mode forward")
     elif args.kernel_case == "bwd":
         # SLA backward on the Wan2.1-1.3B-480P attention shape (B1 H12 N32760, ratio 0.1)
         from sparse_bit_attention_b200 import inputs
